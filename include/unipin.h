@@ -1,0 +1,152 @@
+/*
+ * unipin.h - C ABI of the B200 (sm_100a) library for UniPinRec's cross-stage
+ * KV reuse: the M-FALCON masked prefill attention, the write of the past K/V
+ * into a preallocated cache pool, and the rank decode that scores candidate
+ * tokens against a slot of that pool.
+ *
+ * Sources (the method is described in prose only):
+ *   [notes]  UniPinRec reproduction notes (slinene.github.io, ai-papers-daily,
+ *            "unipinrec-unified-retrieval-ranking-masked-action-kv-share"),
+ *            sub-module details §3 "attention mask", §6 "serving:
+ *            cross-process KV sharing".
+ *   [review] UniPinRec paper review (liuzhao09.github.io,
+ *            "pinterest-unipinrec"), §2.2 joint objective, §2.4 co-serving,
+ *            Faiss and the cross-stage KV cache.
+ *
+ * Conventions shared by every call:
+ *   - Tensors are bfloat16, row-major, in device memory owned by the caller.
+ *     Packed token tensors are [T, H, D]: token t, head h, element d at
+ *     ((t * H + h) * D + d).  Every tensor pointer must be 16-byte aligned.
+ *   - Ragged batches use int32 offset arrays in device memory: cu_seqlens of
+ *     length B+1 (segment b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1).
+ *   - Supported head dims: D in {32, 64, 128}.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = the
+ *     legacy default stream), does no host synchronisation, allocates
+ *     nothing and keeps no pointer after it returns.  The first call of each
+ *     entry point on a device sets kernel attributes and resolves a driver
+ *     entry point, so make one call before capturing a CUDA graph.
+ *   - Host-checkable errors come back as the return value and launch nothing.
+ *     Errors the kernels find in device arrays (a length or slot id out of
+ *     range) and bounded waits that ran out of time are stored into
+ *     *dev_status (device int, may be NULL; 0 = no error, the first error
+ *     wins) and the affected blocks exit without writing; a kernel never
+ *     traps.  The caller clears *dev_status and reads it back when it likes.
+ */
+#ifndef UNIPIN_H
+#define UNIPIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    UNIPIN_OK = 0,
+    UNIPIN_ERR_INVALID_ARG = -1,    /* null pointer, negative size, inconsistent shapes */
+    UNIPIN_ERR_UNSUPPORTED = -2,    /* D not in {32, 64, 128}; device is not sm_100 */
+    UNIPIN_ERR_MISALIGNED = -3,     /* a tensor pointer is not 16-byte aligned */
+    UNIPIN_ERR_OUT_OF_RANGE = -4,   /* slot >= S, n > n_cap, layer >= L, a length > the stated max */
+    UNIPIN_ERR_CUDA = -5,           /* a CUDA runtime / driver call failed */
+    UNIPIN_ERR_DEVICE_TIMEOUT = -6  /* a bounded device wait expired (reported via dev_status) */
+} unipin_status;
+
+/*
+ * The KV cache pool ([review] §2.4, [notes] §6): one preallocated tensor of
+ * shape [L, S, H, n_cap, D] for K and one for V (layer, slot, KV head,
+ * history position, head dim), bfloat16, row-major, caller-owned device
+ * memory.  Row (l, s, h, j) starts at element (((l * S + s) * H + h) * n_cap + j) * D.
+ * A slot holds one user's past K/V; rows j >= that user's n are never read.
+ */
+typedef struct {
+    void* k;
+    void* v;
+    int L, S, H, n_cap, D;
+} unipin_kvpool;
+
+/*
+ * Masked prefill attention over B packed segments [n_b past || k_b candidates]
+ * ([notes] §3, [review] §2.2):
+ *   past row i < n_b      attends to keys j <= i (causal, diagonal included);
+ *   candidate row i >= n_b attends to every past key j < n_b and to itself,
+ *                          never to another candidate.
+ *   O_i = softmax_j(scale * q_i . k_j) v_j over the allowed keys, computed with
+ *   fp32 scores, fp32 online softmax and fp32 accumulation (P rounded to bf16
+ *   for the P.V product).
+ *
+ *   q, k, v        [T, H, D] bf16, T = total_tokens = cu_seqlens[B]
+ *   out            [T, H, D], fp32 if out_fp32 != 0 else bf16 (round to nearest even)
+ *   cu_seqlens     device int32 [B+1]; past_lens device int32 [B], 0 <= n_b <= len_b
+ *   max_seqlen     host int >= every len_b (sizes the grid; a longer segment is a device error)
+ *   scale          softmax scale, normally 1/sqrt(D)
+ *   pool, slot_ids optional (pool == NULL: no pool write).  When given, the
+ *                  past K/V of segment b is also written to pool rows
+ *                  [layer, slot_ids[b], h, 0:n_b) exactly as unipin_kvpool_write does.
+ * Returns UNIPIN_OK or a negative unipin_status.
+ */
+int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                               const int* cu_seqlens, const int* past_lens, int B, int H, int D,
+                               int max_seqlen, int total_tokens, float scale, const unipin_kvpool* pool,
+                               const int* slot_ids, int layer, int* dev_status, void* stream);
+
+/*
+ * Pool write ([review] §2.4: retrieval writes the past K/V of every layer
+ * into the shared pool; [notes] §6: pool [L, S, H, n, D], slot reuse):
+ *   pool.k[layer, slot_ids[b], h, j, :] = k[cu_seqlens[b] + j, h, :]   for j < past_lens[b]
+ * and the same for v.  A byte copy (bit-exact); nothing else in the pool is
+ * touched.  Slot ids within one call must be distinct (a repeated id leaves
+ * that slot holding one of the writers' rows, unspecified which).
+ *   k, v           [T, H, D] bf16 with T = cu_seqlens[B]
+ *   max_past       host int >= every past_lens[b] (sizes the grid)
+ *   total_tokens   T, the number of rows of k and v (rows read are checked against it)
+ */
+int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, const void* v,
+                        const int* cu_seqlens, const int* past_lens, const int* slot_ids, int B, int max_past,
+                        int total_tokens, int* dev_status, void* stream);
+
+/*
+ * Rank decode ([review] §2.4: the ranking node forwards only the candidate
+ * tokens and lets them attend to the cached history K/V; [notes] §6: read
+ * the request's slot, cost O(nk)).  Request r has k_r candidates (rows
+ * cu_seqlens_c[r] .. cu_seqlens_c[r+1]-1 of q_c/k_c/v_c) and n_r = past_lens[r]
+ * cached rows in slot slot_ids[r] of `pool` at `layer`.  Candidate c attends
+ * to pool rows 0..n_r-1 of that slot and to itself (its own k_c, v_c) - the
+ * same mask as the candidate rows of the prefill, so it returns what the
+ * prefill returns for those rows.
+ *   q_c, k_c, v_c  [T_c, H, D] bf16, T_c = total_cand = cu_seqlens_c[R]
+ *   out            [T_c, H, D], fp32 if out_fp32 else bf16
+ *   max_k          host int >= every k_r (sizes the grid)
+ *   workspace      optional device scratch (NULL allowed): with at least
+ *                  unipin_rank_decode_workspace_size(...) bytes the pool sweep
+ *                  of each request is split over several thread blocks
+ *                  (split-n) and merged by a second kernel; without it one
+ *                  block sweeps all n_r rows.  The result is the same either way
+ *                  up to fp32 rounding.
+ */
+int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
+                            const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H,
+                            int D, int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer,
+                            void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/* Bytes of workspace that let unipin_rank_decode_attn split the pool sweep
+ * for these sizes (n_cap = the pool's rows per slot); 0 if it would not split. */
+size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap);
+
+/* Human-readable name of a unipin_status value. */
+const char* unipin_status_string(int status);
+
+/*
+ * Self-test of the bounded device wait used by every kernel: launches one
+ * warp that waits on a barrier nothing ever completes, with a limit of
+ * limit_us microseconds.  The wait gives up, stores UNIPIN_ERR_DEVICE_TIMEOUT
+ * into *dev_status and the kernel returns normally.  Exists so tests can
+ * check the timeout path without any kernel hanging.
+ */
+int unipin_selftest_bounded_wait(int* dev_status, unsigned int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UNIPIN_H */

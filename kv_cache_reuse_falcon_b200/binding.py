@@ -1,0 +1,199 @@
+"""Python binding of the C ABI in ``include/unipin.h``.
+
+Argument marshalling only: torch tensors supply device pointers and the
+current CUDA stream; every step of the computation runs in the CUDA kernels of
+``libunipin.so``.  If the library is missing or fails to load, importing this
+module raises: there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libunipin.so")
+
+UNIPIN_OK = 0
+STATUS_NAMES = {
+    0: "UNIPIN_OK",
+    -1: "UNIPIN_ERR_INVALID_ARG",
+    -2: "UNIPIN_ERR_UNSUPPORTED",
+    -3: "UNIPIN_ERR_MISALIGNED",
+    -4: "UNIPIN_ERR_OUT_OF_RANGE",
+    -5: "UNIPIN_ERR_CUDA",
+    -6: "UNIPIN_ERR_DEVICE_TIMEOUT",
+}
+
+EXPORTS = (
+    "unipin_masked_prefill_attn",
+    "unipin_kvpool_write",
+    "unipin_rank_decode_attn",
+    "unipin_rank_decode_workspace_size",
+    "unipin_status_string",
+    "unipin_selftest_bounded_wait",
+)
+
+
+class UnipinError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (where, STATUS_NAMES.get(code, "?"), code))
+
+
+class KVPool(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("L", ctypes.c_int), ("S", ctypes.c_int),
+                ("H", ctypes.c_int), ("n_cap", ctypes.c_int), ("D", ctypes.c_int)]
+
+
+def _load(path: str = _LIB_PATH):
+    if not os.path.exists(path):
+        raise ImportError("libunipin.so not built (run __graft_entry__.build() or "
+                          "python kv_cache_reuse_falcon_b200/build.py): %s" % path)
+    lib = ctypes.CDLL(path)
+    P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, F, P, P, I, P, P]
+    lib.unipin_masked_prefill_attn.restype = I
+    lib.unipin_kvpool_write.argtypes = [P, I, P, P, P, P, P, I, I, I, P, P]
+    lib.unipin_kvpool_write.restype = I
+    lib.unipin_rank_decode_attn.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, F, P, I, P, SZ, P, P]
+    lib.unipin_rank_decode_attn.restype = I
+    lib.unipin_rank_decode_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.unipin_rank_decode_workspace_size.restype = SZ
+    lib.unipin_status_string.argtypes = [I]
+    lib.unipin_status_string.restype = ctypes.c_char_p
+    lib.unipin_selftest_bounded_wait.argtypes = [P, ctypes.c_uint, P]
+    lib.unipin_selftest_bounded_wait.restype = I
+    return lib
+
+
+LIB = _load()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != UNIPIN_OK:
+        raise UnipinError(rc, where)
+
+
+def _tokens(t: torch.Tensor, name: str, D: Optional[int] = None):
+    if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError("%s must be a contiguous CUDA bfloat16 tensor [T, H, D]" % name)
+    if D is not None and t.shape[2] != D:
+        raise ValueError("%s has head dim %d, expected %d" % (name, t.shape[2], D))
+
+
+def _index(t: torch.Tensor, name: str, n: int):
+    if t.dtype != torch.int32 or t.dim() != 1 or t.shape[0] != n or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError("%s must be a contiguous CUDA int32 tensor of length %d" % (name, n))
+
+
+def _pool(pool_k: torch.Tensor, pool_v: torch.Tensor) -> KVPool:
+    for name, t in (("pool_k", pool_k), ("pool_v", pool_v)):
+        if t.dtype != torch.bfloat16 or t.dim() != 5 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError("%s must be a contiguous CUDA bfloat16 tensor [L, S, H, n_cap, D]" % name)
+    if pool_k.shape != pool_v.shape:
+        raise ValueError("pool_k and pool_v differ in shape")
+    L, S, H, n_cap, D = pool_k.shape
+    return KVPool(pool_k.data_ptr(), pool_v.data_ptr(), L, S, H, n_cap, D)
+
+
+def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=None, out_fp32: bool = True,
+                        scale: Optional[float] = None, pool_k=None, pool_v=None, slot_ids=None, layer: int = 0,
+                        dev_status=None, stream=None):
+    """M-FALCON masked prefill; optionally also writes the past K/V into pool slots."""
+    _tokens(q, "q")
+    T, H, D = q.shape
+    _tokens(k, "k", D)
+    _tokens(v, "v", D)
+    B = past_lens.shape[0]
+    _index(cu_seqlens, "cu_seqlens", B + 1)
+    _index(past_lens, "past_lens", B)
+    if out is None:
+        out = torch.empty((T, H, D), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    elif out.dtype != (torch.float32 if out_fp32 else torch.bfloat16) or out.shape != q.shape or not out.is_contiguous():
+        raise ValueError("out has the wrong dtype or shape")
+    pool = None
+    if pool_k is not None:
+        pool = _pool(pool_k, pool_v)
+        _index(slot_ids, "slot_ids", B)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    rc = LIB.unipin_masked_prefill_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(bool(out_fp32)),
+                                        _ptr(cu_seqlens), _ptr(past_lens), B, H, D, int(max_seqlen), T, scale,
+                                        ctypes.byref(pool) if pool is not None else None,
+                                        _ptr(slot_ids) if pool is not None else None, int(layer),
+                                        _ptr(dev_status), _stream(stream))
+    _check(rc, "unipin_masked_prefill_attn")
+    return out
+
+
+def kvpool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids, max_past: int,
+                 dev_status=None, stream=None):
+    """Byte copy of each segment's past K/V rows into its pool slot at `layer`."""
+    pool = _pool(pool_k, pool_v)
+    _tokens(k, "k", pool.D)
+    _tokens(v, "v", pool.D)
+    B = past_lens.shape[0]
+    _index(cu_seqlens, "cu_seqlens", B + 1)
+    _index(past_lens, "past_lens", B)
+    _index(slot_ids, "slot_ids", B)
+    rc = LIB.unipin_kvpool_write(ctypes.byref(pool), int(layer), _ptr(k), _ptr(v), _ptr(cu_seqlens),
+                                 _ptr(past_lens), _ptr(slot_ids), B, int(max_past), int(k.shape[0]),
+                                 _ptr(dev_status), _stream(stream))
+    _check(rc, "unipin_kvpool_write")
+
+
+def rank_decode_workspace_size(R: int, H: int, D: int, max_k: int, total_cand: int, n_cap: int) -> int:
+    return int(LIB.unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand, n_cap))
+
+
+def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, pool_v, layer: int, max_k: int,
+                     out=None, out_fp32: bool = True, scale: Optional[float] = None, workspace=None,
+                     dev_status=None, stream=None):
+    """Candidates attend to their slot's cached past rows plus themselves."""
+    _tokens(q_c, "q_c")
+    T, H, D = q_c.shape
+    _tokens(k_c, "k_c", D)
+    _tokens(v_c, "v_c", D)
+    pool = _pool(pool_k, pool_v)
+    R = past_lens.shape[0]
+    _index(cu_seqlens_c, "cu_seqlens_c", R + 1)
+    _index(slot_ids, "slot_ids", R)
+    _index(past_lens, "past_lens", R)
+    if out is None:
+        out = torch.empty((T, H, D), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q_c.device)
+    elif out.dtype != (torch.float32 if out_fp32 else torch.bfloat16) or out.shape != q_c.shape or not out.is_contiguous():
+        raise ValueError("out has the wrong dtype or shape")
+    ws_bytes = 0
+    if workspace is not None:
+        if not workspace.is_cuda or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous CUDA tensor")
+        ws_bytes = workspace.numel() * workspace.element_size()
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    rc = LIB.unipin_rank_decode_attn(_ptr(q_c), _ptr(k_c), _ptr(v_c), _ptr(out), int(bool(out_fp32)),
+                                     _ptr(cu_seqlens_c), _ptr(slot_ids), _ptr(past_lens), R, H, D, int(max_k), T,
+                                     scale, ctypes.byref(pool), int(layer), _ptr(workspace), ws_bytes,
+                                     _ptr(dev_status), _stream(stream))
+    _check(rc, "unipin_rank_decode_attn")
+    return out
+
+
+def selftest_bounded_wait(dev_status, limit_us: int, stream=None):
+    rc = LIB.unipin_selftest_bounded_wait(_ptr(dev_status), int(limit_us), _stream(stream))
+    _check(rc, "unipin_selftest_bounded_wait")
+
+
+def status_string(code: int) -> str:
+    return LIB.unipin_status_string(int(code)).decode()

@@ -1,0 +1,388 @@
+// Host side of the C ABI declared in include/unipin.h: argument checks,
+// TMA tensor-map construction, grid sizing and kernel launches.  Everything
+// here is asynchronous on the caller's stream; nothing allocates.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "unipin.h"
+#include "sm100_ptx.cuh"
+#include "attn_sm100.cuh"
+#include "kvpool_sm100.cuh"
+
+using namespace unipin;
+
+namespace {
+
+constexpr int kNumSmsHint = 148;   // B200
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_init_mutex;
+bool g_device_ready[kMaxDevices] = {};
+
+unsigned long long wait_limit_ns()
+{
+    static unsigned long long v = [] {
+        const char* s = std::getenv("UNIPIN_WAIT_LIMIT_MS");
+        long long ms = s ? std::atoll(s) : 0;
+        if (ms <= 0) ms = 2000;
+        return (unsigned long long)ms * 1000000ull;
+    }();
+    return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int D>
+cudaError_t set_attn_attrs()
+{
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         AttnCfg<D>::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                AttnCfg<D>::kSmemBytes);
+}
+
+// Once per device: check it is an sm_100 part, resolve the tensor-map
+// encoder from the driver and raise the kernels' shared-memory limit.
+int ensure_device()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return UNIPIN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_init_mutex);
+    if (g_device_ready[dev]) return UNIPIN_OK;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    if (major != 10 || minor != 0) return UNIPIN_ERR_UNSUPPORTED;
+    if (!g_encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return UNIPIN_ERR_CUDA;
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    if (set_attn_attrs<32>() != cudaSuccess || set_attn_attrs<64>() != cudaSuccess ||
+        set_attn_attrs<128>() != cudaSuccess)
+        return UNIPIN_ERR_CUDA;
+    g_device_ready[dev] = true;
+    return UNIPIN_OK;
+}
+
+// bf16 3-D tensor map, dims innermost first, strides in bytes for dims 1 and 2.
+int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t st1, uint64_t st2,
+             uint32_t b0, uint32_t b1, uint32_t b2, int D)
+{
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {st1, st2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t elem[3] = {1, 1, 1};
+    const CUtensorMapSwizzle sw = D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+// Packed token tensor [T, H, D]: boxes of 128 tokens x 1 head x (D or 64) elements.
+int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D)
+{
+    const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
+    return make_map(m, base, (uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)D * 2, (uint64_t)H * D * 2, box_d, 1,
+                    kBlockN, D);
+}
+
+// Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of 128 history rows.
+int make_pool_map(CUtensorMap* m, const void* base, const unipin_kvpool* pool)
+{
+    const int D = pool->D;
+    const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
+    const uint64_t planes = (uint64_t)pool->L * pool->S * pool->H;
+    return make_map(m, base, (uint64_t)D, (uint64_t)pool->n_cap, planes, (uint64_t)D * 2,
+                    (uint64_t)pool->n_cap * D * 2, box_d, kBlockN, 1, D);
+}
+
+int check_pool(const unipin_kvpool* pool, int H, int D, int layer)
+{
+    if (!pool || !pool->k || !pool->v) return UNIPIN_ERR_INVALID_ARG;
+    if (pool->L < 1 || pool->S < 1 || pool->n_cap < 1 || pool->H != H || pool->D != D) return UNIPIN_ERR_INVALID_ARG;
+    if (!aligned16(pool->k) || !aligned16(pool->v)) return UNIPIN_ERR_MISALIGNED;
+    if (layer < 0 || layer >= pool->L) return UNIPIN_ERR_OUT_OF_RANGE;
+    if ((uint64_t)pool->L * pool->S * pool->H >= (1ull << 31)) return UNIPIN_ERR_INVALID_ARG;
+    return UNIPIN_OK;
+}
+
+bool supported_d(int D) { return D == 32 || D == 64 || D == 128; }
+
+template <bool kDecode>
+int launch_attn(int D, dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const AttnParams& p, cudaStream_t s)
+{
+    switch (D) {
+    case 32:
+        attn_fwd_kernel<32, kDecode><<<grid, kThreads, AttnCfg<32>::kSmemBytes, s>>>(tq, tk, tv, p);
+        break;
+    case 64:
+        attn_fwd_kernel<64, kDecode><<<grid, kThreads, AttnCfg<64>::kSmemBytes, s>>>(tq, tk, tv, p);
+        break;
+    case 128:
+        attn_fwd_kernel<128, kDecode><<<grid, kThreads, AttnCfg<128>::kSmemBytes, s>>>(tq, tk, tv, p);
+        break;
+    default:
+        return UNIPIN_ERR_UNSUPPORTED;
+    }
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+int launch_pool_write(const unipin_kvpool* pool, int layer, const void* k, const void* v, const int* cu,
+                      const int* past, const int* slots, int B, int H, int D, int max_past, int total_tokens,
+                      int* status, cudaStream_t s)
+{
+    if (B == 0 || max_past == 0) return UNIPIN_OK;
+    PoolWriteParams p;
+    p.k = static_cast<const uint4*>(k);
+    p.v = static_cast<const uint4*>(v);
+    p.pool_k = static_cast<uint4*>(pool->k);
+    p.pool_v = static_cast<uint4*>(pool->v);
+    p.cu = cu;
+    p.past = past;
+    p.slots = slots;
+    p.H = H;
+    p.D = D;
+    p.S = pool->S;
+    p.n_cap = pool->n_cap;
+    p.layer = layer;
+    p.total_tokens = total_tokens;
+    p.status = status;
+    const long long vecs = (long long)max_past * (D / 8);
+    const long long blocks = (vecs + 255) / 256;
+    dim3 grid((unsigned)(blocks < 65535 ? blocks : 65535), (unsigned)H, (unsigned)B);
+    kvpool_write_kernel<<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
+{
+    if (R < 1 || H < 1 || max_k < 1 || n_cap < 1) return 1;
+    const long long units = (long long)R * H * ((max_k + kBlockM - 1) / kBlockM);
+    const long long slots = (long long)kNumSmsHint * (D <= 64 ? 2 : 1);
+    const long long target = 4 * slots;
+    if (units >= slots) return 1;
+    const int key_tiles = (n_cap + kBlockN - 1) / kBlockN;
+    long long ns = (target + units - 1) / units;
+    const long long cap = key_tiles / 2 > 1 ? key_tiles / 2 : 1;   // at least two key tiles per split
+    if (ns > cap) ns = cap;
+    if (ns > 32) ns = 32;
+    return (int)(ns < 1 ? 1 : ns);
+}
+
+size_t decode_workspace_bytes(int nsplit, int total_cand, int H, int D)
+{
+    if (nsplit <= 1) return 0;
+    const size_t rows = (size_t)nsplit * (size_t)total_cand * (size_t)H;
+    return rows * (size_t)D * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+__global__ void bounded_wait_selftest_kernel(int* status, unsigned long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    __syncthreads();
+    WaitCtl ctl{&abort_flag, status, limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, ctl);   // nothing ever arrives
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* unipin_status_string(int status)
+{
+    switch (status) {
+    case UNIPIN_OK: return "UNIPIN_OK";
+    case UNIPIN_ERR_INVALID_ARG: return "UNIPIN_ERR_INVALID_ARG";
+    case UNIPIN_ERR_UNSUPPORTED: return "UNIPIN_ERR_UNSUPPORTED";
+    case UNIPIN_ERR_MISALIGNED: return "UNIPIN_ERR_MISALIGNED";
+    case UNIPIN_ERR_OUT_OF_RANGE: return "UNIPIN_ERR_OUT_OF_RANGE";
+    case UNIPIN_ERR_CUDA: return "UNIPIN_ERR_CUDA";
+    case UNIPIN_ERR_DEVICE_TIMEOUT: return "UNIPIN_ERR_DEVICE_TIMEOUT";
+    default: return "UNIPIN_ERR_UNKNOWN";
+    }
+}
+
+int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                               const int* cu_seqlens, const int* past_lens, int B, int H, int D, int max_seqlen,
+                               int total_tokens, float scale, const unipin_kvpool* pool, const int* slot_ids,
+                               int layer, int* dev_status, void* stream)
+{
+    if (B < 0 || H < 1 || max_seqlen < 0 || total_tokens < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return UNIPIN_ERR_INVALID_ARG;
+    if (pool) {
+        int rc = check_pool(pool, H, D, layer);
+        if (rc != UNIPIN_OK) return rc;
+        if (!slot_ids) return UNIPIN_ERR_INVALID_ARG;
+    }
+    if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
+    if (!q || !k || !v || !out || !cu_seqlens || !past_lens) return UNIPIN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return UNIPIN_ERR_MISALIGNED;
+    if (B > 65535 || H > 65535) return UNIPIN_ERR_INVALID_ARG;
+    int rc = ensure_device();
+    if (rc != UNIPIN_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    if (pool) {
+        rc = launch_pool_write(pool, layer, k, v, cu_seqlens, past_lens, slot_ids, B, H, D, max_seqlen, total_tokens,
+                               dev_status, s);
+        if (rc != UNIPIN_OK) return rc;
+    }
+    CUtensorMap tq, tk, tv;
+    if ((rc = make_token_map(&tq, q, total_tokens, H, D)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tk, k, total_tokens, H, D)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tv, v, total_tokens, H, D)) != UNIPIN_OK) return rc;
+
+    AttnParams p = {};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k_self = static_cast<const __nv_bfloat16*>(k);
+    p.v_self = static_cast<const __nv_bfloat16*>(v);
+    p.out = out;
+    p.cu = cu_seqlens;
+    p.past = past_lens;
+    p.slots = nullptr;
+    p.H = H;
+    p.max_rows = max_seqlen;
+    p.total_rows = total_tokens;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.nsplit = 1;
+    p.sl2 = scale * kLog2e;
+    p.status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+    dim3 grid((unsigned)((max_seqlen + kBlockM - 1) / kBlockM), (unsigned)H, (unsigned)B);
+    return launch_attn<false>(D, grid, tq, tk, tv, p, s);
+}
+
+int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, const void* v, const int* cu_seqlens,
+                        const int* past_lens, const int* slot_ids, int B, int max_past, int total_tokens,
+                        int* dev_status, void* stream)
+{
+    if (!pool) return UNIPIN_ERR_INVALID_ARG;
+    if (B < 0 || max_past < 0 || total_tokens < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (!supported_d(pool->D)) return UNIPIN_ERR_UNSUPPORTED;
+    int rc = check_pool(pool, pool->H, pool->D, layer);
+    if (rc != UNIPIN_OK) return rc;
+    if (max_past > pool->n_cap) return UNIPIN_ERR_OUT_OF_RANGE;
+    if (B == 0 || max_past == 0 || total_tokens == 0) return UNIPIN_OK;
+    if (!k || !v || !cu_seqlens || !past_lens || !slot_ids) return UNIPIN_ERR_INVALID_ARG;
+    if (!aligned16(k) || !aligned16(v)) return UNIPIN_ERR_MISALIGNED;
+    if (B > 65535 || pool->H > 65535) return UNIPIN_ERR_INVALID_ARG;
+    rc = ensure_device();
+    if (rc != UNIPIN_OK) return rc;
+    return launch_pool_write(pool, layer, k, v, cu_seqlens, past_lens, slot_ids, B, pool->H, pool->D, max_past,
+                             total_tokens, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap)
+{
+    if (R < 1 || H < 1 || !supported_d(D) || max_k < 1 || total_cand < 1 || n_cap < 1) return 0;
+    return decode_workspace_bytes(decode_nsplit(R, H, D, max_k, n_cap), total_cand, H, D);
+}
+
+int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
+                            const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H, int D,
+                            int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer,
+                            void* workspace, size_t workspace_bytes, int* dev_status, void* stream)
+{
+    if (R < 0 || H < 1 || max_k < 0 || total_cand < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return UNIPIN_ERR_INVALID_ARG;
+    int rc = check_pool(pool, H, D, layer);
+    if (rc != UNIPIN_OK) return rc;
+    if (R == 0 || total_cand == 0 || max_k == 0) return UNIPIN_OK;
+    if (!q_c || !k_c || !v_c || !out || !cu_seqlens_c || !slot_ids || !past_lens) return UNIPIN_ERR_INVALID_ARG;
+    if (!aligned16(q_c) || !aligned16(k_c) || !aligned16(v_c) || !aligned16(out)) return UNIPIN_ERR_MISALIGNED;
+    if (workspace && !aligned16(workspace)) return UNIPIN_ERR_MISALIGNED;
+    if (R > 65535 || H > 65535) return UNIPIN_ERR_INVALID_ARG;
+    rc = ensure_device();
+    if (rc != UNIPIN_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    int nsplit = decode_nsplit(R, H, D, max_k, pool->n_cap);
+    if (nsplit > 1 && (!workspace || workspace_bytes < decode_workspace_bytes(nsplit, total_cand, H, D))) nsplit = 1;
+
+    CUtensorMap tq, tk, tv;
+    if ((rc = make_token_map(&tq, q_c, total_cand, H, D)) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tk, pool->k, pool)) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tv, pool->v, pool)) != UNIPIN_OK) return rc;
+
+    AttnParams p = {};
+    p.q = static_cast<const __nv_bfloat16*>(q_c);
+    p.k_self = static_cast<const __nv_bfloat16*>(k_c);
+    p.v_self = static_cast<const __nv_bfloat16*>(v_c);
+    p.out = out;
+    p.cu = cu_seqlens_c;
+    p.past = past_lens;
+    p.slots = slot_ids;
+    p.H = H;
+    p.max_rows = max_k;
+    p.total_rows = total_cand;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.layer = layer;
+    p.S = pool->S;
+    p.n_cap = pool->n_cap;
+    p.nsplit = nsplit;
+    p.sl2 = scale * kLog2e;
+    p.status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+    if (nsplit > 1) {
+        p.part_o = static_cast<float*>(workspace);
+        p.part_ml = p.part_o + (size_t)nsplit * total_cand * H * D;
+    }
+    const unsigned qtiles = (unsigned)((max_k + kBlockM - 1) / kBlockM);
+    dim3 grid(qtiles * (unsigned)nsplit, (unsigned)H, (unsigned)R);
+    rc = launch_attn<true>(D, grid, tq, tk, tv, p, s);
+    if (rc != UNIPIN_OK || nsplit == 1) return rc;
+
+    const long long rows = (long long)total_cand * H;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    switch (D) {
+    case 32:
+        decode_merge_kernel<32><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
+                                                       p.out_fp32, total_cand, H, nsplit, p.sl2);
+        break;
+    case 64:
+        decode_merge_kernel<64><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
+                                                       p.out_fp32, total_cand, H, nsplit, p.sl2);
+        break;
+    default:
+        decode_merge_kernel<128><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
+                                                        p.out_fp32, total_cand, H, nsplit, p.sl2);
+        break;
+    }
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+int unipin_selftest_bounded_wait(int* dev_status, unsigned int limit_us, void* stream)
+{
+    if (!dev_status || limit_us == 0) return UNIPIN_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        dev_status, (unsigned long long)limit_us * 1000ull);
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -7,9 +7,9 @@ their inputs from here without sharing any of the method's code.
 Recipe (the pages fix no input distribution; these choices are ours):
 
 * Generator: ``numpy.random.Generator(PCG64(seed))``.
-* Values: ``standard_normal`` in float64, rounded to float32 (round to nearest
-  even), then to bfloat16 (round to nearest even).  Arrays hold the raw
-  bfloat16 bit patterns as ``uint16``.
+* Values: ``standard_normal(dtype=float32)``, rounded to bfloat16 (round to
+  nearest even), drawn in chunks of at most 2**26 values in C order.  Arrays
+  hold the raw bfloat16 bit patterns as ``uint16``.
 * Draw order inside one workload: the per-segment lengths (past ``n_b`` then
   candidate ``k_b``), the slot permutation, then Q, K, V, then pool rows.
 * Seeds: ``20261202 + i`` for the i-th named workload in ``WORKLOADS``.
@@ -49,8 +49,19 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return u.view(np.float32).astype(np.float64)
 
 
+_CHUNK = 1 << 26
+
+
 def normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
-    return f64_to_bf16_bits(rng.standard_normal(size=shape))
+    """N(0,1) samples as bfloat16 bit patterns of the given shape."""
+    shape = tuple(int(x) for x in np.atleast_1d(shape)) if not isinstance(shape, tuple) else shape
+    n = int(np.prod(shape)) if len(shape) else 1
+    out = np.empty(n, dtype=np.uint16)
+    for lo in range(0, n, _CHUNK):
+        hi = min(n, lo + _CHUNK)
+        u = rng.standard_normal(hi - lo, dtype=np.float32).view(np.uint32)
+        out[lo:hi] = ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
+    return out.reshape(shape)
 
 
 @dataclasses.dataclass

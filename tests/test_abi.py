@@ -1,0 +1,76 @@
+"""CPU-only checks of the boundary: the library loads and exports what the header declares."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "unipin.h")
+LIB = os.path.join(ROOT, "kv_cache_reuse_falcon_b200", "libunipin.so")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(unipin_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from kv_cache_reuse_falcon_b200 import build
+    build.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_three_hot_path_calls():
+    names = declared_functions()
+    for n in ("unipin_masked_prefill_attn", "unipin_kvpool_write", "unipin_rank_decode_attn"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    lib.unipin_status_string.restype = ctypes.c_char_p
+    lib.unipin_status_string.argtypes = [ctypes.c_int]
+    assert lib.unipin_status_string(0) == b"UNIPIN_OK"
+    assert lib.unipin_status_string(-6) == b"UNIPIN_ERR_DEVICE_TIMEOUT"
+    assert lib.unipin_status_string(42) == b"UNIPIN_ERR_UNKNOWN"
+
+
+def test_host_validation_needs_no_device(lib):
+    """Argument errors are found before any CUDA call, so they work without a GPU."""
+    P, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.unipin_masked_prefill_attn
+    f.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, ctypes.c_float, P, P, I, P, P]
+    f.restype = I
+    assert f(None, None, None, None, 1, None, None, 1, 1, 48, 16, 16, 0.1, None, None, 0, None, None) == -2
+    assert f(None, None, None, None, 1, None, None, -1, 1, 64, 16, 16, 0.1, None, None, 0, None, None) == -1
+    assert f(None, None, None, None, 1, None, None, 1, 1, 64, 16, 16, -1.0, None, None, 0, None, None) == -1
+    # nothing to do: B = 0 returns OK without touching the device
+    assert f(None, None, None, None, 1, None, None, 0, 1, 64, 16, 0, 0.1, None, None, 0, None, None) == 0
+    g = lib.unipin_rank_decode_workspace_size
+    g.argtypes = [I, I, I, I, I, I]
+    g.restype = ctypes.c_size_t
+    assert g(32, 8, 64, 16, 512, 2048) > 0
+    assert g(32, 8, 64, 1000, 32000, 2048) == 0
+
+
+def test_binding_refuses_to_load_without_library(tmp_path):
+    from kv_cache_reuse_falcon_b200 import binding
+    with pytest.raises(ImportError):
+        binding._load(str(tmp_path / "missing.so"))
+
+
+def test_no_oracle_import_in_product_code():
+    pkg = os.path.join(ROOT, "kv_cache_reuse_falcon_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, fn)).read()
+                assert "import oracle" not in src and "from oracle" not in src, fn
