@@ -313,8 +313,11 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
                 ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (i - 1) & 1, ctl));
                 if (!ok) break;
                 tc_fence_after_sync();
-                if (m_new > m) {
-                    const float corr = ex2_approx(m - m_use);
+                // The TMEM load/store below are warp-collective, so the branch is
+                // taken by the whole warp when any row's max grew; rows whose
+                // max did not grow scale by 1.
+                if (__any_sync(0xffffffffu, m_new > m)) {
+                    const float corr = (m_new > m) ? ex2_approx(m - m_use) : 1.f;
                     l *= corr;
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
