@@ -79,9 +79,15 @@ def load_peaks():
 
 # ----------------------------------------------------------------- workload
 
-def make_workload(name: str, seed: int):
-    """Host arrays of one step's inputs (bf16 bits) for the named workload."""
+def make_workload(name: str, seed: int, users: int = 0):
+    """Host arrays of one step's inputs (bf16 bits) for the named workload.
+
+    users > 0 replaces the workload's user count (and pool slot count) to make a
+    smaller case of the same length distribution, e.g. for profiler captures."""
     w = synth.workload(name)
+    if users > 0:
+        import dataclasses
+        w = dataclasses.replace(w, B=users, S=users)
     rng = np.random.Generator(np.random.PCG64(seed))
     past, cand = w.lengths(rng)
     S = w.S if w.S else max(w.B, 1)
@@ -197,7 +203,7 @@ def run_ours(args, rank, world, device, dist):
     name = args.workload
     w = synth.workload(name)
     seed = rank_seed(w.seed, rank)
-    w, batch, S, n_cap = make_workload(name, seed)
+    w, batch, S, n_cap = make_workload(name, seed, args.users)
     H, D = batch.H, batch.D
     T = batch.T
     past, cand = batch.past_lens, batch.cand_lens
@@ -344,7 +350,8 @@ def run_ours(args, rank, world, device, dist):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": name, "users_per_gpu": batch.B, "H": H, "D": D,
+        "config": {"workload": name if not args.users else "%s[users=%d]" % (name, args.users),
+                   "users_per_gpu": batch.B, "H": H, "D": D,
                    "tokens_per_gpu": T, "candidates_per_gpu": Tc, "pool": [L, S, H, n_cap, D],
                    "layers_per_step": 1, "parallelism": "users sharded across %d GPU(s), no collective" % world,
                    "l2": "inputs larger than L2 (no flush)", "seed_rank0": seed},
@@ -400,7 +407,8 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": name, "users_per_gpu": batch.B, "H": batch.H, "D": batch.D},
+        "config": {"workload": name if not args.users else "%s[users=%d]" % (name, args.users),
+                   "users_per_gpu": batch.B, "H": batch.H, "D": batch.D},
         "cpu_baseline": {"value": value, "unit": "candidate tokens/s", "cores": sample["cores"], "kind": "oracle",
                          "sample": sample["sample"]},
         "e2e": {"value": value, "unit": "candidate tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -416,6 +424,7 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--users", type=int, default=0, help="smaller case: this many users (profiling)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -1,0 +1,170 @@
+"""Full-size workloads on the GPU, in the launch configuration the benchmark times.
+
+The CUDA path runs on the whole batch; the oracle checks sampled rows (tile
+edges, the past/candidate boundary, segment ends, plus random rows), since it
+computes rows one by one.  Properties that hold at any size are checked on
+every row: no NaN (no stale pool row is read), bit-exact pool contents, and
+decode rows equal to the prefill's candidate rows.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_reuse_falcon_b200 import synth
+from tests.gpu_helpers import (DevDecode, DevPrefill, bf16_tensor_bits, fill_pool_rows, host_pool_layer,
+                               nan_pool, parity)
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+
+
+@pytest.fixture(scope="module")
+def ub():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from kv_cache_reuse_falcon_b200 import binding
+    return binding
+
+
+def sample_rows(cu, past, count, seed):
+    """Token indices: segment ends, rows around the past/candidate boundary and tile edges, random rows."""
+    rng = np.random.default_rng(seed)
+    B = len(past)
+    picks = set()
+    for b in rng.choice(B, size=min(B, 24), replace=False):
+        lo, hi, n = int(cu[b]), int(cu[b + 1]), int(past[b])
+        for r in (0, 1, 126, 127, 128, 129, n - 1, n, n + 1, hi - lo - 1):
+            if 0 <= r < hi - lo:
+                picks.add(lo + r)
+    T = int(cu[-1])
+    picks.update(rng.integers(0, T, size=max(0, count - len(picks))).tolist())
+    return np.array(sorted(picks), dtype=np.int64)
+
+
+def build(name):
+    w = synth.workload(name)
+    rng = np.random.Generator(np.random.PCG64(w.seed))
+    past, cand = w.lengths(rng)
+    S = w.S if w.S else w.B
+    return w, synth.make_prefill(w.seed, past, cand, w.H, w.D, n_slots=S, rng=rng), rng
+
+
+@pytest.mark.parametrize("name", ["prefill_B64", "table2_B8", "tiny_prefill"])
+def test_prefill_workloads(ub, name):
+    w, batch, _ = build(name)
+    dp = DevPrefill(batch)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ub.masked_prefill_attn(dp.q, dp.k, dp.v, dp.cu, dp.past, dp.max_seqlen, out_fp32=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.isfinite(out).all()
+    rows = sample_rows(batch.cu_seqlens, batch.past_lens, 3000, 1)
+    ref = oracle.prefill(batch.q, batch.k, batch.v, batch.cu_seqlens, batch.past_lens, tokens=rows)
+    parity(out[torch.from_numpy(rows).cuda()].cpu().numpy(), ref, name)
+
+
+def test_prefill_with_pool_write_serving_scale(ub):
+    """B=128, n=1024, k=512, H=8, D=64; pool [12, 256, 8, 1024, 64] at random distinct slots."""
+    w, batch, _ = build("prefill_pool_B128")
+    dp = DevPrefill(batch)
+    layer = 7
+    pk, pv = nan_pool(w.L, w.S, w.H, w.n_cap, w.D)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ub.masked_prefill_attn(dp.q, dp.k, dp.v, dp.cu, dp.past, dp.max_seqlen, out_fp32=True,
+                                 pool_k=pk, pool_v=pv, slot_ids=dp.slots, layer=layer, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = sample_rows(batch.cu_seqlens, batch.past_lens, 3000, 2)
+    ref = oracle.prefill(batch.q, batch.k, batch.v, batch.cu_seqlens, batch.past_lens, tokens=rows)
+    parity(out[torch.from_numpy(rows).cuda()].cpu().numpy(), ref, "serving-scale prefill")
+    # pool: the written layer, byte for byte, against the oracle's mirror of that layer
+    hk = np.full((1, w.S, w.H, w.n_cap, w.D), synth.BF16_NAN, dtype=np.uint16)
+    hv = hk.copy()
+    oracle.pool_write(hk, hv, 0, batch.k, batch.v, batch.cu_seqlens, batch.past_lens, batch.slot_ids)
+    assert bf16_tensor_bits(pk[layer]).tobytes() == hk[0].tobytes()
+    assert bf16_tensor_bits(pv[layer]).tobytes() == hv[0].tobytes()
+    # every other layer is untouched (still the NaN pattern)
+    nan = torch.tensor(0x7FC0, dtype=torch.int16, device="cuda")
+    for t in (pk, pv):
+        other = torch.cat([t[:layer].reshape(-1), t[layer + 1:].reshape(-1)]).view(torch.int16)
+        assert bool((other == nan).all())
+
+
+def test_rank_decode_from_pool_workload(ub):
+    """Pool [12, 256, 8, 2048, 64]; 32 requests, distinct random slots, k=1000 each; one layer."""
+    w = synth.workload("decode_R32")
+    rng = np.random.Generator(np.random.PCG64(w.seed))
+    past = np.full(w.B, w.n, np.int32)
+    cand = np.full(w.B, w.k, np.int32)
+    d = synth.make_decode(w.seed, past, cand, w.H, w.D, n_slots=w.S, rng=rng)
+    ks, vs = synth.pool_rows(rng, past, w.H, w.D)
+    layer = 5
+    pk, pv = nan_pool(w.L, w.S, w.H, w.n_cap, w.D)
+    fill_pool_rows(pk, pv, layer, d.slot_ids, past, ks, vs)
+    dd = DevDecode(d)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, layer, dd.max_k,
+                              out_fp32=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.isfinite(out).all()
+    hk, hv = host_pool_layer(1, w.S, w.H, w.n_cap, w.D, 0, d.slot_ids, past, ks, vs)
+    rows = sample_rows(d.cu_seqlens, np.zeros_like(past), 1500, 3)
+    ref = oracle.decode(d.q, d.k, d.v, d.cu_seqlens, d.slot_ids, d.past_lens, hk, hv, 0, tokens=rows)
+    parity(out[torch.from_numpy(rows).cuda()].cpu().numpy(), ref, "decode R32 k1000")
+    # small-k sweep over the same pool with the split-n path (k = 16 per request)
+    cand16 = np.full(w.B, 16, np.int32)
+    d16 = synth.make_decode(w.seed + 100, past, cand16, w.H, w.D, n_slots=w.S)
+    d16.slot_ids = d.slot_ids
+    dd16 = DevDecode(d16)
+    nbytes = ub.rank_decode_workspace_size(w.B, w.H, w.D, 16, int(d16.cu_seqlens[-1]), w.n_cap)
+    assert nbytes > 0
+    ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device="cuda")
+    o16 = ub.rank_decode_attn(dd16.q, dd16.k, dd16.v, dd16.cu, dd16.slots, dd16.past, pk, pv, layer, 16,
+                              out_fp32=True, workspace=ws, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    ref16 = oracle.decode(d16.q, d16.k, d16.v, d16.cu_seqlens, d16.slot_ids, d16.past_lens, hk, hv, 0)
+    parity(o16.cpu().numpy(), ref16, "decode R32 k16 split-n")
+
+
+def test_ragged_mixed_batch_prefill_then_decode(ub):
+    """256 users, n ~ U{32..4096}, k ~ U{50..2000}, H=8, D=128: prefill + pool write, then decode."""
+    w, batch, _ = build("ragged_B256")
+    dp = DevPrefill(batch)
+    pk, pv = nan_pool(w.L, w.S, w.H, w.n_cap, w.D)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = ub.masked_prefill_attn(dp.q, dp.k, dp.v, dp.cu, dp.past, dp.max_seqlen, out_fp32=True,
+                                 pool_k=pk, pool_v=pv, slot_ids=dp.slots, layer=0, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = sample_rows(batch.cu_seqlens, batch.past_lens, 2000, 4)
+    ref = oracle.prefill(batch.q, batch.k, batch.v, batch.cu_seqlens, batch.past_lens, tokens=rows)
+    parity(out[torch.from_numpy(rows).cuda()].cpu().numpy(), ref, "ragged prefill")
+
+    cidx = np.concatenate([np.arange(batch.cu_seqlens[b] + batch.past_lens[b], batch.cu_seqlens[b + 1])
+                           for b in range(batch.B)])
+    cidx_d = torch.from_numpy(cidx).cuda()
+    d = synth.DecodeBatch(w.H, w.D, batch.past_lens, batch.cand_lens, synth.cu_from_lens(batch.cand_lens),
+                          batch.slot_ids, None, None, None)
+    dd = DevDecode.__new__(DevDecode)
+    dd.q, dd.k, dd.v = dp.q[cidx_d].contiguous(), dp.k[cidx_d].contiguous(), dp.v[cidx_d].contiguous()
+    dd.cu = torch.from_numpy(d.cu_seqlens).cuda()
+    dd.past, dd.slots = dp.past, dp.slots
+    dd.max_k = int(batch.cand_lens.max())
+    for use_ws in (False, True):
+        ws = None
+        if use_ws:
+            nb = ub.rank_decode_workspace_size(batch.B, w.H, w.D, dd.max_k, len(cidx), w.n_cap)
+            ws = torch.empty(nb // 4 + 4, dtype=torch.float32, device="cuda") if nb else None
+        dec = ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, 0, dd.max_k,
+                                  out_fp32=True, workspace=ws, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        assert torch.isfinite(dec).all()
+        # every decode row equals the prefill's row for that candidate
+        assert torch.equal(dec, out[cidx_d])
+    crow = np.random.default_rng(5).choice(len(cidx), size=600, replace=False)
+    ref_c = oracle.prefill(batch.q, batch.k, batch.v, batch.cu_seqlens, batch.past_lens, tokens=cidx[crow])
+    parity(dec[torch.from_numpy(crow).cuda()].cpu().numpy(), ref_c, "ragged decode")
