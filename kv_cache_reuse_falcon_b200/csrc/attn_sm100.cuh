@@ -1,41 +1,50 @@
-// M-FALCON masked attention engine for sm_100a: one thread block per
-// (segment, head, 128-row query tile), tcgen05 UMMA with TMEM accumulators,
-// TMA-staged K/V tiles, fp32 online softmax with one TMEM lane (one thread)
-// per query row.
+// M-FALCON masked attention engine for sm_100a.
+//
+// One thread block per (segment, head, pair of 128-row query tiles A and B).
+// The two tiles share every K/V tile and run as a ping-pong: while the
+// tensor cores work on one tile's S = Q K^T and O += P V, the other tile's
+// softmax warpgroup turns its scores into probabilities.
 //
 // The same engine runs the prefill and the rank decode.  In both, the part
 // of a row's key set that is a contiguous run of keys 0..kmax-1 goes through
 // the tensor cores with the causal predicate j <= i, and a candidate's own
 // key (the diagonal of the candidate block) is merged in afterwards as a
 // per-row fp32 dot product:
-//   prefill ([notes] §3 "attention mask"):  kmax = min(rows in the tile's reach, n_b);
-//       past row i sees j <= i < n_b; candidate row i >= n_b sees all j < n_b,
-//       plus itself through the self term.
+//   prefill ([notes] §3 "attention mask"):  past row i sees j <= i < n_b;
+//       candidate row i >= n_b sees all j < n_b plus itself (self term).
 //   rank decode ([review] §2.4, [notes] §6):  keys are pool rows 0..n_r-1 of
-//       the request's slot; every candidate sees all of them, plus itself.
-// Fully masked key tiles are never visited (the tile loop stops at kmax), and
-// key tiles entirely below the diagonal and below kmax skip the per-element
-// predicate.
+//       the request's slot; every candidate sees all of them plus itself.
+// Key tiles past kmax are never visited; key tiles entirely below the
+// diagonal and below kmax skip the per-element predicate.
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r; row max and
-//              row sum stay in that thread's registers, so no shuffles are
-//              needed for the row statistics; corrects O in TMEM when the
-//              row max grows; writes P (bf16) to shared memory; epilogue.
-//   warp 4     TMA producer (Q once, then K/V tiles through a 2-stage ring).
-//   warp 5     TMEM allocator and the single UMMA-issuing thread.
+// Warp roles (320 threads):
+//   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns
+//              query row r = TMEM lane r, so the row max and row sum stay in
+//              one thread's registers; S is read from TMEM with one wide load,
+//              P (bf16) is written back into TMEM over S and consumed from
+//              there by the P.V MMA.  The O accumulator is rescaled in TMEM
+//              only when a row max grows by more than 2^8 (stale maxima keep
+//              P <= 2^8, exact after the final division).
+//   warp 8     TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through
+//              a ring of shared-memory slots.
+//   warp 9     TMEM allocator and the single UMMA-issuing thread.
+//
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B [256+D, 256+2D);
+// P_X occupies the first 64 columns of S_X.
 #pragma once
 
 #include "sm100_ptx.cuh"
+#include "tmem_wide.cuh"
 #include "unipin.h"
 
 namespace unipin {
 
-constexpr int kBlockM = 128;   // query rows per tile = TMEM lanes
-constexpr int kBlockN = 128;   // keys per tile
-constexpr int kThreads = 192;
-constexpr int kTmemCols = 256; // S: 128 columns, O: D <= 128 columns
+constexpr int kBlockM = 128;     // query rows per tile = TMEM lanes
+constexpr int kBlockN = 128;     // keys per tile
+constexpr int kThreads = 320;
+constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;   // rescale O only when a row max grows by > 2^8
 
 template <int D>
 struct AttnCfg {
@@ -45,16 +54,12 @@ struct AttnCfg {
     static constexpr int kRowBytes = kBoxD * 2;                 // 128 (SW128) or 64 (SW64)
     static constexpr uint32_t kLayout = kRowBytes == 128 ? kLayoutSw128 : kLayoutSw64;
     static constexpr int kAtomBytes = kBlockM * kRowBytes;      // one box of 128 rows
-    static constexpr int kTileBytes = kBlockM * D * 2;          // Q, K or V tile
-    static constexpr int kStages = 2;
-    static constexpr int kPBytes = kBlockM * kBlockN * 2;       // P tile, bf16, SW128 K-major
-    static constexpr int kOffQ = 0;
-    static constexpr int kOffK = kOffQ + kTileBytes;
-    static constexpr int kOffV = kOffK + kStages * kTileBytes;
-    static constexpr int kOffP = kOffV + kStages * kTileBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
-    static constexpr int kSmemBytes = kOffBar + 128;
-    static constexpr int kMinBlocks = D <= 64 ? 2 : 1;
+    static constexpr int kTileBytes = kBlockM * D * 2;          // one Q, K or V tile
+    static constexpr int kStages = D == 128 ? 4 : 8;            // ring slots (each one K or one V tile)
+    static constexpr int kOffQ = 0;                             // Q_A, Q_B
+    static constexpr int kOffRing = 2 * kTileBytes;
+    static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+    static constexpr int kSmemBytes = kOffBar + 256;
 };
 
 struct AttnParams {
@@ -72,7 +77,7 @@ struct AttnParams {
     int total_rows;               // T
     int out_fp32;
     int layer, S, n_cap;          // pool geometry (decode)
-    int nsplit;                   // decode: key-range splits per query tile
+    int nsplit;                   // decode: key-range splits per query-tile pair
     float sl2;                    // scale * log2(e)
     int* status;
     unsigned long long wait_limit_ns;
@@ -88,8 +93,14 @@ __device__ __forceinline__ void key_tile(int t, int nt, int kmax, int& start, in
     start = (t == nt - 1 && (kmax % kBlockN) != 0) ? kmax - kBlockN : lo;
 }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
 template <int D, bool kDecode>
-__global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p)
 {
@@ -102,10 +113,11 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
     const int seg = blockIdx.z;
     const int h = blockIdx.y;
 
-    // ------------------------------------------------------------ work unit
     // A timeout recorded earlier means a block of this or a previous launch
     // gave up; later blocks skip their work instead of waiting again.
     if (p.status && *reinterpret_cast<volatile int*>(p.status) == (int)UNIPIN_ERR_DEVICE_TIMEOUT) return;
+
+    // ------------------------------------------------------------ work unit
     const int tok0 = p.cu[seg];
     const int nrows_seg = p.cu[seg + 1] - tok0;
     const int npast = p.past[seg];
@@ -122,58 +134,69 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
         if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0, (int)UNIPIN_ERR_OUT_OF_RANGE);
         return;
     }
-    const int ntiles_q = (nrows_seg + kBlockM - 1) / kBlockM;
+    const int npairs = (nrows_seg + 2 * kBlockM - 1) / (2 * kBlockM);
     const int split = kDecode ? (int)(blockIdx.x % p.nsplit) : 0;
-    const int qidx = kDecode ? (int)(blockIdx.x / p.nsplit) : (int)blockIdx.x;
-    if (qidx >= ntiles_q) return;
-    // Prefill: the costliest query tile of a segment (the last) launches first.
-    const int qt = kDecode ? qidx : (ntiles_q - 1 - qidx);
-    const int qrow0 = qt * kBlockM;
-    const int nrows = min(kBlockM, nrows_seg - qrow0);
-    const int causal0 = kDecode ? npast + qrow0 : qrow0;   // mask position of row 0
-    const int kmax = kDecode ? npast : min(qrow0 + nrows, npast);
+    const int pidx = kDecode ? (int)(blockIdx.x / p.nsplit) : (int)blockIdx.x;
+    if (pidx >= npairs) return;
+    // Prefill: the costliest pair of a segment (the last) launches first.
+    const int qp = kDecode ? pidx : (npairs - 1 - pidx);
+    const int qrow0 = qp * 2 * kBlockM;                    // first row of tile A
+    const int nrows_a = min(kBlockM, nrows_seg - qrow0);
+    const int nrows_b = min(kBlockM, nrows_seg - qrow0 - kBlockM);
+    const bool has_b = nrows_b > 0;
+    const int pos0 = kDecode ? npast + qrow0 : qrow0;      // mask position of row 0 of tile A
+    const int kmax_a = kDecode ? npast : min(qrow0 + nrows_a, npast);
+    const int kmax_b = !has_b ? 0 : (kDecode ? npast : min(qrow0 + kBlockM + nrows_b, npast));
+    // Tile geometry follows the longer key range; tile A's range is a prefix of
+    // it with identical tiles (kmax_a < kmax_b only when kmax_a is a multiple of 128).
+    const int kmax = has_b ? kmax_b : kmax_a;
     const int nt_all = (kmax + kBlockN - 1) / kBlockN;
-    int t_begin = 0, t_end = nt_all;
+    int t_begin = 0;
+    int t_end_a = (kmax_a + kBlockN - 1) / kBlockN;
+    int t_end_b = (kmax_b + kBlockN - 1) / kBlockN;
     if (kDecode && p.nsplit > 1) {
         const int per = (nt_all + p.nsplit - 1) / p.nsplit;
         t_begin = min(split * per, nt_all);
-        t_end = min(t_begin + per, nt_all);
+        t_end_a = min(t_begin + per, t_end_a);
+        t_end_b = min(t_begin + per, t_end_b);
     }
-    const int nt = t_end - t_begin;   // key tiles this block sweeps
+    const int nt_a = max(t_end_a - t_begin, 0);
+    const int nt_b = has_b ? max(t_end_b - t_begin, 0) : 0;
+    const int nt = max(nt_a, nt_b);                        // key tiles loaded
 
-    if ((smem_u32(smem) & 1023u) != 0) {   // layout needs 1024-byte aligned tiles
+    if ((smem_u32(smem) & 1023u) != 0) {   // the layout needs 1024-byte aligned tiles
         if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0, (int)UNIPIN_ERR_CUDA);
         return;
     }
     uint8_t* sQ = smem + C::kOffQ;
-    uint8_t* sK = smem + C::kOffK;
-    uint8_t* sV = smem + C::kOffV;
-    uint8_t* sP = smem + C::kOffP;
+    uint8_t* ring = smem + C::kOffRing;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_q = bars + 0;
-    uint64_t* bar_s = bars + 1;
-    uint64_t* bar_p = bars + 2;
-    uint64_t* bar_o = bars + 3;
-    uint64_t* bar_drain = bars + 4;
-    uint64_t* full = bars + 5;          // [NS]
-    uint64_t* empty = bars + 5 + NS;    // [NS]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5 + 2 * NS);
+    uint64_t* s_full = bars + 1;          // [2]
+    uint64_t* p_full = bars + 3;          // [2]
+    uint64_t* o_full = bars + 5;          // [2]
+    uint64_t* bar_drain = bars + 7;
+    uint64_t* kv_full = bars + 8;         // [NS]
+    uint64_t* kv_empty = bars + 8 + NS;   // [NS]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * NS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        mbar_init(bar_s, 1);
-        mbar_init(bar_p, kBlockM);
-        mbar_init(bar_o, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(s_full + x, 1);
+            mbar_init(p_full + x, kBlockM);
+            mbar_init(o_full + x, 1);
+        }
         mbar_init(bar_drain, 1);
         for (int s = 0; s < NS; ++s) {
-            mbar_init(full + s, 1);
-            mbar_init(empty + s, 1);
+            mbar_init(kv_full + s, 1);
+            mbar_init(kv_empty + s, 1);
         }
         *abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -181,95 +204,116 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem;          // 128 fp32 columns
-    const uint32_t tO = tmem + 128;    // D fp32 columns
 
     WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------------- producer
         if (lane == 0 && nt > 0) {
             tma_prefetch_map(&tm_q);
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
             int last_use[NS];
+#pragma unroll
             for (int s = 0; s < NS; ++s) last_use[s] = -1;
-            mbar_arrive_expect_tx(bar_q, C::kTileBytes);
-            for (int c = 0; c < C::kChunks; ++c)
-                tma_load_3d(sQ + c * C::kAtomBytes, &tm_q, bar_q, c * C::kBoxD, h, tok0 + qrow0);
-            const int pool_row = ((p.layer * p.S + slot) * p.H + h);
-            for (int i = 0; i < nt; ++i) {
-                const int t = t_begin + i;
-                const int st = i % NS;
-                if (i >= NS && !mbar_wait(empty + st, ((i / NS) - 1) & 1, ctl)) break;
+            mbar_arrive_expect_tx(bar_q, (has_b ? 2 : 1) * C::kTileBytes);
+            for (int x = 0; x < (has_b ? 2 : 1); ++x)
+                for (int c = 0; c < C::kChunks; ++c)
+                    tma_load_3d(sQ + x * C::kTileBytes + c * C::kAtomBytes, &tm_q, bar_q, c * C::kBoxD, h,
+                                tok0 + qrow0 + x * kBlockM);
+            const int pool_plane = (p.layer * p.S + slot) * p.H + h;
+            bool ok = true;
+            for (int i = 0; ok && i < nt; ++i) {
                 int start, lo;
-                key_tile(t, nt_all, kmax, start, lo);
-                mbar_arrive_expect_tx(full + st, 2 * C::kTileBytes);
-                uint8_t* dk = sK + st * C::kTileBytes;
-                uint8_t* dv = sV + st * C::kTileBytes;
-                for (int c = 0; c < C::kChunks; ++c) {
-                    if (kDecode) {
-                        tma_load_3d(dk + c * C::kAtomBytes, &tm_k, full + st, c * C::kBoxD, start, pool_row);
-                        tma_load_3d(dv + c * C::kAtomBytes, &tm_v, full + st, c * C::kBoxD, start, pool_row);
-                    } else {
-                        tma_load_3d(dk + c * C::kAtomBytes, &tm_k, full + st, c * C::kBoxD, h, tok0 + start);
-                        tma_load_3d(dv + c * C::kAtomBytes, &tm_v, full + st, c * C::kBoxD, h, tok0 + start);
+                key_tile(t_begin + i, nt_all, kmax, start, lo);
+                for (int w = 0; w < 2; ++w) {             // K_i then V_i
+                    const int u = 2 * i + w;
+                    const int st = u % NS;
+                    if (u >= NS && !(ok = mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl))) break;
+                    mbar_arrive_expect_tx(kv_full + st, C::kTileBytes);
+                    const CUtensorMap* map = w == 0 ? &tm_k : &tm_v;
+                    uint8_t* dst = ring + st * C::kTileBytes;
+                    for (int c = 0; c < C::kChunks; ++c) {
+                        if (kDecode)
+                            tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, start, pool_plane);
+                        else
+                            tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, h, tok0 + start);
                     }
+                    last_use[st] = u / NS;
                 }
-                last_use[st] = i / NS;
             }
             // Let every issued copy land before shared memory is released.
             mbar_wait_drain(bar_q, 0, p.wait_limit_ns);
+#pragma unroll
             for (int s = 0; s < NS; ++s)
-                if (last_use[s] >= 0) mbar_wait_drain(full + s, last_use[s] & 1, p.wait_limit_ns);
+                if (last_use[s] >= 0) mbar_wait_drain(kv_full + s, last_use[s] & 1, p.wait_limit_ns);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------------ UMMA issuer
         if (lane == 0 && nt > 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
-            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV), aP = smem_u32(sP);
-            // S = Q K^T: A = Q (K-major), B = K tile (K-major); K-steps of 16 elements (32 bytes).
-            auto issue_qk = [&](int st) {
+            const uint32_t aQ = smem_u32(sQ), aRing = smem_u32(ring);
+            // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16 elements.
+            auto issue_qk = [&](int x, int st) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk * 32 / C::kRowBytes) * C::kAtomBytes + (kk * 32) % C::kRowBytes;
-                    const uint64_t a = smem_desc(aQ + off, 16, 8 * C::kRowBytes, C::kLayout);
-                    const uint64_t b = smem_desc(aK + st * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kLayout);
-                    umma_bf16_ss(tS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint64_t a = smem_desc(aQ + x * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kLayout);
+                    const uint64_t b = smem_desc(aRing + st * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kLayout);
+                    umma_bf16_ss(tmem + x * 128, a, b, idesc_qk, kk > 0 ? 1u : 0u);
                 }
             };
-            // O += P V: A = P (K-major over keys, 128-byte swizzle, two 64-key atoms),
-            // B = V tile read MN-major (D contiguous); K-steps of 16 keys.
-            auto issue_pv = [&](int st, bool acc) {
+            // O_x += P_x V: P from TMEM (first 64 columns of S_x, 8 columns per
+            // 16 keys), V read MN-major (D contiguous); K-steps of 16 keys.
+            auto issue_pv = [&](int x, int st, bool acc) {
 #pragma unroll
                 for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    const uint32_t offp = (kk / 4) * (kBlockM * 128) + (kk % 4) * 32;
-                    const uint64_t a = smem_desc(aP + offp, 16, 1024, kLayoutSw128);
-                    const uint32_t offv = kk * 16 * C::kRowBytes;
-                    const uint64_t b = smem_desc(aV + st * C::kTileBytes + offv, C::kAtomBytes,
-                                                 8 * C::kRowBytes, C::kLayout);
-                    umma_bf16_ss(tO, a, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                    const uint64_t b = smem_desc(aRing + st * C::kTileBytes + kk * 16 * C::kRowBytes,
+                                                 C::kAtomBytes, 8 * C::kRowBytes, C::kLayout);
+                    umma_bf16_ts(tmem + 256 + x * D, tmem + x * 128 + kk * 8, b, idesc_pv,
+                                 (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            bool ok = mbar_wait(bar_q, 0, ctl);
-            for (int i = 0; ok && i < nt; ++i) {
-                if (i > 0) {
-                    if (!(ok = mbar_wait(bar_p, (i - 1) & 1, ctl))) break;
-                    tc_fence_after_sync();
-                    issue_pv((i - 1) % NS, i - 1 > 0);
-                    umma_commit(bar_o);
-                    if (i - 1 + NS < nt) umma_commit(empty + (i - 1) % NS);
+            auto slot_of = [](int u) { return u % NS; };
+            auto par_of = [](int u) { return (uint32_t)((u / NS) & 1); };
+            // the producer reuses slot u % NS for use u + NS; release only uses it will wait on
+            auto release = [&](int u) {
+                if (u + NS < 2 * nt) umma_commit(kv_empty + slot_of(u));
+            };
+            bool ok = mbar_wait(bar_q, 0, ctl) && mbar_wait(kv_full + slot_of(0), par_of(0), ctl);
+            if (ok) {
+                tc_fence_after_sync();
+                issue_qk(0, slot_of(0));
+                umma_commit(s_full + 0);
+                if (nt_b > 0) {
+                    issue_qk(1, slot_of(0));
+                    umma_commit(s_full + 1);
                 }
-                if (!(ok = mbar_wait(full + i % NS, (i / NS) & 1, ctl))) break;
-                tc_fence_after_sync();
-                issue_qk(i % NS);
-                umma_commit(bar_s);
+                release(0);
             }
-            if (ok && mbar_wait(bar_p, (nt - 1) & 1, ctl)) {
-                tc_fence_after_sync();
-                issue_pv((nt - 1) % NS, nt - 1 > 0);
-                umma_commit(bar_o);
+            for (int i = 0; ok && i < nt; ++i) {
+                const int uv = 2 * i + 1;      // V_i
+                const int uk = 2 * i + 2;      // K_{i+1}
+                if (!(ok = mbar_wait(kv_full + slot_of(uv), par_of(uv), ctl))) break;
+                for (int x = 0; x < 2; ++x) {
+                    const int ntx = x == 0 ? nt_a : nt_b;
+                    if (i >= ntx) continue;
+                    if (!(ok = mbar_wait(p_full + x, i & 1, ctl))) break;
+                    tc_fence_after_sync();
+                    issue_pv(x, slot_of(uv), i > 0);
+                    if (i + 1 < ntx) {
+                        if (!(ok = mbar_wait(kv_full + slot_of(uk), par_of(uk), ctl))) break;
+                        tc_fence_after_sync();
+                        issue_qk(x, slot_of(uk));
+                        umma_commit(s_full + x);
+                    } else {
+                        umma_commit(o_full + x);
+                    }
+                }
+                if (!ok) break;
+                release(uv);
+                if (i + 1 < nt) release(uk);
             }
             // Every MMA issued above completes before TMEM is released.
             umma_commit(bar_drain);
@@ -277,99 +321,94 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
         }
     } else {
         // ------------------------------------------------ softmax + epilogue
-        const int r = threadIdx.x;                       // query row in the tile
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        const int irow = causal0 + r;                    // mask position of this row
+        const int x = warp / 4;                            // 0: tile A, 1: tile B
+        const int r = threadIdx.x - x * kBlockM;           // query row in the tile
+        const int ntx = x == 0 ? nt_a : nt_b;
+        const int nrows_x = x == 0 ? nrows_a : nrows_b;
+        const int kmax_x = x == 0 ? kmax_a : kmax_b;
+        const int posx0 = pos0 + x * kBlockM;              // mask position of row 0 of this tile
+        const int irow = posx0 + r;
+        const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
+        const uint32_t tS = tmem + x * 128 + lane_off;
+        const uint32_t tO = tmem + 256 + x * D + lane_off;
         const float sl2 = p.sl2;
-        float m = -INFINITY;                             // running max, log2 units
-        float l = 0.f;                                   // running sum
-        bool ok = true;
-        for (int i = 0; i < nt; ++i) {
-            const int t = t_begin + i;
+        float m = -INFINITY;     // reference max (log2 units) the P values and O are relative to
+        float l = 0.f;           // row sum relative to m
+        bool ok = nrows_x > 0;
+        for (int i = 0; ok && i < ntx; ++i) {
             int start, lo;
-            key_tile(t, nt_all, kmax, start, lo);
-            const bool full_tile = (start == lo) && (start + kBlockN <= kmax) && (start + kBlockN - 1 <= causal0);
-            // Waits are made warp-uniform: the TMEM loads below are warp-collective.
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_s, i & 1, ctl));
+            key_tile(t_begin + i, nt_all, kmax, start, lo);
+            const bool full_tile = (start == lo) && (start + kBlockN <= kmax_x) && (start + kBlockN - 1 <= posx0);
+            // warp-uniform: the TMEM accesses below are warp-collective
+            ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, i & 1, ctl));
             if (!ok) break;
             tc_fence_after_sync();
-            // pass 1: row max of the allowed scores
-            float mx = -INFINITY;
+            uint32_t s[kBlockN];
+            tmem_ld128(tS, s);
+            if (!full_tile) {
 #pragma unroll
-            for (int c4 = 0; c4 < kBlockN / 32; ++c4) {
-                uint32_t v[32];
-                tmem_ld32(tS + lane_off + c4 * 32, v);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int j = start + c4 * 32 + e;
-                    const bool allow = full_tile || (j >= lo && j < kmax && j <= irow);
-                    if (allow) mx = fmaxf(mx, __uint_as_float(v[e]));
+                for (int e = 0; e < kBlockN; ++e) {
+                    const int j = start + e;
+                    if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
                 }
             }
-            const float m_new = fmaxf(m, mx * sl2);
-            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-            if (i > 0) {
-                // P buffer and O are only touched after the previous P.V finished.
-                ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (i - 1) & 1, ctl));
-                if (!ok) break;
-                tc_fence_after_sync();
-                // The TMEM load/store below are warp-collective, so the branch is
-                // taken by the whole warp when any row's max grew; rows whose
-                // max did not grow scale by 1.
-                if (__any_sync(0xffffffffu, m_new > m)) {
-                    const float corr = (m_new > m) ? ex2_approx(m - m_use) : 1.f;
-                    l *= corr;
+            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < kBlockN; e += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(s[e]));
+                mx1 = fmaxf(mx1, __uint_as_float(s[e + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(s[e + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(s[e + 3]));
+            }
+            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+            // Lazy rescale: move the reference max only when some row of the
+            // warp would otherwise see P > 2^8; then every row moves to its own max.
+            const bool need = m_tile > m + kRescaleLog2;
+            if (__any_sync(0xffffffffu, need)) {
+                const float m_new = fmaxf(m, m_tile);
+                const float corr = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+                if (i > 0) {
+                    // O_x is stable: the P.V of the previous tile completed before S of this one.
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(tO + lane_off + c * 32, o);
+                        tmem_ld32(tO + c * 32, o);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-                        tmem_st32(tO + lane_off + c * 32, o);
+                        tmem_st32(tO + c * 32, o);
                     }
                 }
+                l *= corr;
+                m = m_new;
             }
-            // pass 2: P = 2^(s*scale*log2e - m), rounded to bf16; row sum of the rounded values
-            float ls = 0.f;
-            uint8_t* prow = sP + r * 128;
+            const float m_use = (m == -INFINITY) ? 0.f : m;
+            uint32_t pk[kBlockN / 2];
+            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
-            for (int c4 = 0; c4 < kBlockN / 32; ++c4) {
-                uint32_t v[32];
-                tmem_ld32(tS + lane_off + c4 * 32, v);
-                uint32_t pk[16];
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    const int j = start + c4 * 32 + e;
-                    const bool a0 = full_tile || (j >= lo && j < kmax && j <= irow);
-                    const bool a1 = full_tile || (j + 1 >= lo && j + 1 < kmax && j + 1 <= irow);
-                    const float p0 = a0 ? ex2_approx(fmaf(__uint_as_float(v[e]), sl2, -m_use)) : 0.f;
-                    const float p1 = a1 ? ex2_approx(fmaf(__uint_as_float(v[e + 1]), sl2, -m_use)) : 0.f;
-                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-                    ls += __low2float(b2) + __high2float(b2);
-                    pk[e / 2] = *reinterpret_cast<const uint32_t*>(&b2);
-                }
-                // keys c4*32 .. c4*32+31 live in 64-key atom (c4/2), 16-byte chunks (c4%2)*4 .. +3
-                uint8_t* atom = prow + (c4 / 2) * (kBlockM * 128);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int chunk = ((c4 % 2) * 4 + q) ^ (r & 7);
-                    *reinterpret_cast<uint4*>(atom + chunk * 16) =
-                        make_uint4(pk[4 * q + 0], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                }
+            for (int e = 0; e < kBlockN; e += 4) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(s[e]), sl2, -m_use));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(s[e + 1]), sl2, -m_use));
+                const float p2 = ex2_approx(fmaf(__uint_as_float(s[e + 2]), sl2, -m_use));
+                const float p3 = ex2_approx(fmaf(__uint_as_float(s[e + 3]), sl2, -m_use));
+                l0 += p0;
+                l1 += p1;
+                l2 += p2;
+                l3 += p3;
+                pk[e / 2] = pack_bf16x2(p0, p1);
+                pk[e / 2 + 1] = pack_bf16x2(p2, p3);
             }
-            l += ls;
-            m = m_new;
-            fence_proxy_async_smem();
+            l += (l0 + l1) + (l2 + l3);
+            tmem_st64(tS, pk);                             // P over the first 64 columns of S
             tc_fence_before_sync();
-            mbar_arrive(bar_p);
+            mbar_arrive(p_full + x);
         }
-        if (ok && nt > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_o, (nt - 1) & 1, ctl));
+        if (ok && ntx > 0) {
+            ok = __all_sync(0xffffffffu, mbar_wait(o_full + x, 0, ctl));
             tc_fence_after_sync();
         }
         if (ok) {
-            const bool row_valid = r < nrows;
-            const long long tok = (long long)tok0 + qrow0 + r;
+            const bool row_valid = r < nrows_x;
+            const long long tok = (long long)tok0 + qrow0 + x * kBlockM + r;
             const size_t base = ((size_t)tok * p.H + h) * D;
             const bool split_mode = kDecode && p.nsplit > 1;
             // self term: a candidate row's own key (prefill rows i >= n_b; every decode row)
@@ -380,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
                 if (self) {
                     const uint4* q4 = reinterpret_cast<const uint4*>(p.q + base);
                     const uint4* k4 = reinterpret_cast<const uint4*>(p.k_self + base);
-                    float dot = 0.f;
+                    float dot0 = 0.f, dot1 = 0.f;
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) {
                         const uint4 qa = q4[c], ka = k4[c];
@@ -390,11 +429,11 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
                         for (int e = 0; e < 4; ++e) {
                             const float2 qf = __bfloat1622float2(qh[e]);
                             const float2 kf = __bfloat1622float2(kh[e]);
-                            dot = fmaf(qf.x, kf.x, dot);
-                            dot = fmaf(qf.y, kf.y, dot);
+                            dot0 = fmaf(qf.x, kf.x, dot0);
+                            dot1 = fmaf(qf.y, kf.y, dot1);
                         }
                     }
-                    ss = dot * sl2;
+                    ss = (dot0 + dot1) * sl2;
                 }
                 const float m_fin = fmaxf(m, ss);
                 a = (m == -INFINITY) ? 0.f : ex2_approx(m - m_fin);
@@ -405,8 +444,8 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
-                if (nt > 0) {
-                    tmem_ld32(tO + lane_off + c * 32, o);   // warp-collective: every lane loads
+                if (ntx > 0) {
+                    tmem_ld32(tO + c * 32, o);   // warp-collective: every lane loads
                 } else {
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = 0u;
@@ -447,18 +486,10 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
                 } else {
                     __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + base + c * 32;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 8) {
-                        uint4 w;
-                        __nv_bfloat162 b0 = __floats2bfloat162_rn(res[e], res[e + 1]);
-                        __nv_bfloat162 b1 = __floats2bfloat162_rn(res[e + 2], res[e + 3]);
-                        __nv_bfloat162 b2 = __floats2bfloat162_rn(res[e + 4], res[e + 5]);
-                        __nv_bfloat162 b3 = __floats2bfloat162_rn(res[e + 6], res[e + 7]);
-                        w.x = *reinterpret_cast<uint32_t*>(&b0);
-                        w.y = *reinterpret_cast<uint32_t*>(&b1);
-                        w.z = *reinterpret_cast<uint32_t*>(&b2);
-                        w.w = *reinterpret_cast<uint32_t*>(&b3);
-                        *reinterpret_cast<uint4*>(dst + e) = w;
-                    }
+                    for (int e = 0; e < 32; e += 8)
+                        *reinterpret_cast<uint4*>(dst + e) =
+                            make_uint4(pack_bf16x2(res[e], res[e + 1]), pack_bf16x2(res[e + 2], res[e + 3]),
+                                       pack_bf16x2(res[e + 4], res[e + 5]), pack_bf16x2(res[e + 6], res[e + 7]));
                 }
             }
             if (split_mode && row_valid) {
@@ -471,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, AttnCfg<D>::kMinBlocks)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         __syncwarp();
         tc_fence_after_sync();
         tmem_dealloc(tmem, kTmemCols);

@@ -172,8 +172,8 @@ int launch_pool_write(const unipin_kvpool* pool, int layer, const void* k, const
 int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
 {
     if (R < 1 || H < 1 || max_k < 1 || n_cap < 1) return 1;
-    const long long units = (long long)R * H * ((max_k + kBlockM - 1) / kBlockM);
-    const long long slots = (long long)kNumSmsHint * (D <= 64 ? 2 : 1);
+    const long long units = (long long)R * H * ((max_k + 2 * kBlockM - 1) / (2 * kBlockM));
+    const long long slots = (long long)kNumSmsHint;   // one block per SM (all of TMEM)
     const long long target = 4 * slots;
     if (units >= slots) return 1;
     const int key_tiles = (n_cap + kBlockN - 1) / kBlockN;
@@ -271,7 +271,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.sl2 = scale * kLog2e;
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
-    dim3 grid((unsigned)((max_seqlen + kBlockM - 1) / kBlockM), (unsigned)H, (unsigned)B);
+    dim3 grid((unsigned)((max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM)), (unsigned)H, (unsigned)B);
     return launch_attn<false>(D, grid, tq, tk, tv, p, s);
 }
 
@@ -351,8 +351,8 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
         p.part_o = static_cast<float*>(workspace);
         p.part_ml = p.part_o + (size_t)nsplit * total_cand * H * D;
     }
-    const unsigned qtiles = (unsigned)((max_k + kBlockM - 1) / kBlockM);
-    dim3 grid(qtiles * (unsigned)nsplit, (unsigned)H, (unsigned)R);
+    const unsigned qpairs = (unsigned)((max_k + 2 * kBlockM - 1) / (2 * kBlockM));
+    dim3 grid(qpairs * (unsigned)nsplit, (unsigned)H, (unsigned)R);
     rc = launch_attn<true>(D, grid, tq, tk, tv, p, s);
     if (rc != UNIPIN_OK || nsplit == 1) return rc;
 
