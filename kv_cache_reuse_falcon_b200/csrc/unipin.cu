@@ -175,7 +175,7 @@ int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
     const long long units = (long long)R * H * ((max_k + 2 * kBlockM - 1) / (2 * kBlockM));
     const long long slots = (long long)kNumSmsHint;   // one block per SM (all of TMEM)
     const long long target = 4 * slots;
-    if (units >= slots) return 1;
+    if (units >= 2 * slots) return 1;   // two or more waves already: no split
     const int key_tiles = (n_cap + kBlockN - 1) / kBlockN;
     long long ns = (target + units - 1) / units;
     const long long cap = key_tiles / 2 > 1 ? key_tiles / 2 : 1;   // at least two key tiles per split
