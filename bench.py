@@ -336,7 +336,9 @@ def run_ours(args, rank, world, device, dist):
     dec_tflops = df / (dec_ms * 1e-3) / 1e12
     dec_gbs = db / (dec_ms * 1e-3) / 1e9
     pool_gbs = pwb / (pool_ms * 1e-3) / 1e9
-    peak = peaks["bf16_tflops_sustained"]
+    # The prefill kernel runs for milliseconds inside a sub-second timed region at
+    # full clock, so the burst GEMM figure is its denominator (the stricter one).
+    peak = peaks["bf16_tflops"]
     result = {
         "metric": METRIC,
         "value": cand_total / (ms_step * 1e-3),
@@ -359,11 +361,12 @@ def run_ours(args, rank, world, device, dist):
                    "prefill_tflops": pre_tflops, "decode_tflops": dec_tflops, "decode_gbs": dec_gbs,
                    "pool_write_gbs": pool_gbs,
                    "prefill_frac_tensor": pre_tflops / peak,
+                   "prefill_frac_tensor_sustained": pre_tflops / peaks["bf16_tflops_sustained"],
                    "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
                    "pool_write_frac_hbm": pool_gbs / peaks["hbm_gbs"]},
         "roofline": {"kernel": "attn_fwd_kernel<128,prefill>", "bound": "tensor", "achieved": pre_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": pre_tflops / peak, "traffic": None,
-                     "peak_source": "%s bf16_tflops_sustained" % peaks["source"],
+                     "peak_source": "%s bf16_tflops (burst)" % peaks["source"],
                      "work_per_launch": "4*D*H*sum_b[n_b(n_b+1)/2 + k_b(n_b+1)] = %.4g FLOP" % pf},
         "e2e": {"value": cand_total / (e2e_ms * 1e-3), "unit": "candidate tokens/s",
                 "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
