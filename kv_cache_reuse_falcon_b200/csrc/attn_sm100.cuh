@@ -1,9 +1,12 @@
 // M-FALCON masked attention engine for sm_100a.
 //
-// One thread block per (segment, head, pair of 128-row query tiles A and B).
+// Work item = (segment, head, pair of 128-row query tiles A and B[, key split]).
 // The two tiles share every K/V tile and run as a ping-pong: while the
 // tensor cores work on one tile's S = Q K^T and O += P V, the other tile's
-// softmax warpgroup turns its scores into probabilities.
+// softmax warpgroup turns its scores into probabilities.  Blocks are
+// persistent (one per SM): each walks its share of the items, and the next
+// item's Q and first K/V tiles load, and its first S MMAs run, while the
+// softmax warpgroups finish the previous item's epilogue.
 //
 // The same engine runs the prefill and the rank decode.  In both, the part
 // of a row's key set that is a contiguous run of keys 0..kmax-1 goes through
@@ -17,7 +20,7 @@
 // Key tiles past kmax are never visited; key tiles entirely below the
 // diagonal and below kmax skip the per-element predicate.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns
 //              query row r = TMEM lane r, so the row max and row sum stay in
 //              one thread's registers; S is read from TMEM with one wide load,
@@ -25,9 +28,11 @@
 //              there by the P.V MMA.  The O accumulator is rescaled in TMEM
 //              only when a row max grows by more than 2^8 (stale maxima keep
 //              P <= 2^8, exact after the final division).
-//   warp 8     TMA producer: Q tiles once, then K_0, V_0, K_1, V_1, ... through
-//              a ring of shared-memory slots.
+//   warp 8     TMA producer: per item the Q tiles, then K_0, V_0, K_1, V_1, ...
+//              through a ring of shared-memory slots (the ring runs across items).
 //   warp 9     TMEM allocator and the single UMMA-issuing thread.
+//   warps 10-11 idle (they complete the third warpgroup for the register split).
+// Every warp walks the same item sequence (ItemWalker), so no queue is shared.
 //
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B [256+D, 256+2D);
 // P_X occupies the first 64 columns of S_X.
@@ -41,7 +46,15 @@ namespace unipin {
 
 constexpr int kBlockM = 128;     // query rows per tile = TMEM lanes
 constexpr int kBlockN = 128;     // keys per tile
-constexpr int kThreads = 320;
+constexpr int kPairRows = 2 * kBlockM;
+constexpr int kThreads = 384;
+// Register split: the block launches with kLaunchRegs per thread (the most
+// 384 threads can have); the producer/MMA warpgroup gives registers back and
+// the two softmax warpgroups take them: 128*72 + 256*216 = 384*168.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsOther = 96;
+constexpr int kRegsSoftmax = 200;
+static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when a row max grows by > 2^8
@@ -72,8 +85,9 @@ struct AttnParams {
     const int* cu;                // [nseg + 1]
     const int* past;              // [nseg]
     const int* slots;             // [nseg] (decode)
+    int nseg;
     int H;
-    int max_rows;                 // host bound on rows per segment (grid size)
+    int max_rows;                 // host bound on rows per segment
     int total_rows;               // T
     int out_fp32;
     int layer, S, n_cap;          // pool geometry (decode)
@@ -99,6 +113,143 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
+__device__ __forceinline__ void report(int* status, int code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+// Warp-cooperative walk over the work items of this block: item g (global,
+// segment-major) belongs to block g % gridDim.x.  Every lane of the calling
+// warp must call next() together; all lanes get the same answer.
+struct ItemWalker {
+    const int* cu;
+    int nseg, max_rows, mult;     // mult = items per query-tile pair
+    int c0;                       // first segment of the loaded chunk of 32
+    long long base;               // items before segment c0
+    int cnt, pre;                 // this lane's segment: item count, exclusive prefix in chunk
+    int chunk_total;
+    long long g;
+    int* status;
+
+    __device__ void load_chunk(int lane)
+    {
+        const int s = c0 + lane;
+        int items = 0;
+        if (s < nseg) {
+            const int len = cu[s + 1] - cu[s];
+            if (len < 0 || len > max_rows) {
+                report(status, (int)UNIPIN_ERR_OUT_OF_RANGE);   // such a segment yields no item
+            } else {
+                items = ((len + kPairRows - 1) / kPairRows) * mult;
+            }
+        }
+        int incl = items;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        cnt = items;
+        pre = incl - items;
+        chunk_total = __shfl_sync(0xffffffffu, incl, 31);
+    }
+
+    __device__ void init(const AttnParams& p, int lane)
+    {
+        cu = p.cu;
+        nseg = p.nseg;
+        max_rows = p.max_rows;
+        mult = p.H * p.nsplit;
+        status = p.status;
+        c0 = 0;
+        base = 0;
+        g = blockIdx.x;
+        load_chunk(lane);
+    }
+
+    // Next item of this block: its segment and index within the segment.
+    __device__ bool next(int lane, int& seg, int& local)
+    {
+        while (g >= base + chunk_total) {
+            if (c0 + 32 >= nseg) return false;
+            base += chunk_total;
+            c0 += 32;
+            load_chunk(lane);
+        }
+        const long long rel = g - base;
+        const unsigned hit = __ballot_sync(0xffffffffu, cnt > 0 && rel >= pre && rel < pre + cnt);
+        const int L = __ffs(hit) - 1;
+        seg = c0 + L;
+        local = (int)(rel - __shfl_sync(0xffffffffu, pre, L));
+        g += gridDim.x;
+        return true;
+    }
+};
+
+// Everything about one item that every role derives identically.
+struct Work {
+    bool valid;
+    int seg, h, split;
+    int tok0, npast, slot;
+    int qrow0;                  // first row of tile A within the segment
+    int nrows_a, nrows_b;       // rows of tile A / B (B may have none)
+    bool has_b;
+    int pos0;                   // mask position of row 0 of tile A
+    int kmax_a, kmax_b, kmax;   // key ranges; tile geometry follows kmax
+    int nt_all, t_begin;
+    int nt_a, nt_b, nt;         // key tiles swept for A, B, and loaded
+};
+
+template <bool kDecode>
+__device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int local)
+{
+    Work w;
+    w.seg = seg;
+    const int per_pair = p.H * p.nsplit;
+    const int pair_rank = local / per_pair;
+    const int rest = local - pair_rank * per_pair;
+    w.h = rest / p.nsplit;
+    w.split = rest - w.h * p.nsplit;
+    w.tok0 = p.cu[seg];
+    const int nrows_seg = p.cu[seg + 1] - w.tok0;
+    w.npast = p.past[seg];
+    w.slot = kDecode ? p.slots[seg] : 0;
+    bool bad = w.tok0 < 0 || w.npast < 0 || (long long)w.tok0 + nrows_seg > (long long)p.total_rows;
+    if (kDecode)
+        bad = bad || w.slot < 0 || w.slot >= p.S || w.npast > p.n_cap;
+    else
+        bad = bad || w.npast > nrows_seg;
+    w.valid = !bad;
+    const int npairs = (nrows_seg + kPairRows - 1) / kPairRows;
+    // Prefill: the costliest pair of a segment (the last) comes first.
+    const int qp = kDecode ? pair_rank : (npairs - 1 - pair_rank);
+    w.qrow0 = qp * kPairRows;
+    w.nrows_a = min(kBlockM, nrows_seg - w.qrow0);
+    w.nrows_b = min(kBlockM, nrows_seg - w.qrow0 - kBlockM);
+    w.has_b = w.nrows_b > 0;
+    w.pos0 = kDecode ? w.npast + w.qrow0 : w.qrow0;
+    w.kmax_a = kDecode ? w.npast : min(w.qrow0 + w.nrows_a, w.npast);
+    w.kmax_b = !w.has_b ? 0 : (kDecode ? w.npast : min(w.qrow0 + kBlockM + w.nrows_b, w.npast));
+    // Tile A's range is a prefix of B's with identical tiles (kmax_a < kmax_b
+    // only when kmax_a is a multiple of 128).
+    w.kmax = w.has_b ? w.kmax_b : w.kmax_a;
+    w.nt_all = (w.kmax + kBlockN - 1) / kBlockN;
+    w.t_begin = 0;
+    int t_end_a = (w.kmax_a + kBlockN - 1) / kBlockN;
+    int t_end_b = (w.kmax_b + kBlockN - 1) / kBlockN;
+    if (kDecode && p.nsplit > 1) {
+        const int per = (w.nt_all + p.nsplit - 1) / p.nsplit;
+        w.t_begin = min(w.split * per, w.nt_all);
+        t_end_a = min(w.t_begin + per, t_end_a);
+        t_end_b = min(w.t_begin + per, t_end_b);
+    }
+    w.nt_a = max(t_end_a - w.t_begin, 0);
+    w.nt_b = w.has_b ? max(t_end_b - w.t_begin, 0) : 0;
+    w.nt = w.valid ? max(w.nt_a, w.nt_b) : 0;
+    if (!w.valid) w.nt_a = w.nt_b = 0;
+    return w;
+}
+
 template <int D, bool kDecode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -110,79 +261,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
-    const int seg = blockIdx.z;
-    const int h = blockIdx.y;
 
     // A timeout recorded earlier means a block of this or a previous launch
     // gave up; later blocks skip their work instead of waiting again.
     if (p.status && *reinterpret_cast<volatile int*>(p.status) == (int)UNIPIN_ERR_DEVICE_TIMEOUT) return;
-
-    // ------------------------------------------------------------ work unit
-    const int tok0 = p.cu[seg];
-    const int nrows_seg = p.cu[seg + 1] - tok0;
-    const int npast = p.past[seg];
-    int slot = 0;
-    bool bad = tok0 < 0 || nrows_seg < 0 || nrows_seg > p.max_rows || npast < 0 ||
-               (long long)tok0 + nrows_seg > (long long)p.total_rows;
-    if (kDecode) {
-        slot = p.slots[seg];
-        bad = bad || slot < 0 || slot >= p.S || npast > p.n_cap;
-    } else {
-        bad = bad || npast > nrows_seg;
-    }
-    if (bad) {
-        if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0, (int)UNIPIN_ERR_OUT_OF_RANGE);
-        return;
-    }
-    const int npairs = (nrows_seg + 2 * kBlockM - 1) / (2 * kBlockM);
-    const int split = kDecode ? (int)(blockIdx.x % p.nsplit) : 0;
-    const int pidx = kDecode ? (int)(blockIdx.x / p.nsplit) : (int)blockIdx.x;
-    if (pidx >= npairs) return;
-    // Prefill: the costliest pair of a segment (the last) launches first.
-    const int qp = kDecode ? pidx : (npairs - 1 - pidx);
-    const int qrow0 = qp * 2 * kBlockM;                    // first row of tile A
-    const int nrows_a = min(kBlockM, nrows_seg - qrow0);
-    const int nrows_b = min(kBlockM, nrows_seg - qrow0 - kBlockM);
-    const bool has_b = nrows_b > 0;
-    const int pos0 = kDecode ? npast + qrow0 : qrow0;      // mask position of row 0 of tile A
-    const int kmax_a = kDecode ? npast : min(qrow0 + nrows_a, npast);
-    const int kmax_b = !has_b ? 0 : (kDecode ? npast : min(qrow0 + kBlockM + nrows_b, npast));
-    // Tile geometry follows the longer key range; tile A's range is a prefix of
-    // it with identical tiles (kmax_a < kmax_b only when kmax_a is a multiple of 128).
-    const int kmax = has_b ? kmax_b : kmax_a;
-    const int nt_all = (kmax + kBlockN - 1) / kBlockN;
-    int t_begin = 0;
-    int t_end_a = (kmax_a + kBlockN - 1) / kBlockN;
-    int t_end_b = (kmax_b + kBlockN - 1) / kBlockN;
-    if (kDecode && p.nsplit > 1) {
-        const int per = (nt_all + p.nsplit - 1) / p.nsplit;
-        t_begin = min(split * per, nt_all);
-        t_end_a = min(t_begin + per, t_end_a);
-        t_end_b = min(t_begin + per, t_end_b);
-    }
-    const int nt_a = max(t_end_a - t_begin, 0);
-    const int nt_b = has_b ? max(t_end_b - t_begin, 0) : 0;
-    const int nt = max(nt_a, nt_b);                        // key tiles loaded
-
     if ((smem_u32(smem) & 1023u) != 0) {   // the layout needs 1024-byte aligned tiles
-        if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0, (int)UNIPIN_ERR_CUDA);
+        if (threadIdx.x == 0) report(p.status, (int)UNIPIN_ERR_CUDA);
         return;
     }
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* ring = smem + C::kOffRing;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-    uint64_t* bar_q = bars + 0;
-    uint64_t* s_full = bars + 1;          // [2]
-    uint64_t* p_full = bars + 3;          // [2]
-    uint64_t* o_full = bars + 5;          // [2]
-    uint64_t* bar_drain = bars + 7;
-    uint64_t* kv_full = bars + 8;         // [NS]
-    uint64_t* kv_empty = bars + 8 + NS;   // [NS]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 8 + 2 * NS);
+    uint64_t* bar_q = bars + 0;           // Q tiles of the current item landed
+    uint64_t* q_empty = bars + 1;         // every S MMA of an item finished with Q
+    uint64_t* s_full = bars + 2;          // [2]
+    uint64_t* p_full = bars + 4;          // [2]
+    uint64_t* o_full = bars + 6;          // [2]
+    uint64_t* bar_drain = bars + 8;
+    uint64_t* kv_full = bars + 9;         // [NS]
+    uint64_t* kv_empty = bars + 9 + NS;   // [NS]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * NS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
+        mbar_init(q_empty, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full + x, 1);
             mbar_init(p_full + x, kBlockM);
@@ -206,235 +309,306 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = *tmem_slot;
 
     WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
+    ItemWalker walk;
+    walk.init(p, lane);
+    int seg, local;
 
-    if (warp == 8) {
+    // The producer and MMA warps run their loops with all 32 lanes (the item
+    // walker is warp-collective); waits are taken by every lane and made
+    // warp-uniform, and only lane 0 issues copies, MMAs and commits.
+    const bool leader = lane == 0;
+    if (warp >= 8) {
+      setmaxnreg_dec<kRegsOther>();   // all four warps of the third warpgroup
+      if (warp == 8) {
         // ------------------------------------------------------- producer
-        if (lane == 0 && nt > 0) {
+        if (leader) {
             tma_prefetch_map(&tm_q);
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
-            int last_use[NS];
-#pragma unroll
-            for (int s = 0; s < NS; ++s) last_use[s] = -1;
-            mbar_arrive_expect_tx(bar_q, (has_b ? 2 : 1) * C::kTileBytes);
-            for (int x = 0; x < (has_b ? 2 : 1); ++x)
-                for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sQ + x * C::kTileBytes + c * C::kAtomBytes, &tm_q, bar_q, c * C::kBoxD, h,
-                                tok0 + qrow0 + x * kBlockM);
-            const int pool_plane = (p.layer * p.S + slot) * p.H + h;
-            bool ok = true;
-            for (int i = 0; ok && i < nt; ++i) {
+        }
+        int u = 0;          // ring uses issued so far (use u lives in slot u % NS)
+        int nq = 0;         // Q loads issued so far
+        bool ok = true;
+        while (ok && walk.next(lane, seg, local)) {
+            const Work w = make_work<kDecode>(p, seg, local);
+            if (!w.valid) {
+                if (leader) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
+                continue;
+            }
+            if (w.nt == 0) continue;
+            // Q of this item may overwrite Q of the previous one once its S MMAs are done.
+            if (nq > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (nq - 1) & 1, ctl));
+                if (!ok) break;
+            }
+            if (leader) {
+                mbar_arrive_expect_tx(bar_q, (w.has_b ? 2 : 1) * C::kTileBytes);
+                for (int x = 0; x < (w.has_b ? 2 : 1); ++x)
+                    for (int c = 0; c < C::kChunks; ++c)
+                        tma_load_3d(sQ + x * C::kTileBytes + c * C::kAtomBytes, &tm_q, bar_q, c * C::kBoxD, w.h,
+                                    w.tok0 + w.qrow0 + x * kBlockM);
+            }
+            ++nq;
+            const int pool_plane = (p.layer * p.S + w.slot) * p.H + w.h;
+            for (int i = 0; ok && i < w.nt; ++i) {
                 int start, lo;
-                key_tile(t_begin + i, nt_all, kmax, start, lo);
-                for (int w = 0; w < 2; ++w) {             // K_i then V_i
-                    const int u = 2 * i + w;
+                key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
+                for (int kv = 0; kv < 2; ++kv) {          // K_i then V_i
                     const int st = u % NS;
-                    if (u >= NS && !(ok = mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl))) break;
-                    mbar_arrive_expect_tx(kv_full + st, C::kTileBytes);
-                    const CUtensorMap* map = w == 0 ? &tm_k : &tm_v;
-                    uint8_t* dst = ring + st * C::kTileBytes;
-                    for (int c = 0; c < C::kChunks; ++c) {
-                        if (kDecode)
-                            tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, start, pool_plane);
-                        else
-                            tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, h, tok0 + start);
+                    if (u >= NS) {
+                        ok = __all_sync(0xffffffffu, mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl));
+                        if (!ok) break;
                     }
-                    last_use[st] = u / NS;
+                    if (leader) {
+                        mbar_arrive_expect_tx(kv_full + st, C::kTileBytes);
+                        const CUtensorMap* map = kv == 0 ? &tm_k : &tm_v;
+                        uint8_t* dst = ring + st * C::kTileBytes;
+                        for (int c = 0; c < C::kChunks; ++c) {
+                            if (kDecode)
+                                tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, start,
+                                            pool_plane);
+                            else
+                                tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, w.h,
+                                            w.tok0 + start);
+                        }
+                    }
+                    ++u;
                 }
             }
-            // Let every issued copy land before shared memory is released.
-            mbar_wait_drain(bar_q, 0, p.wait_limit_ns);
-#pragma unroll
-            for (int s = 0; s < NS; ++s)
-                if (last_use[s] >= 0) mbar_wait_drain(kv_full + s, last_use[s] & 1, p.wait_limit_ns);
+        }
+        if (leader) {
+            // Consume the last arrival of every barrier the MMA thread signals to
+            // this warp, so nothing lands in shared memory after the block exits.
+            if (nq > 0) mbar_wait_drain(q_empty, (nq - 1) & 1, p.wait_limit_ns);
+            for (int v = (u > NS ? u - NS : 0); v < u; ++v)
+                mbar_wait_drain(kv_empty + v % NS, (v / NS) & 1, p.wait_limit_ns);
         }
     } else if (warp == 9) {
         // ------------------------------------------------------ UMMA issuer
-        if (lane == 0 && nt > 0) {
-            constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
-            const uint32_t aQ = smem_u32(sQ), aRing = smem_u32(ring);
-            // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16 elements.
-            auto issue_qk = [&](int x, int st) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
+        // Descriptors are built once; a K-step moves only the start-address
+        // field (low 14 bits, in 16-byte units), by compile-time offsets.
+        const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dk0 = smem_desc(smem_u32(ring), 16, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dv0 = smem_desc(smem_u32(ring), C::kAtomBytes, 8 * C::kRowBytes, C::kLayout);
+        // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16 elements.
+        auto issue_qk = [&](int x, int st) {
+            const uint64_t a0 = dq0 + (uint64_t)((x * C::kTileBytes) >> 4);
+            const uint64_t b0 = dk0 + (uint64_t)((st * C::kTileBytes) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk * 32 / C::kRowBytes) * C::kAtomBytes + (kk * 32) % C::kRowBytes;
-                    const uint64_t a = smem_desc(aQ + x * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kLayout);
-                    const uint64_t b = smem_desc(aRing + st * C::kTileBytes + off, 16, 8 * C::kRowBytes, C::kLayout);
-                    umma_bf16_ss(tmem + x * 128, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-                }
-            };
-            // O_x += P_x V: P from TMEM (first 64 columns of S_x, 8 columns per
-            // 16 keys), V read MN-major (D contiguous); K-steps of 16 keys.
-            auto issue_pv = [&](int x, int st, bool acc) {
-#pragma unroll
-                for (int kk = 0; kk < kBlockN / 16; ++kk) {
-                    const uint64_t b = smem_desc(aRing + st * C::kTileBytes + kk * 16 * C::kRowBytes,
-                                                 C::kAtomBytes, 8 * C::kRowBytes, C::kLayout);
-                    umma_bf16_ts(tmem + 256 + x * D, tmem + x * 128 + kk * 8, b, idesc_pv,
-                                 (acc || kk > 0) ? 1u : 0u);
-                }
-            };
-            auto slot_of = [](int u) { return u % NS; };
-            auto par_of = [](int u) { return (uint32_t)((u / NS) & 1); };
-            // the producer reuses slot u % NS for use u + NS; release only uses it will wait on
-            auto release = [&](int u) {
-                if (u + NS < 2 * nt) umma_commit(kv_empty + slot_of(u));
-            };
-            bool ok = mbar_wait(bar_q, 0, ctl) && mbar_wait(kv_full + slot_of(0), par_of(0), ctl);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_qk(0, slot_of(0));
-                umma_commit(s_full + 0);
-                if (nt_b > 0) {
-                    issue_qk(1, slot_of(0));
-                    umma_commit(s_full + 1);
-                }
-                release(0);
+            for (int kk = 0; kk < D / 16; ++kk) {
+                constexpr int kStep = 32;
+                const uint32_t off = ((kk * kStep / C::kRowBytes) * C::kAtomBytes + (kk * kStep) % C::kRowBytes) >> 4;
+                umma_bf16_ss(tmem + x * 128, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
             }
-            for (int i = 0; ok && i < nt; ++i) {
-                const int uv = 2 * i + 1;      // V_i
-                const int uk = 2 * i + 2;      // K_{i+1}
-                if (!(ok = mbar_wait(kv_full + slot_of(uv), par_of(uv), ctl))) break;
+            umma_commit(s_full + x);
+        };
+        // O_x += P_x V: P from TMEM (first 64 columns of S_x, 8 columns per
+        // 16 keys), V read MN-major (D contiguous); K-steps of 16 keys.
+        auto issue_pv = [&](int x, int st, bool acc) {
+            const uint64_t b0 = dv0 + (uint64_t)((st * C::kTileBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kBlockN / 16; ++kk) {
+                const uint32_t off = (kk * 16 * C::kRowBytes) >> 4;
+                umma_bf16_ts(tmem + 256 + x * D, tmem + x * 128 + kk * 8, b0 + off, idesc_pv,
+                             (acc || kk > 0) ? 1u : 0u);
+            }
+        };
+        int u = 0;                 // ring uses consumed
+        int nq = 0;                // items with MMAs
+        int np[2] = {0, 0};        // p_full completions consumed per tile
+        bool ok = true;
+        while (ok && walk.next(lane, seg, local)) {
+            const Work w = make_work<kDecode>(p, seg, local);
+            if (w.nt == 0) continue;
+            const int ntx[2] = {w.nt_a, w.nt_b};
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_q, nq & 1, ctl) &&
+                                             mbar_wait(kv_full + u % NS, (u / NS) & 1, ctl));
+            if (!ok) break;
+            tc_fence_after_sync();
+            if (leader) {
+                for (int x = 0; x < 2; ++x)
+                    if (ntx[x] > 0) issue_qk(x, u % NS);
+                if (w.nt == 1) umma_commit(q_empty);   // no S MMA after these
+                umma_commit(kv_empty + u % NS);        // K_0
+            }
+            for (int i = 0; ok && i < w.nt; ++i) {
+                const int uv = u + 1;          // V_i
+                const int uk = u + 2;          // K_{i+1}
+                ok = __all_sync(0xffffffffu, mbar_wait(kv_full + uv % NS, (uv / NS) & 1, ctl));
+                if (!ok) break;
                 for (int x = 0; x < 2; ++x) {
-                    const int ntx = x == 0 ? nt_a : nt_b;
-                    if (i >= ntx) continue;
-                    if (!(ok = mbar_wait(p_full + x, i & 1, ctl))) break;
+                    if (i >= ntx[x]) continue;
+                    ok = __all_sync(0xffffffffu, mbar_wait(p_full + x, np[x] & 1, ctl));
+                    if (!ok) break;
+                    ++np[x];
                     tc_fence_after_sync();
-                    issue_pv(x, slot_of(uv), i > 0);
-                    if (i + 1 < ntx) {
-                        if (!(ok = mbar_wait(kv_full + slot_of(uk), par_of(uk), ctl))) break;
+                    if (leader) issue_pv(x, uv % NS, i > 0);
+                    if (i + 1 < ntx[x]) {
+                        ok = __all_sync(0xffffffffu, mbar_wait(kv_full + uk % NS, (uk / NS) & 1, ctl));
+                        if (!ok) break;
                         tc_fence_after_sync();
-                        issue_qk(x, slot_of(uk));
-                        umma_commit(s_full + x);
-                    } else {
+                        if (leader) issue_qk(x, uk % NS);
+                    } else if (leader) {
                         umma_commit(o_full + x);
                     }
                 }
                 if (!ok) break;
-                release(uv);
-                if (i + 1 < nt) release(uk);
+                if (leader) {
+                    if (i + 2 == w.nt) umma_commit(q_empty);   // the S MMAs of K_{i+1} were the last
+                    umma_commit(kv_empty + uv % NS);
+                    if (i + 1 < w.nt) umma_commit(kv_empty + uk % NS);
+                }
+                u += 2;
             }
+            ++nq;
+        }
+        if (leader) {
             // Every MMA issued above completes before TMEM is released.
             umma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.wait_limit_ns);
         }
+    }
     } else {
+        setmaxnreg_inc<kRegsSoftmax>();
         // ------------------------------------------------ softmax + epilogue
         const int x = warp / 4;                            // 0: tile A, 1: tile B
         const int r = threadIdx.x - x * kBlockM;           // query row in the tile
-        const int ntx = x == 0 ? nt_a : nt_b;
-        const int nrows_x = x == 0 ? nrows_a : nrows_b;
-        const int kmax_x = x == 0 ? kmax_a : kmax_b;
-        const int posx0 = pos0 + x * kBlockM;              // mask position of row 0 of this tile
-        const int irow = posx0 + r;
         const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
         const uint32_t tS = tmem + x * 128 + lane_off;
         const uint32_t tO = tmem + 256 + x * D + lane_off;
         const float sl2 = p.sl2;
-        float m = -INFINITY;     // reference max (log2 units) the P values and O are relative to
-        float l = 0.f;           // row sum relative to m
-        bool ok = nrows_x > 0;
-        for (int i = 0; ok && i < ntx; ++i) {
-            int start, lo;
-            key_tile(t_begin + i, nt_all, kmax, start, lo);
-            const bool full_tile = (start == lo) && (start + kBlockN <= kmax_x) && (start + kBlockN - 1 <= posx0);
-            // warp-uniform: the TMEM accesses below are warp-collective
-            ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, i & 1, ctl));
-            if (!ok) break;
-            tc_fence_after_sync();
-            uint32_t s[kBlockN];
-            tmem_ld128(tS, s);
-            if (!full_tile) {
+        const bool split_mode = kDecode && p.nsplit > 1;
+        int ns = 0;          // s_full completions consumed
+        int no = 0;          // o_full completions consumed
+        bool ok = true;
+        while (ok && walk.next(lane, seg, local)) {
+            const Work w = make_work<kDecode>(p, seg, local);
+            if (!w.valid) continue;
+            const int ntx = x == 0 ? w.nt_a : w.nt_b;
+            const int nrows_x = x == 0 ? w.nrows_a : w.nrows_b;
+            if (nrows_x <= 0) continue;
+            const int kmax_x = x == 0 ? w.kmax_a : w.kmax_b;
+            const int posx0 = w.pos0 + x * kBlockM;       // mask position of row 0 of this tile
+            const int irow = posx0 + r;
+            const bool row_valid = r < nrows_x;
+            const long long tok = (long long)w.tok0 + w.qrow0 + x * kBlockM + r;
+            const size_t base = ((size_t)tok * p.H + w.h) * D;
+            // self term: a candidate row's own key (prefill rows i >= n_b; every decode row)
+            const bool self = row_valid && !split_mode && (kDecode || irow >= w.npast);
+            float ss = -INFINITY;
+            if (self) {
+                // issued before the first S wait so its latency overlaps the MMAs
+                const uint4* q4 = reinterpret_cast<const uint4*>(p.q + base);
+                const uint4* k4 = reinterpret_cast<const uint4*>(p.k_self + base);
+                float dot0 = 0.f, dot1 = 0.f;
 #pragma unroll
-                for (int e = 0; e < kBlockN; ++e) {
-                    const int j = start + e;
-                    if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
-                }
-            }
-            float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 qa = __ldg(q4 + c), ka = __ldg(k4 + c);
+                    const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qa);
+                    const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&ka);
 #pragma unroll
-            for (int e = 0; e < kBlockN; e += 4) {
-                mx0 = fmaxf(mx0, __uint_as_float(s[e]));
-                mx1 = fmaxf(mx1, __uint_as_float(s[e + 1]));
-                mx2 = fmaxf(mx2, __uint_as_float(s[e + 2]));
-                mx3 = fmaxf(mx3, __uint_as_float(s[e + 3]));
-            }
-            const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
-            // Lazy rescale: move the reference max only when some row of the
-            // warp would otherwise see P > 2^8; then every row moves to its own max.
-            const bool need = m_tile > m + kRescaleLog2;
-            if (__any_sync(0xffffffffu, need)) {
-                const float m_new = fmaxf(m, m_tile);
-                const float corr = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-                if (i > 0) {
-                    // O_x is stable: the P.V of the previous tile completed before S of this one.
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-                        tmem_st32(tO + c * 32, o);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 qf = __bfloat1622float2(qh[e]);
+                        const float2 kf = __bfloat1622float2(kh[e]);
+                        dot0 = fmaf(qf.x, kf.x, dot0);
+                        dot1 = fmaf(qf.y, kf.y, dot1);
                     }
                 }
-                l *= corr;
-                m = m_new;
+                ss = (dot0 + dot1) * sl2;
             }
-            const float m_use = (m == -INFINITY) ? 0.f : m;
-            uint32_t pk[kBlockN / 2];
-            float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+            float m = -INFINITY;     // reference max (log2 units) the P values and O are relative to
+            float l = 0.f;           // row sum relative to m
+            for (int i = 0; i < ntx; ++i) {
+                int start, lo;
+                key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
+                const bool full_tile = (start == lo) && (start + kBlockN <= kmax_x) && (start + kBlockN - 1 <= posx0);
+                // warp-uniform: the TMEM accesses below are warp-collective
+                ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, ns & 1, ctl));
+                if (!ok) break;
+                ++ns;
+                tc_fence_after_sync();
+                uint32_t s[kBlockN];
+                tmem_ld128(tS, s);
+                if (!full_tile) {
 #pragma unroll
-            for (int e = 0; e < kBlockN; e += 4) {
-                const float p0 = ex2_approx(fmaf(__uint_as_float(s[e]), sl2, -m_use));
-                const float p1 = ex2_approx(fmaf(__uint_as_float(s[e + 1]), sl2, -m_use));
-                const float p2 = ex2_approx(fmaf(__uint_as_float(s[e + 2]), sl2, -m_use));
-                const float p3 = ex2_approx(fmaf(__uint_as_float(s[e + 3]), sl2, -m_use));
-                l0 += p0;
-                l1 += p1;
-                l2 += p2;
-                l3 += p3;
-                pk[e / 2] = pack_bf16x2(p0, p1);
-                pk[e / 2 + 1] = pack_bf16x2(p2, p3);
-            }
-            l += (l0 + l1) + (l2 + l3);
-            tmem_st64(tS, pk);                             // P over the first 64 columns of S
-            tc_fence_before_sync();
-            mbar_arrive(p_full + x);
-        }
-        if (ok && ntx > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(o_full + x, 0, ctl));
-            tc_fence_after_sync();
-        }
-        if (ok) {
-            const bool row_valid = r < nrows_x;
-            const long long tok = (long long)tok0 + qrow0 + x * kBlockM + r;
-            const size_t base = ((size_t)tok * p.H + h) * D;
-            const bool split_mode = kDecode && p.nsplit > 1;
-            // self term: a candidate row's own key (prefill rows i >= n_b; every decode row)
-            const bool self = !split_mode && (kDecode || irow >= npast);
-            float a = 1.f, b = 0.f, inv = 0.f;
-            if (row_valid && !split_mode) {
-                float ss = -INFINITY;
-                if (self) {
-                    const uint4* q4 = reinterpret_cast<const uint4*>(p.q + base);
-                    const uint4* k4 = reinterpret_cast<const uint4*>(p.k_self + base);
-                    float dot0 = 0.f, dot1 = 0.f;
+                    for (int e = 0; e < kBlockN; ++e) {
+                        const int j = start + e;
+                        if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
+                    }
+                }
+                float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                    for (int c = 0; c < D / 8; ++c) {
-                        const uint4 qa = q4[c], ka = k4[c];
-                        const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qa);
-                        const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&ka);
+                for (int e = 0; e < kBlockN; e += 4) {
+                    mx0 = fmaxf(mx0, __uint_as_float(s[e]));
+                    mx1 = fmaxf(mx1, __uint_as_float(s[e + 1]));
+                    mx2 = fmaxf(mx2, __uint_as_float(s[e + 2]));
+                    mx3 = fmaxf(mx3, __uint_as_float(s[e + 3]));
+                }
+                const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                // Lazy rescale: move the reference max only when some row of the
+                // warp would otherwise see P > 2^8; then every row moves to its own max.
+                const bool need = m_tile > m + kRescaleLog2;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float m_new = fmaxf(m, m_tile);
+                    const float corr = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+                    if (i > 0) {
+                        // O_x is stable: the P.V of the previous tile completed before S of this one.
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 qf = __bfloat1622float2(qh[e]);
-                            const float2 kf = __bfloat1622float2(kh[e]);
-                            dot0 = fmaf(qf.x, kf.x, dot0);
-                            dot1 = fmaf(qf.y, kf.y, dot1);
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + c * 32, o);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+                            tmem_st32(tO + c * 32, o);
                         }
                     }
-                    ss = (dot0 + dot1) * sl2;
+                    l *= corr;
+                    m = m_new;
                 }
+                const float m_use = (m == -INFINITY) ? 0.f : m;
+                float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+                // P over the first 64 columns of S, written in two halves of 64 keys
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 64; e += 4) {
+                        const int c = half * 64 + e;
+                        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -m_use));
+                        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
+                        const float p2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, -m_use));
+                        const float p3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, -m_use));
+                        l0 += p0;
+                        l1 += p1;
+                        l2 += p2;
+                        l3 += p3;
+                        pk[e / 2] = pack_bf16x2(p0, p1);
+                        pk[e / 2 + 1] = pack_bf16x2(p2, p3);
+                    }
+                    tmem_st32(tS + half * 32, pk);
+                }
+                l += (l0 + l1) + (l2 + l3);
+                tc_fence_before_sync();
+                mbar_arrive(p_full + x);
+            }
+            if (!ok) break;
+            // ---- epilogue: the own value (self term) is fetched before waiting for O
+            uint4 vr[D / 8];
+            {
+                const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + base);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) vr[c] = self ? __ldg(v4 + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (ntx > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(o_full + x, no & 1, ctl));
+                if (!ok) break;
+                ++no;
+                tc_fence_after_sync();
+            }
+            float a = 1.f, b = 0.f, inv = 0.f;
+            if (row_valid && !split_mode) {
                 const float m_fin = fmaxf(m, ss);
                 a = (m == -INFINITY) ? 0.f : ex2_approx(m - m_fin);
                 b = self ? ex2_approx(ss - m_fin) : 0.f;
@@ -450,22 +624,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) o[e] = 0u;
                 }
-                if (!row_valid) continue;
-                if (split_mode) {
-                    float* dst = p.part_o + ((size_t)split * p.total_rows * p.H) * D + base + c * 32;
+                if (row_valid && split_mode) {
+                    float* dst = p.part_o + ((size_t)w.split * p.total_rows * p.H) * D + base + c * 32;
 #pragma unroll
                     for (int e = 0; e < 32; e += 4)
                         *reinterpret_cast<float4*>(dst + e) =
                             make_float4(__uint_as_float(o[e]), __uint_as_float(o[e + 1]),
                                         __uint_as_float(o[e + 2]), __uint_as_float(o[e + 3]));
-                    continue;
                 }
-                float res[32];
-                if (self) {
-                    const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + base + c * 32);
+                if (row_valid && !split_mode) {
+                    float res[32];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        const uint4 va = v4[q];
+                        const uint4 va = vr[c * 4 + q];
                         const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&va);
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
@@ -474,26 +645,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                             res[q * 8 + 2 * e + 1] = (__uint_as_float(o[q * 8 + 2 * e + 1]) * a + b * vf.y) * inv;
                         }
                     }
-                } else {
+                    if (p.out_fp32) {
+                        float* dst = reinterpret_cast<float*>(p.out) + base + c * 32;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) res[e] = __uint_as_float(o[e]) * a * inv;
-                }
-                if (p.out_fp32) {
-                    float* dst = reinterpret_cast<float*>(p.out) + base + c * 32;
+                        for (int e = 0; e < 32; e += 4)
+                            *reinterpret_cast<float4*>(dst + e) =
+                                make_float4(res[e], res[e + 1], res[e + 2], res[e + 3]);
+                    } else {
+                        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + base + c * 32;
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4)
-                        *reinterpret_cast<float4*>(dst + e) = make_float4(res[e], res[e + 1], res[e + 2], res[e + 3]);
-                } else {
-                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + base + c * 32;
-#pragma unroll
-                    for (int e = 0; e < 32; e += 8)
-                        *reinterpret_cast<uint4*>(dst + e) =
-                            make_uint4(pack_bf16x2(res[e], res[e + 1]), pack_bf16x2(res[e + 2], res[e + 3]),
-                                       pack_bf16x2(res[e + 4], res[e + 5]), pack_bf16x2(res[e + 6], res[e + 7]));
+                        for (int e = 0; e < 32; e += 8)
+                            *reinterpret_cast<uint4*>(dst + e) =
+                                make_uint4(pack_bf16x2(res[e], res[e + 1]), pack_bf16x2(res[e + 2], res[e + 3]),
+                                           pack_bf16x2(res[e + 4], res[e + 5]), pack_bf16x2(res[e + 6], res[e + 7]));
+                    }
                 }
             }
             if (split_mode && row_valid) {
-                float* ml = p.part_ml + (((size_t)split * p.total_rows + tok) * p.H + h) * 2;
+                float* ml = p.part_ml + (((size_t)w.split * p.total_rows + tok) * p.H + w.h) * 2;
                 ml[0] = m;
                 ml[1] = l;
             }

@@ -25,6 +25,7 @@ constexpr int kMaxDevices = 64;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::mutex g_init_mutex;
 bool g_device_ready[kMaxDevices] = {};
+int g_num_sms[kMaxDevices] = {};
 
 unsigned long long wait_limit_ns()
 {
@@ -39,14 +40,35 @@ unsigned long long wait_limit_ns()
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int D>
-cudaError_t set_attn_attrs()
+// Persistent grid: one block per SM, fewer if there cannot be that many items.
+unsigned persistent_blocks(long long item_bound)
 {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         AttnCfg<D>::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(attn_fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                AttnCfg<D>::kSmemBytes);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int sms = (dev >= 0 && dev < kMaxDevices && g_num_sms[dev] > 0) ? g_num_sms[dev] : kNumSmsHint;
+    long long n = item_bound < sms ? item_bound : sms;
+    return (unsigned)(n < 1 ? 1 : n);
+}
+
+template <typename K>
+int set_attn_attr(K kernel, int smem_bytes)
+{
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) != cudaSuccess)
+        return UNIPIN_ERR_CUDA;
+    // The kernel moves registers between warpgroups; that is only safe when it
+    // launches with exactly the per-thread count the split was computed for.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    if (fa.numRegs != kLaunchRegs) return UNIPIN_ERR_UNSUPPORTED;
+    return UNIPIN_OK;
+}
+
+template <int D>
+int set_attn_attrs()
+{
+    int rc = set_attn_attr(attn_fwd_kernel<D, false>, AttnCfg<D>::kSmemBytes);
+    if (rc != UNIPIN_OK) return rc;
+    return set_attn_attr(attn_fwd_kernel<D, true>, AttnCfg<D>::kSmemBytes);
 }
 
 // Once per device: check it is an sm_100 part, resolve the tensor-map
@@ -62,6 +84,9 @@ int ensure_device()
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
     if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
     if (major != 10 || minor != 0) return UNIPIN_ERR_UNSUPPORTED;
+    if (cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        g_num_sms[dev] < 1)
+        return UNIPIN_ERR_CUDA;
     if (!g_encode) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
@@ -70,9 +95,10 @@ int ensure_device()
             return UNIPIN_ERR_CUDA;
         g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
     }
-    if (set_attn_attrs<32>() != cudaSuccess || set_attn_attrs<64>() != cudaSuccess ||
-        set_attn_attrs<128>() != cudaSuccess)
-        return UNIPIN_ERR_CUDA;
+    int rc = set_attn_attrs<32>();
+    if (rc == UNIPIN_OK) rc = set_attn_attrs<64>();
+    if (rc == UNIPIN_OK) rc = set_attn_attrs<128>();
+    if (rc != UNIPIN_OK) return rc;
     g_device_ready[dev] = true;
     return UNIPIN_OK;
 }
@@ -172,7 +198,7 @@ int launch_pool_write(const unipin_kvpool* pool, int layer, const void* k, const
 int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
 {
     if (R < 1 || H < 1 || max_k < 1 || n_cap < 1) return 1;
-    const long long units = (long long)R * H * ((max_k + 2 * kBlockM - 1) / (2 * kBlockM));
+    const long long units = (long long)R * H * ((max_k + kPairRows - 1) / kPairRows);
     const long long slots = (long long)kNumSmsHint;   // one block per SM (all of TMEM)
     const long long target = 4 * slots;
     if (units >= 2 * slots) return 1;   // two or more waves already: no split
@@ -240,7 +266,6 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
     if (!q || !k || !v || !out || !cu_seqlens || !past_lens) return UNIPIN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return UNIPIN_ERR_MISALIGNED;
-    if (B > 65535 || H > 65535) return UNIPIN_ERR_INVALID_ARG;
     int rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -263,6 +288,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.cu = cu_seqlens;
     p.past = past_lens;
     p.slots = nullptr;
+    p.nseg = B;
     p.H = H;
     p.max_rows = max_seqlen;
     p.total_rows = total_tokens;
@@ -271,7 +297,8 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.sl2 = scale * kLog2e;
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
-    dim3 grid((unsigned)((max_seqlen + 2 * kBlockM - 1) / (2 * kBlockM)), (unsigned)H, (unsigned)B);
+    const long long bound = (long long)B * H * ((max_seqlen + kPairRows - 1) / kPairRows);
+    dim3 grid(persistent_blocks(bound), 1, 1);
     return launch_attn<false>(D, grid, tq, tk, tv, p, s);
 }
 
@@ -315,7 +342,6 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     if (!q_c || !k_c || !v_c || !out || !cu_seqlens_c || !slot_ids || !past_lens) return UNIPIN_ERR_INVALID_ARG;
     if (!aligned16(q_c) || !aligned16(k_c) || !aligned16(v_c) || !aligned16(out)) return UNIPIN_ERR_MISALIGNED;
     if (workspace && !aligned16(workspace)) return UNIPIN_ERR_MISALIGNED;
-    if (R > 65535 || H > 65535) return UNIPIN_ERR_INVALID_ARG;
     rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -336,6 +362,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     p.cu = cu_seqlens_c;
     p.past = past_lens;
     p.slots = slot_ids;
+    p.nseg = R;
     p.H = H;
     p.max_rows = max_k;
     p.total_rows = total_cand;
@@ -351,8 +378,8 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
         p.part_o = static_cast<float*>(workspace);
         p.part_ml = p.part_o + (size_t)nsplit * total_cand * H * D;
     }
-    const unsigned qpairs = (unsigned)((max_k + 2 * kBlockM - 1) / (2 * kBlockM));
-    dim3 grid(qpairs * (unsigned)nsplit, (unsigned)H, (unsigned)R);
+    const long long bound = (long long)R * H * nsplit * ((max_k + kPairRows - 1) / kPairRows);
+    dim3 grid(persistent_blocks(bound), 1, 1);
     rc = launch_attn<true>(D, grid, tq, tk, tv, p, s);
     if (rc != UNIPIN_OK || nsplit == 1) return rc;
 
