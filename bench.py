@@ -229,7 +229,9 @@ def run_ours(args, rank, world, device, dist):
     max_past = int(past.max())
     max_k = int(cand.max())
     ws_bytes = ub.rank_decode_workspace_size(batch.B, H, D, max_k, Tc, n_cap)
-    ws = torch.empty(max(ws_bytes // 4, 1), dtype=torch.float32, device=device) if ws_bytes else None
+    ws = torch.empty(ws_bytes // 4 + 4, dtype=torch.float32, device=device)
+    ws_pre = torch.empty(ub.masked_prefill_workspace_size() // 4 + 4, dtype=torch.float32, device=device)
+    decode_split = ws_bytes > 256
     status = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
     layer = 0
@@ -240,8 +242,8 @@ def run_ours(args, rank, world, device, dist):
         ub.kvpool_write(pool_k, pool_v, layer, k, v, cu, pl, sl, max_past, dev_status=status, stream=stream)
         if ev is not None:
             ev[1].record(stream)
-        ub.masked_prefill_attn(q, k, v, cu, pl, max_seqlen, out=out_p, out_fp32=False, dev_status=status,
-                               stream=stream)
+        ub.masked_prefill_attn(q, k, v, cu, pl, max_seqlen, out=out_p, out_fp32=False, workspace=ws_pre,
+                               dev_status=status, stream=stream)
         if ev is not None:
             ev[2].record(stream)
         ub.rank_decode_attn(qc, kc, vc, cu_c, sl, pl, pool_k, pool_v, layer, max_k, out=out_d, out_fp32=False,
@@ -371,7 +373,7 @@ def run_ours(args, rank, world, device, dist):
         "e2e": {"value": cand_total / (e2e_ms * 1e-3), "unit": "candidate tokens/s",
                 "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
                 "steps": e2e_steps},
-        "gpu_launches": args.steps * (3 + (1 if ws is not None else 0)),
+        "gpu_launches": args.steps * (3 + (1 if decode_split else 0)),
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

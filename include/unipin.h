@@ -83,12 +83,23 @@ typedef struct {
  *   pool, slot_ids optional (pool == NULL: no pool write).  When given, the
  *                  past K/V of segment b is also written to pool rows
  *                  [layer, slot_ids[b], h, 0:n_b) exactly as unipin_kvpool_write does.
+ *   workspace      optional device scratch, 16-byte aligned (NULL allowed).  With at
+ *                  least unipin_masked_prefill_workspace_size() bytes, the persistent
+ *                  thread blocks take (segment, head, query-tile pair) work items from
+ *                  a shared counter; without it each block takes a fixed stride of
+ *                  items.  Same result either way.  Two calls that overlap in time
+ *                  must not share a workspace.
  * Returns UNIPIN_OK or a negative unipin_status.
  */
 int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32,
                                const int* cu_seqlens, const int* past_lens, int B, int H, int D,
                                int max_seqlen, int total_tokens, float scale, const unipin_kvpool* pool,
-                               const int* slot_ids, int layer, int* dev_status, void* stream);
+                               const int* slot_ids, int layer, void* workspace, size_t workspace_bytes,
+                               int* dev_status, void* stream);
+
+/* Bytes of scratch that let unipin_masked_prefill_attn hand out work
+ * dynamically (a work counter the call zeroes on `stream` before its kernel). */
+size_t unipin_masked_prefill_workspace_size(void);
 
 /*
  * Pool write ([review] §2.4: retrieval writes the past K/V of every layer
@@ -117,20 +128,23 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
  *   q_c, k_c, v_c  [T_c, H, D] bf16, T_c = total_cand = cu_seqlens_c[R]
  *   out            [T_c, H, D], fp32 if out_fp32 else bf16
  *   max_k          host int >= every k_r (sizes the grid)
- *   workspace      optional device scratch (NULL allowed): with at least
- *                  unipin_rank_decode_workspace_size(...) bytes the pool sweep
- *                  of each request is split over several thread blocks
- *                  (split-n) and merged by a second kernel; without it one
- *                  block sweeps all n_r rows.  The result is the same either way
- *                  up to fp32 rounding.
+ *   workspace      optional device scratch, 16-byte aligned (NULL allowed).  With at
+ *                  least 256 bytes the blocks take work items from a shared counter
+ *                  (zeroed by the call on `stream`); with at least
+ *                  unipin_rank_decode_workspace_size(...) bytes the pool sweep of
+ *                  each request is also split over several thread blocks (split-n)
+ *                  and merged by a second kernel when that helps.  The result is
+ *                  the same either way up to fp32 rounding.  Two calls that overlap
+ *                  in time must not share a workspace.
  */
 int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
                             const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H,
                             int D, int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer,
                             void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
 
-/* Bytes of workspace that let unipin_rank_decode_attn split the pool sweep
- * for these sizes (n_cap = the pool's rows per slot); 0 if it would not split. */
+/* Bytes of workspace unipin_rank_decode_attn uses at most for these sizes
+ * (n_cap = the pool's rows per slot): 256 for the work counter, plus the
+ * split-n partial results when it would split. */
 size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap);
 
 /* Human-readable name of a unipin_status value. */

@@ -33,6 +33,7 @@ EXPORTS = (
     "unipin_kvpool_write",
     "unipin_rank_decode_attn",
     "unipin_rank_decode_workspace_size",
+    "unipin_masked_prefill_workspace_size",
     "unipin_status_string",
     "unipin_selftest_bounded_wait",
 )
@@ -55,7 +56,9 @@ def _load(path: str = _LIB_PATH):
                           "python kv_cache_reuse_falcon_b200/build.py): %s" % path)
     lib = ctypes.CDLL(path)
     P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, F, P, P, I, P, P]
+    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, F, P, P, I, P, SZ, P, P]
+    lib.unipin_masked_prefill_workspace_size.argtypes = []
+    lib.unipin_masked_prefill_workspace_size.restype = SZ
     lib.unipin_masked_prefill_attn.restype = I
     lib.unipin_kvpool_write.argtypes = [P, I, P, P, P, P, P, I, I, I, P, P]
     lib.unipin_kvpool_write.restype = I
@@ -110,9 +113,28 @@ def _pool(pool_k: torch.Tensor, pool_v: torch.Tensor) -> KVPool:
     return KVPool(pool_k.data_ptr(), pool_v.data_ptr(), L, S, H, n_cap, D)
 
 
+def _workspace(workspace, nbytes: int, device):
+    """'auto': a fresh device buffer of nbytes; None: no workspace; else the given tensor."""
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a CUDA tensor")
+        if nbytes <= 0:
+            return None, 0
+        workspace = torch.empty((nbytes + 15) // 16 * 4, dtype=torch.float32, device=device)
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def masked_prefill_workspace_size() -> int:
+    return int(LIB.unipin_masked_prefill_workspace_size())
+
+
 def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=None, out_fp32: bool = True,
                         scale: Optional[float] = None, pool_k=None, pool_v=None, slot_ids=None, layer: int = 0,
-                        dev_status=None, stream=None):
+                        workspace="auto", dev_status=None, stream=None):
     """M-FALCON masked prefill; optionally also writes the past K/V into pool slots."""
     _tokens(q, "q")
     T, H, D = q.shape
@@ -130,11 +152,12 @@ def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=Non
         pool = _pool(pool_k, pool_v)
         _index(slot_ids, "slot_ids", B)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    ws, ws_bytes = _workspace(workspace, masked_prefill_workspace_size(), q.device)
     rc = LIB.unipin_masked_prefill_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(bool(out_fp32)),
                                         _ptr(cu_seqlens), _ptr(past_lens), B, H, D, int(max_seqlen), T, scale,
                                         ctypes.byref(pool) if pool is not None else None,
                                         _ptr(slot_ids) if pool is not None else None, int(layer),
-                                        _ptr(dev_status), _stream(stream))
+                                        _ptr(ws), ws_bytes, _ptr(dev_status), _stream(stream))
     _check(rc, "unipin_masked_prefill_attn")
     return out
 
@@ -160,7 +183,7 @@ def rank_decode_workspace_size(R: int, H: int, D: int, max_k: int, total_cand: i
 
 
 def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, pool_v, layer: int, max_k: int,
-                     out=None, out_fp32: bool = True, scale: Optional[float] = None, workspace=None,
+                     out=None, out_fp32: bool = True, scale: Optional[float] = None, workspace="auto",
                      dev_status=None, stream=None):
     """Candidates attend to their slot's cached past rows plus themselves."""
     _tokens(q_c, "q_c")
@@ -176,15 +199,12 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
         out = torch.empty((T, H, D), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q_c.device)
     elif out.dtype != (torch.float32 if out_fp32 else torch.bfloat16) or out.shape != q_c.shape or not out.is_contiguous():
         raise ValueError("out has the wrong dtype or shape")
-    ws_bytes = 0
-    if workspace is not None:
-        if not workspace.is_cuda or not workspace.is_contiguous():
-            raise ValueError("workspace must be a contiguous CUDA tensor")
-        ws_bytes = workspace.numel() * workspace.element_size()
+    ws, ws_bytes = _workspace(workspace, rank_decode_workspace_size(R, H, D, int(max_k), T, pool.n_cap)
+                              if isinstance(workspace, str) else 0, q_c.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     rc = LIB.unipin_rank_decode_attn(_ptr(q_c), _ptr(k_c), _ptr(v_c), _ptr(out), int(bool(out_fp32)),
                                      _ptr(cu_seqlens_c), _ptr(slot_ids), _ptr(past_lens), R, H, D, int(max_k), T,
-                                     scale, ctypes.byref(pool), int(layer), _ptr(workspace), ws_bytes,
+                                     scale, ctypes.byref(pool), int(layer), _ptr(ws), ws_bytes,
                                      _ptr(dev_status), _stream(stream))
     _check(rc, "unipin_rank_decode_attn")
     return out

@@ -52,6 +52,8 @@ constexpr int kThreads = 384;
 // 384 threads can have); the producer/MMA warpgroup gives registers back and
 // the two softmax warpgroups take them: 128*72 + 256*216 = 384*168.
 constexpr int kLaunchRegs = 168;
+constexpr int kItemSlots = 4;        // items handed from the producer warp to the others
+constexpr int kItemConsumers = 9;    // the MMA warp and the eight softmax warps
 constexpr int kRegsOther = 96;
 constexpr int kRegsSoftmax = 200;
 static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
@@ -72,7 +74,7 @@ struct AttnCfg {
     static constexpr int kOffQ = 0;                             // Q_A, Q_B
     static constexpr int kOffRing = 2 * kTileBytes;
     static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
-    static constexpr int kSmemBytes = kOffBar + 256;
+    static constexpr int kSmemBytes = kOffBar + 512;
 };
 
 struct AttnParams {
@@ -95,6 +97,7 @@ struct AttnParams {
     float sl2;                    // scale * log2(e)
     int* status;
     unsigned long long wait_limit_ns;
+    unsigned long long* sched;    // zeroed item counter (dynamic scheduling) or null (static striding)
 };
 
 // Key tile t of nt covering keys [0, kmax): tiles are 128 wide from key 0;
@@ -118,9 +121,9 @@ __device__ __forceinline__ void report(int* status, int code)
     if (status) atomicCAS(status, 0, code);
 }
 
-// Warp-cooperative walk over the work items of this block: item g (global,
-// segment-major) belongs to block g % gridDim.x.  Every lane of the calling
-// warp must call next() together; all lanes get the same answer.
+// Warp-cooperative map from a global item index g (segment-major: the items
+// of segment 0, then of segment 1, ...) to its segment.  Every lane of the
+// calling warp must call locate() together; all lanes get the same answer.
 struct ItemWalker {
     const int* cu;
     int nseg, max_rows, mult;     // mult = items per query-tile pair
@@ -128,7 +131,6 @@ struct ItemWalker {
     long long base;               // items before segment c0
     int cnt, pre;                 // this lane's segment: item count, exclusive prefix in chunk
     int chunk_total;
-    long long g;
     int* status;
 
     __device__ void load_chunk(int lane)
@@ -163,12 +165,12 @@ struct ItemWalker {
         status = p.status;
         c0 = 0;
         base = 0;
-        g = blockIdx.x;
         load_chunk(lane);
     }
 
-    // Next item of this block: its segment and index within the segment.
-    __device__ bool next(int lane, int& seg, int& local)
+    // Segment and index within the segment of global item g; g must not
+    // decrease between calls.  Returns false when g is past the last item.
+    __device__ bool locate(int lane, long long g, int& seg, int& local)
     {
         while (g >= base + chunk_total) {
             if (c0 + 32 >= nseg) return false;
@@ -181,7 +183,6 @@ struct ItemWalker {
         const int L = __ffs(hit) - 1;
         seg = c0 + L;
         local = (int)(rel - __shfl_sync(0xffffffffu, pre, L));
-        g += gridDim.x;
         return true;
     }
 };
@@ -280,7 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bar_drain = bars + 8;
     uint64_t* kv_full = bars + 9;         // [NS]
     uint64_t* kv_empty = bars + 9 + NS;   // [NS]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9 + 2 * NS);
+    uint64_t* item_full = bars + 9 + 2 * NS;       // [kItemSlots]
+    uint64_t* item_empty = item_full + kItemSlots;  // [kItemSlots]
+    volatile long long* item_ring = reinterpret_cast<volatile long long*>(item_empty + kItemSlots);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 2 * kItemSlots);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     if (threadIdx.x == 0) {
@@ -292,6 +296,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(o_full + x, 1);
         }
         mbar_init(bar_drain, 1);
+        for (int s = 0; s < kItemSlots; ++s) {
+            mbar_init(item_full + s, 1);
+            mbar_init(item_empty + s, kItemConsumers);
+        }
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full + s, 1);
             mbar_init(kv_empty + s, 1);
@@ -312,6 +320,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     ItemWalker walk;
     walk.init(p, lane);
     int seg, local;
+    int n_items = 0;     // items taken from the ring by this warp
+    // Consumers: next item from the producer's ring (warp-uniform); false at the end.
+    auto pop_item = [&](bool& ok_flag) -> bool {
+        const int slot_i = n_items % kItemSlots;
+        ok_flag = __all_sync(0xffffffffu, mbar_wait(item_full + slot_i, (n_items / kItemSlots) & 1, ctl));
+        if (!ok_flag) return false;
+        const long long g = item_ring[slot_i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(item_empty + slot_i);
+        ++n_items;
+        if (g < 0) return false;
+        return walk.locate(lane, g, seg, local);
+    };
 
     // The producer and MMA warps run their loops with all 32 lanes (the item
     // walker is warp-collective); waits are taken by every lane and made
@@ -329,7 +350,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         int u = 0;          // ring uses issued so far (use u lives in slot u % NS)
         int nq = 0;         // Q loads issued so far
         bool ok = true;
-        while (ok && walk.next(lane, seg, local)) {
+        long long g_static = blockIdx.x;
+        while (ok) {
+            // claim the next item and hand it to the other warps
+            const int slot_i = n_items % kItemSlots;
+            if (n_items >= kItemSlots) {
+                ok = __all_sync(0xffffffffu, mbar_wait(item_empty + slot_i, ((n_items / kItemSlots) - 1) & 1, ctl));
+                if (!ok) break;
+            }
+            long long g = 0;
+            if (p.sched) {
+                if (leader) g = (long long)atomicAdd(p.sched, 1ull);
+                g = __shfl_sync(0xffffffffu, g, 0);
+            } else {
+                g = g_static;
+                g_static += gridDim.x;
+            }
+            const bool found = walk.locate(lane, g, seg, local);
+            if (leader) {
+                item_ring[slot_i] = found ? g : -1;
+                mbar_arrive(item_full + slot_i);   // release semantics publish the ring entry
+            }
+            ++n_items;
+            if (!found) break;
             const Work w = make_work<kDecode>(p, seg, local);
             if (!w.valid) {
                 if (leader) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
@@ -376,9 +419,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
+        if (!ok && leader) {
+            // stop the consumers: an end marker in the next ring slot
+            const int slot_i = n_items % kItemSlots;
+            if (n_items < kItemSlots ||
+                mbar_wait_drain(item_empty + slot_i, ((n_items / kItemSlots) - 1) & 1, p.wait_limit_ns)) {
+                item_ring[slot_i] = -1;
+                mbar_arrive(item_full + slot_i);
+                ++n_items;
+            }
+        }
         if (leader) {
-            // Consume the last arrival of every barrier the MMA thread signals to
+            // Consume the last arrival of every barrier the other warps signal to
             // this warp, so nothing lands in shared memory after the block exits.
+            for (int v = (n_items > kItemSlots ? n_items - kItemSlots : 0); v < n_items; ++v)
+                mbar_wait_drain(item_empty + v % kItemSlots, (v / kItemSlots) & 1, p.wait_limit_ns);
             if (nq > 0) mbar_wait_drain(q_empty, (nq - 1) & 1, p.wait_limit_ns);
             for (int v = (u > NS ? u - NS : 0); v < u; ++v)
                 mbar_wait_drain(kv_empty + v % NS, (v / NS) & 1, p.wait_limit_ns);
@@ -419,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nq = 0;                // items with MMAs
         int np[2] = {0, 0};        // p_full completions consumed per tile
         bool ok = true;
-        while (ok && walk.next(lane, seg, local)) {
+        while (pop_item(ok)) {
             const Work w = make_work<kDecode>(p, seg, local);
             if (w.nt == 0) continue;
             const int ntx[2] = {w.nt_a, w.nt_b};
@@ -483,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ns = 0;          // s_full completions consumed
         int no = 0;          // o_full completions consumed
         bool ok = true;
-        while (ok && walk.next(lane, seg, local)) {
+        while (pop_item(ok)) {
             const Work w = make_work<kDecode>(p, seg, local);
             if (!w.valid) continue;
             const int ntx = x == 0 ? w.nt_a : w.nt_b;

@@ -210,11 +210,13 @@ int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
     return (int)(ns < 1 ? 1 : ns);
 }
 
+constexpr size_t kSchedBytes = 256;   // work counter at the start of every workspace
+
 size_t decode_workspace_bytes(int nsplit, int total_cand, int H, int D)
 {
-    if (nsplit <= 1) return 0;
+    if (nsplit <= 1) return kSchedBytes;
     const size_t rows = (size_t)nsplit * (size_t)total_cand * (size_t)H;
-    return rows * (size_t)D * sizeof(float) + rows * 2 * sizeof(float);
+    return kSchedBytes + rows * (size_t)D * sizeof(float) + rows * 2 * sizeof(float);
 }
 
 __global__ void bounded_wait_selftest_kernel(int* status, unsigned long long limit_ns)
@@ -250,10 +252,12 @@ const char* unipin_status_string(int status)
     }
 }
 
+size_t unipin_masked_prefill_workspace_size(void) { return kSchedBytes; }
+
 int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32,
                                const int* cu_seqlens, const int* past_lens, int B, int H, int D, int max_seqlen,
                                int total_tokens, float scale, const unipin_kvpool* pool, const int* slot_ids,
-                               int layer, int* dev_status, void* stream)
+                               int layer, void* workspace, size_t workspace_bytes, int* dev_status, void* stream)
 {
     if (B < 0 || H < 1 || max_seqlen < 0 || total_tokens < 0) return UNIPIN_ERR_INVALID_ARG;
     if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
@@ -266,9 +270,15 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
     if (!q || !k || !v || !out || !cu_seqlens || !past_lens) return UNIPIN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return UNIPIN_ERR_MISALIGNED;
+    if (workspace && !aligned16(workspace)) return UNIPIN_ERR_MISALIGNED;
     int rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    unsigned long long* sched = nullptr;
+    if (workspace && workspace_bytes >= kSchedBytes) {
+        sched = static_cast<unsigned long long*>(workspace);
+        if (cudaMemsetAsync(sched, 0, sizeof(unsigned long long), s) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    }
 
     if (pool) {
         rc = launch_pool_write(pool, layer, k, v, cu_seqlens, past_lens, slot_ids, B, H, D, max_seqlen, total_tokens,
@@ -297,6 +307,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.sl2 = scale * kLog2e;
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
+    p.sched = sched;
     const long long bound = (long long)B * H * ((max_seqlen + kPairRows - 1) / kPairRows);
     dim3 grid(persistent_blocks(bound), 1, 1);
     return launch_attn<false>(D, grid, tq, tk, tv, p, s);
@@ -348,6 +359,11 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
 
     int nsplit = decode_nsplit(R, H, D, max_k, pool->n_cap);
     if (nsplit > 1 && (!workspace || workspace_bytes < decode_workspace_bytes(nsplit, total_cand, H, D))) nsplit = 1;
+    unsigned long long* sched = nullptr;
+    if (workspace && workspace_bytes >= kSchedBytes) {
+        sched = static_cast<unsigned long long*>(workspace);
+        if (cudaMemsetAsync(sched, 0, sizeof(unsigned long long), s) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    }
 
     CUtensorMap tq, tk, tv;
     if ((rc = make_token_map(&tq, q_c, total_cand, H, D)) != UNIPIN_OK) return rc;
@@ -374,8 +390,9 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     p.sl2 = scale * kLog2e;
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
+    p.sched = sched;
     if (nsplit > 1) {
-        p.part_o = static_cast<float*>(workspace);
+        p.part_o = reinterpret_cast<float*>(static_cast<char*>(workspace) + kSchedBytes);
         p.part_ml = p.part_o + (size_t)nsplit * total_cand * H * D;
     }
     const long long bound = (long long)R * H * nsplit * ((max_k + kPairRows - 1) / kPairRows);

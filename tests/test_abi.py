@@ -47,18 +47,22 @@ def test_host_validation_needs_no_device(lib):
     """Argument errors are found before any CUDA call, so they work without a GPU."""
     P, I = ctypes.c_void_p, ctypes.c_int
     f = lib.unipin_masked_prefill_attn
-    f.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, ctypes.c_float, P, P, I, P, P]
+    SZ = ctypes.c_size_t
+    f.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, ctypes.c_float, P, P, I, P, SZ, P, P]
     f.restype = I
-    assert f(None, None, None, None, 1, None, None, 1, 1, 48, 16, 16, 0.1, None, None, 0, None, None) == -2
-    assert f(None, None, None, None, 1, None, None, -1, 1, 64, 16, 16, 0.1, None, None, 0, None, None) == -1
-    assert f(None, None, None, None, 1, None, None, 1, 1, 64, 16, 16, -1.0, None, None, 0, None, None) == -1
+    assert f(None, None, None, None, 1, None, None, 1, 1, 48, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -2
+    assert f(None, None, None, None, 1, None, None, -1, 1, 64, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -1
+    assert f(None, None, None, None, 1, None, None, 1, 1, 64, 16, 16, -1.0, None, None, 0, None, 0, None, None) == -1
     # nothing to do: B = 0 returns OK without touching the device
-    assert f(None, None, None, None, 1, None, None, 0, 1, 64, 16, 0, 0.1, None, None, 0, None, None) == 0
+    assert f(None, None, None, None, 1, None, None, 0, 1, 64, 16, 0, 0.1, None, None, 0, None, 0, None, None) == 0
     g = lib.unipin_rank_decode_workspace_size
     g.argtypes = [I, I, I, I, I, I]
-    g.restype = ctypes.c_size_t
-    assert g(32, 8, 64, 16, 512, 2048) > 0
-    assert g(32, 8, 64, 1000, 32000, 2048) == 0
+    g.restype = SZ
+    assert g(32, 8, 64, 16, 512, 2048) > 256       # small k: split-n partials on top of the work counter
+    assert g(32, 8, 64, 1000, 32000, 2048) == 256  # large k: the work counter only
+    wp = lib.unipin_masked_prefill_workspace_size
+    wp.restype = SZ
+    assert wp() == 256
 
 
 def test_binding_refuses_to_load_without_library(tmp_path):

@@ -119,7 +119,7 @@ def test_rank_decode_from_pool_workload(ub):
     d16.slot_ids = d.slot_ids
     dd16 = DevDecode(d16)
     nbytes = ub.rank_decode_workspace_size(w.B, w.H, w.D, 16, int(d16.cu_seqlens[-1]), w.n_cap)
-    assert nbytes > 0
+    assert nbytes > 256
     ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device="cuda")
     o16 = ub.rank_decode_attn(dd16.q, dd16.k, dd16.v, dd16.cu, dd16.slots, dd16.past, pk, pv, layer, 16,
                               out_fp32=True, workspace=ws, dev_status=status)
@@ -153,11 +153,7 @@ def test_ragged_mixed_batch_prefill_then_decode(ub):
     dd.cu = torch.from_numpy(d.cu_seqlens).cuda()
     dd.past, dd.slots = dp.past, dp.slots
     dd.max_k = int(batch.cand_lens.max())
-    for use_ws in (False, True):
-        ws = None
-        if use_ws:
-            nb = ub.rank_decode_workspace_size(batch.B, w.H, w.D, dd.max_k, len(cidx), w.n_cap)
-            ws = torch.empty(nb // 4 + 4, dtype=torch.float32, device="cuda") if nb else None
+    for ws in (None, "auto"):
         dec = ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, 0, dd.max_k,
                                   out_fp32=True, workspace=ws, dev_status=status)
         torch.cuda.synchronize()
