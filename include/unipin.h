@@ -159,6 +159,14 @@ const char* unipin_status_string(int status);
  */
 int unipin_selftest_bounded_wait(int* dev_status, unsigned int limit_us, void* stream);
 
+/*
+ * Self-test of the exp2 the softmax evaluates on the FMA pipe for one score
+ * pair in four (a degree-3 polynomial after rounding the argument to an
+ * integer, see csrc/sm100_ptx.cuh): y[i] = 2^x[i] for n device floats, so
+ * tests can compare it with CUDA's exp2f.  Arguments below -127 give 0.
+ */
+int unipin_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,6 +36,7 @@ EXPORTS = (
     "unipin_masked_prefill_workspace_size",
     "unipin_status_string",
     "unipin_selftest_bounded_wait",
+    "unipin_selftest_exp2",
 )
 
 
@@ -70,6 +71,8 @@ def _load(path: str = _LIB_PATH):
     lib.unipin_status_string.restype = ctypes.c_char_p
     lib.unipin_selftest_bounded_wait.argtypes = [P, ctypes.c_uint, P]
     lib.unipin_selftest_bounded_wait.restype = I
+    lib.unipin_selftest_exp2.argtypes = [P, P, I, P]
+    lib.unipin_selftest_exp2.restype = I
     return lib
 
 
@@ -213,6 +216,15 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
 def selftest_bounded_wait(dev_status, limit_us: int, stream=None):
     rc = LIB.unipin_selftest_bounded_wait(_ptr(dev_status), int(limit_us), _stream(stream))
     _check(rc, "unipin_selftest_bounded_wait")
+
+
+def selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The softmax's FMA-pipe exp2 on a CUDA float32 tensor."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    _check(LIB.unipin_selftest_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "unipin_selftest_exp2")
+    return y
 
 
 def status_string(code: int) -> str:

@@ -595,11 +595,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < kBlockN; e += 4) {
-                    mx0 = fmaxf(mx0, __uint_as_float(s[e]));
-                    mx1 = fmaxf(mx1, __uint_as_float(s[e + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(s[e + 2]));
-                    mx3 = fmaxf(mx3, __uint_as_float(s[e + 3]));
+                for (int e = 0; e < kBlockN; e += 8) {
+                    mx0 = max3f(mx0, __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+                    mx1 = max3f(mx1, __uint_as_float(s[e + 2]), __uint_as_float(s[e + 3]));
+                    mx2 = max3f(mx2, __uint_as_float(s[e + 4]), __uint_as_float(s[e + 5]));
+                    mx3 = max3f(mx3, __uint_as_float(s[e + 6]), __uint_as_float(s[e + 7]));
                 }
                 const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
                 // Lazy rescale: move the reference max only when some row of the
@@ -623,28 +623,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = m_new;
                 }
                 const float m_use = (m == -INFINITY) ? 0.f : m;
-                float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-                // P over the first 64 columns of S, written in two halves of 64 keys
+                // P = 2^(s * scale * log2e - m): packed fp32 pairs; one pair in four
+                // takes the polynomial exp2 on the FMA pipe, the rest the MUFU ex2,
+                // so the two pipes share the load.  P goes over the first 64
+                // columns of S, written in two halves of 64 keys.
+                const uint64_t sc2 = f2_pack(sl2, sl2);
+                const uint64_t nm2 = f2_pack(-m_use, -m_use);
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[32];
 #pragma unroll
-                    for (int e = 0; e < 64; e += 4) {
-                        const int c = half * 64 + e;
-                        const float p0 = ex2_approx(fmaf(__uint_as_float(s[c]), sl2, -m_use));
-                        const float p1 = ex2_approx(fmaf(__uint_as_float(s[c + 1]), sl2, -m_use));
-                        const float p2 = ex2_approx(fmaf(__uint_as_float(s[c + 2]), sl2, -m_use));
-                        const float p3 = ex2_approx(fmaf(__uint_as_float(s[c + 3]), sl2, -m_use));
-                        l0 += p0;
-                        l1 += p1;
-                        l2 += p2;
-                        l3 += p3;
-                        pk[e / 2] = pack_bf16x2(p0, p1);
-                        pk[e / 2 + 1] = pack_bf16x2(p2, p3);
+                    for (int c = 0; c < 32; ++c) {
+                        const int e = half * 64 + 2 * c;
+                        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2);
+                        float p0, p1;
+                        if ((c & 3) == 3) {
+                            exp2_poly2(x2, p0, p1);
+                        } else {
+                            float x0, x1;
+                            f2_unpack(x2, x0, x1);
+                            p0 = ex2_approx(x0);
+                            p1 = ex2_approx(x1);
+                        }
+                        acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
+                        pk[c] = pack_bf16x2(p0, p1);
                     }
                     tmem_st32(tS + half * 32, pk);
                 }
-                l += (l0 + l1) + (l2 + l3);
+                {
+                    const uint64_t a01 = f2_add(acc[0], acc[1]);
+                    const uint64_t a23 = f2_add(acc[2], acc[3]);
+                    float lo, hi;
+                    f2_unpack(f2_add(a01, a23), lo, hi);
+                    l += lo + hi;
+                }
                 tc_fence_before_sync();
                 mbar_arrive(p_full + x);
             }
@@ -731,6 +744,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// Evaluates the FMA-pipe exp2 used by the softmax on n inputs (for tests).
+__global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, int n)
+{
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float a = x[i];
+    const float b = (i + 1 < n) ? x[i + 1] : 0.f;
+    float r0, r1;
+    exp2_poly2(f2_pack(a, b), r0, r1);
+    y[i] = r0;
+    if (i + 1 < n) y[i + 1] = r1;
 }
 
 // Split-n merge for the rank decode: each (candidate, head) row combines the

@@ -33,6 +33,73 @@ __device__ __forceinline__ float ex2_approx(float x)
     return y;
 }
 
+// ------------------------------------------------- packed fp32 pair math
+// Blackwell executes two fp32 FMAs / adds per lane in one instruction.
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^x for a pair of fp32 values on the FMA pipe (no MUFU):
+//   x is clamped to >= -127 (so -inf and masked scores give 0),
+//   n = round(x) by adding and subtracting 1.5 * 2^23, f = x - n in [-1/2, 1/2],
+//   2^f ~= 1 + c1 f + c2 f^2 + c3 f^3, and n is added to the exponent field.
+// c1..c3 were fitted here for this kernel (relative-error least squares with
+// Lawson reweighting toward the minimax fit, p(0) = 1 fixed so integer x are
+// exact); max relative error 1.02e-4 over the used range, far below the
+// bf16 rounding the probabilities get next.
+__device__ __forceinline__ void exp2_poly2(uint64_t x2, float& r0, float& r1)
+{
+    constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+    constexpr float kC1 = 0x1.62f5fap-1f;
+    constexpr float kC2 = 0x1.f00c4ep-3f;
+    constexpr float kC3 = 0x1.c2a216p-5f;
+    float x0, x1;
+    f2_unpack(x2, x0, x1);
+    const uint64_t xc = f2_pack(fmaxf(x0, -127.f), fmaxf(x1, -127.f));
+    const uint64_t t = f2_add(xc, f2_pack(kMagic, kMagic));
+    const uint64_t n = f2_add(t, f2_pack(-kMagic, -kMagic));
+    const uint64_t fr = f2_fma(n, f2_pack(-1.f, -1.f), xc);
+    uint64_t pp = f2_fma(f2_pack(kC3, kC3), fr, f2_pack(kC2, kC2));
+    pp = f2_fma(pp, fr, f2_pack(kC1, kC1));
+    pp = f2_fma(pp, fr, f2_pack(1.f, 1.f));
+    float p0, p1, t0, t1;
+    f2_unpack(pp, p0, p1);
+    f2_unpack(t, t0, t1);
+    // the low mantissa bits of t hold n; shifting them into the exponent field adds n
+    r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // --------------------------------------------------------------- mbarriers
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)

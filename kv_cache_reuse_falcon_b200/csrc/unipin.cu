@@ -419,6 +419,16 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 
+int unipin_selftest_exp2(const float* x, float* y, int n, void* stream)
+{
+    if (n < 0 || (n > 0 && (!x || !y))) return UNIPIN_ERR_INVALID_ARG;
+    if (n == 0) return UNIPIN_OK;
+    const int threads = 256;
+    const int blocks = (n / 2 + threads) / threads;
+    exp2_poly_selftest_kernel<<<blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
 int unipin_selftest_bounded_wait(int* dev_status, unsigned int limit_us, void* stream)
 {
     if (!dev_status || limit_us == 0) return UNIPIN_ERR_INVALID_ARG;

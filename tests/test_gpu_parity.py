@@ -274,3 +274,18 @@ def test_bounded_wait_times_out_with_status_not_hang(ub):
     # the context is still usable afterwards
     x = torch.ones(4, device="cuda")
     assert float(x.sum().item()) == 4.0
+
+
+def test_fma_pipe_exp2_against_cuda_exp2f(ub):
+    """The polynomial exp2 the softmax uses for one score pair in four, against CUDA's exp2f."""
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1 << 20, device="cuda"),
+                   torch.tensor([0.0, 1.0, -1.0, 8.0, -0.5, 0.5, 3.0, -126.0], device="cuda")])
+    y = ub.selftest_exp2(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel < 1.2e-4, rel
+    # integers are exact (p(0) = 1), arguments at or below -127 and -inf give 0
+    ints = torch.arange(-120, 9, device="cuda", dtype=torch.float32)
+    assert torch.equal(ub.selftest_exp2(ints), torch.exp2(ints))
+    low = torch.tensor([-127.0, -200.0, -1e30, float("-inf")], device="cuda")
+    assert torch.count_nonzero(ub.selftest_exp2(low)) == 0
