@@ -30,8 +30,9 @@
 //              P <= 2^8, exact after the final division).
 //   warp 8     TMA producer: per item the Q tiles, then K_0, V_0, K_1, V_1, ...
 //              through a ring of shared-memory slots (the ring runs across items).
-//   warp 9     TMEM allocator and the single UMMA-issuing thread.
-//   warps 10-11 idle (they complete the third warpgroup for the register split).
+//   warps 9, 10 the UMMA issuers of tile A and tile B (one elected thread each);
+//              warp 9 also allocates TMEM.
+//   warp 11    idle (it completes the third warpgroup for the register split).
 // Every warp walks the same item sequence (ItemWalker), so no queue is shared.
 //
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B [256+D, 256+2D);
@@ -53,7 +54,7 @@ constexpr int kThreads = 384;
 // the two softmax warpgroups take them: 128*72 + 256*216 = 384*168.
 constexpr int kLaunchRegs = 168;
 constexpr int kItemSlots = 4;        // items handed from the producer warp to the others
-constexpr int kItemConsumers = 9;    // the MMA warp and the eight softmax warps
+constexpr int kItemConsumers = 10;   // the two MMA warps and the eight softmax warps
 constexpr int kRegsOther = 96;
 constexpr int kRegsSoftmax = 200;
 static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
@@ -278,10 +279,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* s_full = bars + 2;          // [2]
     uint64_t* p_full = bars + 4;          // [2]
     uint64_t* o_full = bars + 6;          // [2]
-    uint64_t* bar_drain = bars + 8;
-    uint64_t* kv_full = bars + 9;         // [NS]
-    uint64_t* kv_empty = bars + 9 + NS;   // [NS]
-    uint64_t* item_full = bars + 9 + 2 * NS;       // [kItemSlots]
+    uint64_t* bar_drain = bars + 8;       // [2] (bars + 8, bars + 9)
+    uint64_t* kv_full = bars + 10;        // [NS]
+    uint64_t* kv_empty = bars + 10 + NS;  // [NS]
+    uint64_t* item_full = bars + 10 + 2 * NS;      // [kItemSlots]
     uint64_t* item_empty = item_full + kItemSlots;  // [kItemSlots]
     volatile long long* item_ring = reinterpret_cast<volatile long long*>(item_empty + kItemSlots);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 2 * kItemSlots);
@@ -289,20 +290,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        mbar_init(q_empty, 1);
+        mbar_init(q_empty, 2);            // one arrival from each MMA warp
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full + x, 1);
             mbar_init(p_full + x, kBlockM);
             mbar_init(o_full + x, 1);
         }
-        mbar_init(bar_drain, 1);
+        mbar_init(bar_drain + 0, 1);
+        mbar_init(bar_drain + 1, 1);
         for (int s = 0; s < kItemSlots; ++s) {
             mbar_init(item_full + s, 1);
             mbar_init(item_empty + s, kItemConsumers);
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full + s, 1);
-            mbar_init(kv_empty + s, 1);
+            mbar_init(kv_empty + s, 2);   // one arrival from each MMA warp
         }
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -438,82 +440,101 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int v = (u > NS ? u - NS : 0); v < u; ++v)
                 mbar_wait_drain(kv_empty + v % NS, (v / NS) & 1, p.wait_limit_ns);
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------------ UMMA issuer
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------- UMMA issuers
+        // Warp 9 issues the MMAs of tile A, warp 10 those of tile B, so each
+        // tile's next MMAs go out as soon as its own P is ready, never queued
+        // behind the other tile's issue.  Both release every K/V ring use and
+        // every Q load (arrival count 2); a use a warp does not need is still
+        // released, after its fill, so the two warps' arrivals stay in phase.
+        const int x = warp - 9;
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
         // Descriptors are built once; a K-step moves only the start-address
         // field (low 14 bits, in 16-byte units), by compile-time offsets.
-        const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dq0 = smem_desc(smem_u32(sQ) + x * C::kTileBytes, 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dk0 = smem_desc(smem_u32(ring), 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dv0 = smem_desc(smem_u32(ring), C::kAtomBytes, 8 * C::kRowBytes, C::kLayout);
+        const uint32_t tS = tmem + x * 128;
+        const uint32_t tO = tmem + 256 + x * D;
         // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16 elements.
-        auto issue_qk = [&](int x, int st) {
-            const uint64_t a0 = dq0 + (uint64_t)((x * C::kTileBytes) >> 4);
+        auto issue_qk = [&](int st) {
             const uint64_t b0 = dk0 + (uint64_t)((st * C::kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 constexpr int kStep = 32;
                 const uint32_t off = ((kk * kStep / C::kRowBytes) * C::kAtomBytes + (kk * kStep) % C::kRowBytes) >> 4;
-                umma_bf16_ss(tmem + x * 128, a0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+                umma_bf16_ss(tS, dq0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
             }
             umma_commit(s_full + x);
         };
         // O_x += P_x V: P from TMEM (first 64 columns of S_x, 8 columns per
         // 16 keys), V read MN-major (D contiguous); K-steps of 16 keys.
-        auto issue_pv = [&](int x, int st, bool acc) {
+        auto issue_pv = [&](int st, bool acc) {
             const uint64_t b0 = dv0 + (uint64_t)((st * C::kTileBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < kBlockN / 16; ++kk) {
                 const uint32_t off = (kk * 16 * C::kRowBytes) >> 4;
-                umma_bf16_ts(tmem + 256 + x * D, tmem + x * 128 + kk * 8, b0 + off, idesc_pv,
-                             (acc || kk > 0) ? 1u : 0u);
+                umma_bf16_ts(tO, tS + kk * 8, b0 + off, idesc_pv, (acc || kk > 0) ? 1u : 0u);
             }
+        };
+        auto wait_fill = [&](int u) {
+            return __all_sync(0xffffffffu, mbar_wait(kv_full + u % NS, (u / NS) & 1, ctl));
         };
         int u = 0;                 // ring uses consumed
         int nq = 0;                // items with MMAs
-        int np[2] = {0, 0};        // p_full completions consumed per tile
+        int np = 0;                // p_full completions consumed
         bool ok = true;
         while (pop_item(ok)) {
             const Work w = make_work<kDecode>(p, seg, local);
             if (w.nt == 0) continue;
-            const int ntx[2] = {w.nt_a, w.nt_b};
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_q, nq & 1, ctl) &&
-                                             mbar_wait(kv_full + u % NS, (u / NS) & 1, ctl));
+            const int ntx = x == 0 ? w.nt_a : w.nt_b;
+            // Q landed: this also means both warps released the previous Q.
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_q, nq & 1, ctl)) && wait_fill(u);
             if (!ok) break;
             tc_fence_after_sync();
             if (leader) {
-                for (int x = 0; x < 2; ++x)
-                    if (ntx[x] > 0) issue_qk(x, u % NS);
-                if (w.nt == 1) umma_commit(q_empty);   // no S MMA after these
-                umma_commit(kv_empty + u % NS);        // K_0
+                if (ntx > 0) {
+                    issue_qk(u % NS);
+                    umma_commit(kv_empty + u % NS);                 // K_0
+                    if (ntx == 1) umma_commit(q_empty);            // no S MMA of this tile after this
+                } else {
+                    mbar_arrive(kv_empty + u % NS);
+                    mbar_arrive(q_empty);
+                }
             }
             for (int i = 0; ok && i < w.nt; ++i) {
                 const int uv = u + 1;          // V_i
                 const int uk = u + 2;          // K_{i+1}
-                ok = __all_sync(0xffffffffu, mbar_wait(kv_full + uv % NS, (uv / NS) & 1, ctl));
-                if (!ok) break;
-                for (int x = 0; x < 2; ++x) {
-                    if (i >= ntx[x]) continue;
-                    ok = __all_sync(0xffffffffu, mbar_wait(p_full + x, np[x] & 1, ctl));
+                if (!(ok = wait_fill(uv))) break;
+                if (i < ntx) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(p_full + x, np & 1, ctl));
                     if (!ok) break;
-                    ++np[x];
+                    ++np;
                     tc_fence_after_sync();
-                    if (leader) issue_pv(x, uv % NS, i > 0);
-                    if (i + 1 < ntx[x]) {
-                        ok = __all_sync(0xffffffffu, mbar_wait(kv_full + uk % NS, (uk / NS) & 1, ctl));
-                        if (!ok) break;
+                    if (leader) issue_pv(uv % NS, i > 0);
+                    if (i + 1 < ntx) {
+                        if (!(ok = wait_fill(uk))) break;
                         tc_fence_after_sync();
-                        if (leader) issue_qk(x, uk % NS);
+                        if (leader) {
+                            issue_qk(uk % NS);
+                            if (i + 2 == ntx) umma_commit(q_empty);   // that was this tile's last S MMA
+                        }
                     } else if (leader) {
                         umma_commit(o_full + x);
                     }
+                    if (leader) umma_commit(kv_empty + uv % NS);
+                } else if (leader) {
+                    mbar_arrive(kv_empty + uv % NS);
                 }
-                if (!ok) break;
-                if (leader) {
-                    if (i + 2 == w.nt) umma_commit(q_empty);   // the S MMAs of K_{i+1} were the last
-                    umma_commit(kv_empty + uv % NS);
-                    if (i + 1 < w.nt) umma_commit(kv_empty + uk % NS);
+                if (i + 1 < w.nt) {
+                    if (i + 1 >= ntx) {
+                        // K_{i+1} is only for the other tile: release it once it has landed
+                        if (!(ok = wait_fill(uk))) break;
+                        if (leader) mbar_arrive(kv_empty + uk % NS);
+                    } else if (leader) {
+                        umma_commit(kv_empty + uk % NS);
+                    }
                 }
                 u += 2;
             }
@@ -521,8 +542,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (leader) {
             // Every MMA issued above completes before TMEM is released.
-            umma_commit(bar_drain);
-            mbar_wait_drain(bar_drain, 0, p.wait_limit_ns);
+            umma_commit(bar_drain + x);
+            mbar_wait_drain(bar_drain + x, 0, p.wait_limit_ns);
         }
     }
     } else {
