@@ -621,26 +621,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 ++ns;
                 tc_fence_after_sync();
-                // Row max in two 64-column TMEM loads (keeps the live set small).
+                uint32_t s[kBlockN];
+                tmem_ld128(tS, s);
+                if (!full_tile) {
+#pragma unroll
+                    for (int e = 0; e < kBlockN; ++e) {
+                        const int j = start + e;
+                        if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
+                    }
+                }
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t s[64];
-                    tmem_ld64(tS + half * 64, s);
-                    if (!full_tile) {
-#pragma unroll
-                        for (int e = 0; e < 64; ++e) {
-                            const int j = start + half * 64 + e;
-                            if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
-                        }
-                    }
-#pragma unroll
-                    for (int e = 0; e < 64; e += 8) {
-                        mx0 = max3f(mx0, __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
-                        mx1 = max3f(mx1, __uint_as_float(s[e + 2]), __uint_as_float(s[e + 3]));
-                        mx2 = max3f(mx2, __uint_as_float(s[e + 4]), __uint_as_float(s[e + 5]));
-                        mx3 = max3f(mx3, __uint_as_float(s[e + 6]), __uint_as_float(s[e + 7]));
-                    }
+                for (int e = 0; e < kBlockN; e += 8) {
+                    mx0 = max3f(mx0, __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
+                    mx1 = max3f(mx1, __uint_as_float(s[e + 2]), __uint_as_float(s[e + 3]));
+                    mx2 = max3f(mx2, __uint_as_float(s[e + 4]), __uint_as_float(s[e + 5]));
+                    mx3 = max3f(mx3, __uint_as_float(s[e + 6]), __uint_as_float(s[e + 7]));
                 }
                 const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
                 // Lazy rescale: move the reference max only when some row of the
@@ -664,29 +660,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = m_new;
                 }
                 const float m_use = (m == -INFINITY) ? 0.f : m;
-                // P = 2^(s * scale * log2e - m) on packed fp32 pairs; one pair in four
+                // P = 2^(s * scale * log2e - m): packed fp32 pairs; one pair in four
                 // takes the polynomial exp2 on the FMA pipe, the rest the MUFU ex2,
-                // so the two pipes share the load.  Each 64-key half of S is read
-                // again and its P written over the first 64 columns of S (half h to
-                // columns 32h..32h+31, already consumed).
+                // so the two pipes share the load.  P goes over the first 64
+                // columns of S, written in two halves of 64 keys.
                 const uint64_t sc2 = f2_pack(sl2, sl2);
                 const uint64_t nm2 = f2_pack(-m_use, -m_use);
                 uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    uint32_t s[64];
-                    tmem_ld64(tS + half * 64, s);
-                    if (!full_tile) {
-#pragma unroll
-                        for (int e = 0; e < 64; ++e) {
-                            const int j = start + half * 64 + e;
-                            if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
-                        }
-                    }
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
-                        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[2 * c]), __uint_as_float(s[2 * c + 1])), sc2, nm2);
+                        const int e = half * 64 + 2 * c;
+                        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2);
                         float p0, p1;
                         if ((c & 3) == 3) {
                             exp2_poly2(x2, p0, p1);
@@ -704,9 +691,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 {
                     const uint64_t a01 = f2_add(acc[0], acc[1]);
                     const uint64_t a23 = f2_add(acc[2], acc[3]);
-                    float lo2, hi2;
-                    f2_unpack(f2_add(a01, a23), lo2, hi2);
-                    l += lo2 + hi2;
+                    float lo, hi;
+                    f2_unpack(f2_add(a01, a23), lo, hi);
+                    l += lo + hi;
                 }
                 tc_fence_before_sync();
                 mbar_arrive(p_full + x);
