@@ -54,7 +54,6 @@ constexpr int kThreads = 384;
 // the two softmax warpgroups take them: 128*72 + 256*216 = 384*168.
 constexpr int kLaunchRegs = 168;
 constexpr int kItemSlots = 4;        // items handed from the producer warp to the others
-constexpr int kPrefetchAhead = 3;    // key tiles the producer warms L2 ahead of its loads
 constexpr int kItemConsumers = 10;   // the two MMA warps and the eight softmax warps
 constexpr int kRegsOther = 96;
 constexpr int kRegsSoftmax = 200;
@@ -72,7 +71,7 @@ struct AttnCfg {
     static constexpr uint32_t kLayout = kRowBytes == 128 ? kLayoutSw128 : kLayoutSw64;
     static constexpr int kAtomBytes = kBlockM * kRowBytes;      // one box of 128 rows
     static constexpr int kTileBytes = kBlockM * D * 2;          // one Q, K or V tile
-    static constexpr int kStages = D == 128 ? 5 : 8;            // ring slots (each one K or one V tile)
+    static constexpr int kStages = D == 128 ? 4 : 8;            // ring slots (each one K or one V tile)
     static constexpr int kOffQ = 0;                             // Q_A, Q_B
     static constexpr int kOffRing = 2 * kTileBytes;
     static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
@@ -399,21 +398,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; ok && i < w.nt; ++i) {
                 int start, lo;
                 key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
-                if (leader && i + kPrefetchAhead < w.nt) {
-                    // warm L2 with the K/V tiles kPrefetchAhead steps ahead, so the
-                    // ring refill that follows a slot release hits L2
-                    int pstart, plo;
-                    key_tile(w.t_begin + i + kPrefetchAhead, w.nt_all, w.kmax, pstart, plo);
-                    for (int c = 0; c < C::kChunks; ++c) {
-                        if (kDecode) {
-                            tma_prefetch_3d(&tm_k, c * C::kBoxD, pstart, pool_plane);
-                            tma_prefetch_3d(&tm_v, c * C::kBoxD, pstart, pool_plane);
-                        } else {
-                            tma_prefetch_3d(&tm_k, c * C::kBoxD, w.h, w.tok0 + pstart);
-                            tma_prefetch_3d(&tm_v, c * C::kBoxD, w.h, w.tok0 + pstart);
-                        }
-                    }
-                }
                 for (int kv = 0; kv < 2; ++kv) {          // K_i then V_i
                     const int st = u % NS;
                     if (u >= NS) {

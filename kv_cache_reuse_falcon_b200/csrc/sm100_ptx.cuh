@@ -197,15 +197,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-// Warm L2 with a 3-D tile (no shared-memory destination, no completion to wait for).
-__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0, int c1, int c2)
-{
-    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-
 // Generic-proxy shared-memory writes -> visible to the async proxy (UMMA operands).
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
