@@ -147,6 +147,35 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
  * split-n partial results when it would split. */
 size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap);
 
+/*
+ * Rank decode that allocates nothing and takes no workspace.  There is no
+ * counterpart to this on the pages; it exists for callers that cannot call
+ * cudaMalloc at decode time: a serving process whose device memory is already
+ * handed to another framework's pool, or a loop that must not allocate after
+ * start-up.  Arguments, results and errors are those of
+ * unipin_rank_decode_attn; the scratch it needs (a work counter and, for
+ * small candidate counts, the split-n partial results) lives in a device
+ * array of unipin_rank_decode_noalloc_scratch_bytes() bytes (32 MiB) that the
+ * library reserves on every device it is loaded on and keeps until the
+ * process exits.
+ *   - If unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand,
+ *     pool->n_cap) exceeds that size, nothing is launched and
+ *     UNIPIN_ERR_OUT_OF_RANGE is returned.
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents
+ *     (the call zeroes the work counter it needs on `stream` itself), so two
+ *     calls that overlap on the GPU - on different streams, or from different
+ *     host threads - race and may give wrong results.  Serialise them.
+ */
+int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
+                                    const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R,
+                                    int H, int D, int max_k, int total_cand, float scale,
+                                    const unipin_kvpool* pool, int layer, int* dev_status, void* stream);
+
+/* Size of the array behind unipin_rank_decode_attn_noalloc (32 MiB). */
+size_t unipin_rank_decode_noalloc_scratch_bytes(void);
+
 /* Human-readable name of a unipin_status value. */
 const char* unipin_status_string(int status);
 

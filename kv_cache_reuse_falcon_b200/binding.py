@@ -37,6 +37,8 @@ EXPORTS = (
     "unipin_status_string",
     "unipin_selftest_bounded_wait",
     "unipin_selftest_exp2",
+    "unipin_rank_decode_attn_noalloc",
+    "unipin_rank_decode_noalloc_scratch_bytes",
 )
 
 
@@ -73,6 +75,10 @@ def _load(path: str = _LIB_PATH):
     lib.unipin_selftest_bounded_wait.restype = I
     lib.unipin_selftest_exp2.argtypes = [P, P, I, P]
     lib.unipin_selftest_exp2.restype = I
+    lib.unipin_rank_decode_attn_noalloc.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, F, P, I, P, P]
+    lib.unipin_rank_decode_attn_noalloc.restype = I
+    lib.unipin_rank_decode_noalloc_scratch_bytes.argtypes = []
+    lib.unipin_rank_decode_noalloc_scratch_bytes.restype = SZ
     return lib
 
 
@@ -211,6 +217,39 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
                                      _ptr(dev_status), _stream(stream))
     _check(rc, "unipin_rank_decode_attn")
     return out
+
+
+def rank_decode_attn_noalloc(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, pool_v, layer: int,
+                             max_k: int, out, out_fp32: bool = True, scale: Optional[float] = None,
+                             dev_status=None, stream=None):
+    """Rank decode through the entry point that allocates nothing (the caller passes `out`).
+
+    For callers that cannot allocate device memory while serving: the scratch
+    lives in a fixed device array inside the library, shared by every call, so
+    calls must not overlap on the GPU.
+    """
+    _tokens(q_c, "q_c")
+    T, H, D = q_c.shape
+    _tokens(k_c, "k_c", D)
+    _tokens(v_c, "v_c", D)
+    pool = _pool(pool_k, pool_v)
+    R = past_lens.shape[0]
+    _index(cu_seqlens_c, "cu_seqlens_c", R + 1)
+    _index(slot_ids, "slot_ids", R)
+    _index(past_lens, "past_lens", R)
+    if out.dtype != (torch.float32 if out_fp32 else torch.bfloat16) or out.shape != q_c.shape or not out.is_contiguous():
+        raise ValueError("out has the wrong dtype or shape")
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    rc = LIB.unipin_rank_decode_attn_noalloc(_ptr(q_c), _ptr(k_c), _ptr(v_c), _ptr(out), int(bool(out_fp32)),
+                                             _ptr(cu_seqlens_c), _ptr(slot_ids), _ptr(past_lens), R, H, D,
+                                             int(max_k), T, scale, ctypes.byref(pool), int(layer),
+                                             _ptr(dev_status), _stream(stream))
+    _check(rc, "unipin_rank_decode_attn_noalloc")
+    return out
+
+
+def rank_decode_noalloc_scratch_bytes() -> int:
+    return int(LIB.unipin_rank_decode_noalloc_scratch_bytes())
 
 
 def selftest_bounded_wait(dev_status, limit_us: int, stream=None):

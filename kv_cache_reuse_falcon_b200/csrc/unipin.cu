@@ -234,6 +234,30 @@ __global__ void bounded_wait_selftest_kernel(int* status, unsigned long long lim
     __syncthreads();
 }
 
+// Scratch for unipin_rank_decode_attn_noalloc: device memory the library
+// owns from the moment the module loads on a device until the process exits,
+// so callers of that entry point never allocate.  Host code only sees a
+// stand-in for this symbol; its device address comes from
+// cudaGetSymbolAddress, looked up once per device.
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;   // 32 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+void* g_noalloc_addr[kMaxDevices] = {};
+
+int noalloc_scratch_address(void** addr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return UNIPIN_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_init_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void* a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_noalloc_scratch) != cudaSuccess || a == nullptr) return UNIPIN_ERR_CUDA;
+        g_noalloc_addr[dev] = a;
+    }
+    *addr = g_noalloc_addr[dev];
+    return UNIPIN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -418,6 +442,26 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     }
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
+
+int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
+                                    const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R,
+                                    int H, int D, int max_k, int total_cand, float scale,
+                                    const unipin_kvpool* pool, int layer, int* dev_status, void* stream)
+{
+    if (!pool) return UNIPIN_ERR_INVALID_ARG;
+    if (R < 0 || H < 1 || max_k < 0 || total_cand < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
+    if (R == 0 || total_cand == 0 || max_k == 0) return UNIPIN_OK;
+    const size_t need = unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand, pool->n_cap);
+    if (need > kNoAllocScratchBytes) return UNIPIN_ERR_OUT_OF_RANGE;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch_address(&scratch);
+    if (rc != UNIPIN_OK) return rc;
+    return unipin_rank_decode_attn(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, slot_ids, past_lens, R, H, D, max_k,
+                                   total_cand, scale, pool, layer, scratch, kNoAllocScratchBytes, dev_status, stream);
+}
+
+size_t unipin_rank_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
 
 int unipin_selftest_exp2(const float* x, float* y, int n, void* stream)
 {

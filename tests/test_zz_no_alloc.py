@@ -1,0 +1,74 @@
+"""The allocation-free rank decode entry point, checked against the regular one.
+
+unipin_rank_decode_attn_noalloc serves callers that cannot allocate device
+memory while they run (their memory belongs to another framework's pool, or
+their serving loop must not allocate after start-up): its scratch is a fixed
+array inside the library.  This file is collected last on purpose, so a
+failure here leaves every other test already run; it also passes alone.
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_reuse_falcon_b200 import synth
+from tests.gpu_helpers import DevDecode, fill_pool_rows, nan_pool, parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ub():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from kv_cache_reuse_falcon_b200 import binding
+    return binding
+
+
+def _setup(seed, past, cand, H, D, S, n_cap, layer):
+    rng = np.random.Generator(np.random.PCG64(seed))
+    d = synth.make_decode(seed, past, cand, H, D, n_slots=S, rng=rng)
+    ks, vs = synth.pool_rows(rng, past, H, D)
+    pk, pv = nan_pool(layer + 1, S, H, n_cap, D)
+    fill_pool_rows(pk, pv, layer, d.slot_ids, past, ks, vs)
+    return d, DevDecode(d), pk, pv
+
+
+@pytest.mark.parametrize("shape", [
+    # small k: the split-n partial results live in the library's array
+    ([2048] * 8, [16] * 8, 4, 64, 12, 2048),
+    # ragged lengths, one request without history, D=128
+    ([700, 0, 1500, 129], [300, 40, 260, 128], 4, 128, 6, 1536),
+])
+def test_noalloc_decode_matches_regular_decode_twice_in_a_row(ub, shape):
+    past, cand, H, D, S, n_cap = shape
+    layer = 1
+    d, dd, pk, pv = _setup(7000, past, cand, H, D, S, n_cap, layer)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ref = ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, layer, dd.max_k,
+                              out_fp32=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for _ in range(2):   # the shared array keeps the previous call's contents
+        out = torch.full_like(ref, float("nan"))
+        ub.rank_decode_attn_noalloc(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, layer, dd.max_k,
+                                    out, out_fp32=True, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        parity(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "no-alloc decode")
+
+
+def test_noalloc_decode_rejects_requests_beyond_its_array(ub):
+    """A shape whose split-n scratch exceeds the fixed array returns OUT_OF_RANGE and launches nothing."""
+    limit = ub.rank_decode_noalloc_scratch_bytes()
+    H, D, n_cap = 4, 128, 4096
+    R, k = 37, 256          # 148 (request, head) units: under two waves of blocks, so the sweep splits
+    need = ub.rank_decode_workspace_size(R, H, D, k, R * k, n_cap)
+    assert need > limit
+    P, I = ctypes.c_void_p, ctypes.c_int
+    pool = ub.KVPool(16, 16, 1, 1, H, n_cap, D)      # never dereferenced: the call returns first
+    rc = ub.LIB.unipin_rank_decode_attn_noalloc(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), R, H, D,
+                                                k, R * k, 0.1, ctypes.byref(pool), 0, None, None)
+    assert rc == -4
