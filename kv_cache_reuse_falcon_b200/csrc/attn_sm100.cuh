@@ -703,10 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int e = half * 64 + 2 * c;
                         const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2);
                         float p0, p1;
-                        // (the diagonal tile's live entry sits at the row's own column,
-                        // which differs between a prefill and a decode tile: it always
-                        // takes the MUFU path so both give the same bits)
-                        if ((c & 3) == 3 && !diag) {
+                        if ((c & 3) == 3) {
                             exp2_poly2(x2, p0, p1);
                         } else {
                             float x0, x1;
