@@ -11,16 +11,14 @@
 // The same engine runs the prefill and the rank decode.  In both, the part
 // of a row's key set that is a contiguous run of keys 0..kmax-1 goes through
 // the tensor cores with the causal predicate j <= i, and a candidate's own
-// key (the diagonal of the candidate block) comes from one extra "diagonal"
-// key tile holding the keys of the tile's own rows, masked to j == i:
+// key (the diagonal of the candidate block) is merged in afterwards as a
+// per-row fp32 dot product:
 //   prefill ([notes] §3 "attention mask"):  past row i sees j <= i < n_b;
-//       candidate row i >= n_b sees all j < n_b plus itself.
+//       candidate row i >= n_b sees all j < n_b plus itself (self term).
 //   rank decode ([review] §2.4, [notes] §6):  keys are pool rows 0..n_r-1 of
 //       the request's slot; every candidate sees all of them plus itself.
-// Both sweep the same key tiles in the same order, so a candidate's prefill
-// row and its decode row come out bit-identical.  Key tiles past kmax are
-// never visited; key tiles entirely below the diagonal and below kmax skip
-// the per-element predicate.
+// Key tiles past kmax are never visited; key tiles entirely below the
+// diagonal and below kmax skip the per-element predicate.
 //
 // Warp roles (384 threads):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns
@@ -81,6 +79,9 @@ struct AttnCfg {
 };
 
 struct AttnParams {
+    const __nv_bfloat16* q;       // [T, H, D] query-side tokens
+    const __nv_bfloat16* k_self;  // [T, H, D] key of each query token (self term)
+    const __nv_bfloat16* v_self;  // [T, H, D] value of each query token (self term)
     void* out;                    // [T, H, D] fp32 or bf16
     float* part_o;                // split-n partials [nsplit, T, H, D] (decode, nsplit > 1)
     float* part_ml;               // split-n row stats [nsplit, T, H, 2] = (m in log2 units, l)
@@ -198,9 +199,7 @@ struct Work {
     int pos0;                   // mask position of row 0 of tile A
     int kmax_a, kmax_b, kmax;   // key ranges; tile geometry follows kmax
     int nt_all, t_begin;
-    int nt_a, nt_b, nt;         // regular key tiles swept for A, B, and loaded
-    int nd_a, nd_b;             // 1 if tile A / B also sweeps its diagonal tile (own keys)
-    int uses;                   // ring uses of the item: 2 * (nt + nd_a + nd_b)
+    int nt_a, nt_b, nt;         // key tiles swept for A, B, and loaded
 };
 
 template <bool kDecode>
@@ -250,35 +249,13 @@ __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int loca
     w.nt_b = w.has_b ? max(t_end_b - w.t_begin, 0) : 0;
     w.nt = w.valid ? max(w.nt_a, w.nt_b) : 0;
     if (!w.valid) w.nt_a = w.nt_b = 0;
-    // Candidate rows see their own key: a tile holding any candidate row also
-    // sweeps its "diagonal" key tile (the keys of its own rows, mask j == i).
-    // In a split decode sweep the last split takes it.
-    const bool last_split = !kDecode || w.split == p.nsplit - 1;
-    w.nd_a = (w.valid && last_split && w.nrows_a > 0 && (kDecode || w.qrow0 + w.nrows_a > w.npast)) ? 1 : 0;
-    w.nd_b = (w.valid && last_split && w.has_b && (kDecode || w.qrow0 + kBlockM + w.nrows_b > w.npast)) ? 1 : 0;
-    w.uses = 2 * (w.nt + w.nd_a + w.nd_b);
     return w;
-}
-
-// Ring use u of an item: regular key tile u/2 for u < 2*nt, then the
-// diagonal tile of A (if any), then that of B.  Returns the query tile that
-// owns it (0 = A, 1 = B, 2 = both) and, for a diagonal use, marks it.
-__device__ __forceinline__ int use_owner(const Work& w, int u, bool& diag)
-{
-    if (u < 2 * w.nt) {
-        diag = false;
-        const int t = u / 2;
-        return (t < w.nt_a && t < w.nt_b) ? 2 : (t < w.nt_a ? 0 : 1);
-    }
-    diag = true;
-    return (u < 2 * w.nt + 2 * w.nd_a) ? 0 : 1;
 }
 
 template <int D, bool kDecode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_ks,
-                    const __grid_constant__ CUtensorMap tm_vs, const AttnParams p)
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p)
 {
     using C = AttnCfg<D>;
     constexpr int NS = C::kStages;
@@ -371,8 +348,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_prefetch_map(&tm_q);
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
-            tma_prefetch_map(&tm_ks);
-            tma_prefetch_map(&tm_vs);
         }
         int u = 0;          // ring uses issued so far (use u lives in slot u % NS)
         int nq = 0;         // Q loads issued so far
@@ -405,7 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (leader) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
                 continue;
             }
-            if (w.uses == 0) continue;
+            if (w.nt == 0) continue;
             // Q of this item may overwrite Q of the previous one once its S MMAs are done.
             if (nq > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(q_empty, (nq - 1) & 1, ctl));
@@ -441,26 +416,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, w.h,
                                             w.tok0 + start);
                         }
-                    }
-                    ++u;
-                }
-            }
-            // diagonal tiles: the keys and values of tile A's / B's own rows
-            for (int x = 0; ok && x < 2; ++x) {
-                if ((x == 0 ? w.nd_a : w.nd_b) == 0) continue;
-                for (int kv = 0; kv < 2; ++kv) {
-                    const int st = u % NS;
-                    if (u >= NS) {
-                        ok = __all_sync(0xffffffffu, mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl));
-                        if (!ok) break;
-                    }
-                    if (leader) {
-                        mbar_arrive_expect_tx(kv_full + st, C::kTileBytes);
-                        const CUtensorMap* map = kv == 0 ? &tm_ks : &tm_vs;
-                        uint8_t* dst = ring + st * C::kTileBytes;
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, w.h,
-                                        w.tok0 + w.qrow0 + x * kBlockM);
                     }
                     ++u;
                 }
@@ -526,76 +481,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         auto wait_fill = [&](int u) {
             return __all_sync(0xffffffffu, mbar_wait(kv_full + u % NS, (u / NS) & 1, ctl));
         };
-        int u0 = 0;                // ring uses of earlier items
+        int u = 0;                 // ring uses consumed
         int nq = 0;                // items with MMAs
         int np = 0;                // p_full completions consumed
         bool ok = true;
         while (pop_item(ok)) {
             const Work w = make_work<kDecode>(p, seg, local);
-            if (w.uses == 0) continue;
+            if (w.nt == 0) continue;
             const int ntx = x == 0 ? w.nt_a : w.nt_b;
-            const int ndx = x == 0 ? w.nd_a : w.nd_b;
-            const int ntiles = ntx + ndx;              // this tile's key tiles, diagonal last
-            // ring use of this tile's key tile t (K; its V is the next use)
-            auto kuse = [&](int t) {
-                return u0 + (t < ntx ? 2 * t : 2 * w.nt + (x == 1 ? 2 * w.nd_a : 0));
-            };
-            int rp = u0;   // ring uses below rp are handled (released or consumed)
-            // Release, in ring order, every use below `upto` this tile does not
-            // consume: only after its fill, so both warps' arrivals stay in phase.
-            auto release_others = [&](int upto) -> bool {
-                for (; rp < upto; ++rp) {
-                    bool dg;
-                    const int own = use_owner(w, rp - u0, dg);
-                    if (own == 2 || own == x) continue;          // consumed (and released) by this warp
-                    if (!__all_sync(0xffffffffu, mbar_wait(kv_full + rp % NS, (rp / NS) & 1, ctl))) return false;
-                    if (leader) mbar_arrive(kv_empty + rp % NS);
-                }
-                return true;
-            };
             // Q landed: this also means both warps released the previous Q.
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_q, nq & 1, ctl));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_q, nq & 1, ctl)) && wait_fill(u);
             if (!ok) break;
-            if (ntiles == 0) {
-                if (leader) mbar_arrive(q_empty);
-            } else {
-                const int k0 = kuse(0);
-                ok = release_others(k0) && wait_fill(k0);
-                if (!ok) break;
-                tc_fence_after_sync();
-                if (leader) {
-                    issue_qk(k0 % NS);
-                    umma_commit(kv_empty + k0 % NS);
-                    if (ntiles == 1) umma_commit(q_empty);   // no S MMA of this tile after this
+            tc_fence_after_sync();
+            if (leader) {
+                if (ntx > 0) {
+                    issue_qk(u % NS);
+                    umma_commit(kv_empty + u % NS);                 // K_0
+                    if (ntx == 1) umma_commit(q_empty);            // no S MMA of this tile after this
+                } else {
+                    mbar_arrive(kv_empty + u % NS);
+                    mbar_arrive(q_empty);
                 }
-                for (int t = 0; ok && t < ntiles; ++t) {
-                    const int uv = kuse(t) + 1;
-                    if (!(ok = release_others(uv) && wait_fill(uv))) break;
+            }
+            for (int i = 0; ok && i < w.nt; ++i) {
+                const int uv = u + 1;          // V_i
+                const int uk = u + 2;          // K_{i+1}
+                if (!(ok = wait_fill(uv))) break;
+                if (i < ntx) {
                     ok = __all_sync(0xffffffffu, mbar_wait(p_full + x, np & 1, ctl));
                     if (!ok) break;
                     ++np;
                     tc_fence_after_sync();
-                    if (leader) issue_pv(uv % NS, t > 0);
-                    if (t + 1 < ntiles) {
-                        const int uk = kuse(t + 1);
-                        if (!(ok = release_others(uk) && wait_fill(uk))) break;
+                    if (leader) issue_pv(uv % NS, i > 0);
+                    if (i + 1 < ntx) {
+                        if (!(ok = wait_fill(uk))) break;
                         tc_fence_after_sync();
                         if (leader) {
                             issue_qk(uk % NS);
-                            umma_commit(kv_empty + uk % NS);
-                            if (t + 2 == ntiles) umma_commit(q_empty);   // that was this tile's last S MMA
+                            if (i + 2 == ntx) umma_commit(q_empty);   // that was this tile's last S MMA
                         }
                     } else if (leader) {
                         umma_commit(o_full + x);
                     }
                     if (leader) umma_commit(kv_empty + uv % NS);
-                    rp = uv + 1 > rp ? uv + 1 : rp;
+                } else if (leader) {
+                    mbar_arrive(kv_empty + uv % NS);
                 }
-                if (!ok) break;
+                if (i + 1 < w.nt) {
+                    if (i + 1 >= ntx) {
+                        // K_{i+1} is only for the other tile: release it once it has landed
+                        if (!(ok = wait_fill(uk))) break;
+                        if (leader) mbar_arrive(kv_empty + uk % NS);
+                    } else if (leader) {
+                        umma_commit(kv_empty + uk % NS);
+                    }
+                }
+                u += 2;
             }
-            // everything after this tile's last use
-            if (!(ok = release_others(u0 + w.uses))) break;
-            u0 += w.uses;
             ++nq;
         }
         if (leader) {
@@ -629,17 +571,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_valid = r < nrows_x;
             const long long tok = (long long)w.tok0 + w.qrow0 + x * kBlockM + r;
             const size_t base = ((size_t)tok * p.H + w.h) * D;
+            // self term: a candidate row's own key (prefill rows i >= n_b; every decode row)
+            const bool self = row_valid && !split_mode && (kDecode || irow >= w.npast);
+            float ss = -INFINITY;
+            if (self) {
+                // issued before the first S wait so its latency overlaps the MMAs
+                const uint4* q4 = reinterpret_cast<const uint4*>(p.q + base);
+                const uint4* k4 = reinterpret_cast<const uint4*>(p.k_self + base);
+                float dot0 = 0.f, dot1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint4 qa = __ldg(q4 + c), ka = __ldg(k4 + c);
+                    const __nv_bfloat162* qh = reinterpret_cast<const __nv_bfloat162*>(&qa);
+                    const __nv_bfloat162* kh = reinterpret_cast<const __nv_bfloat162*>(&ka);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 qf = __bfloat1622float2(qh[e]);
+                        const float2 kf = __bfloat1622float2(kh[e]);
+                        dot0 = fmaf(qf.x, kf.x, dot0);
+                        dot1 = fmaf(qf.y, kf.y, dot1);
+                    }
+                }
+                ss = (dot0 + dot1) * sl2;
+            }
             float m = -INFINITY;     // reference max (log2 units) the P values and O are relative to
             float l = 0.f;           // row sum relative to m
-            const int ndx = x == 0 ? w.nd_a : w.nd_b;
-            // a candidate row's own key: the diagonal of the last (diagonal) tile
-            const bool cand_row = kDecode || irow >= w.npast;
-            for (int i = 0; i < ntx + ndx; ++i) {
-                const bool diag = i == ntx;
-                int start = 0, lo = 0;
-                if (!diag) key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
-                const bool full_tile = !diag && (start == lo) && (start + kBlockN <= kmax_x) &&
-                                       (start + kBlockN - 1 <= posx0);
+            for (int i = 0; i < ntx; ++i) {
+                int start, lo;
+                key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
+                const bool full_tile = (start == lo) && (start + kBlockN <= kmax_x) && (start + kBlockN - 1 <= posx0);
                 // warp-uniform: the TMEM accesses below are warp-collective
                 ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, ns & 1, ctl));
                 if (!ok) break;
@@ -647,11 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after_sync();
                 uint32_t s[kBlockN];
                 tmem_ld128(tS, s);
-                if (diag) {
-#pragma unroll
-                    for (int e = 0; e < kBlockN; ++e)
-                        if (!(e == r && cand_row)) s[e] = 0xff800000u;   // -inf
-                } else if (!full_tile) {
+                if (!full_tile) {
 #pragma unroll
                     for (int e = 0; e < kBlockN; ++e) {
                         const int j = start + e;
@@ -714,10 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
                         pk[c] = pack_bf16x2(p0, p1);
                     }
-                    if (half == 0)
-                        tmem_st32_nowait(tS, pk);    // its latency overlaps the second half
-                    else
-                        tmem_st32(tS + 32, pk);      // waits for both halves
+                    tmem_st32(tS + half * 32, pk);
                 }
                 {
                     const uint64_t a01 = f2_add(acc[0], acc[1]);
@@ -730,19 +683,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(p_full + x);
             }
             if (!ok) break;
-            // ---- epilogue: O / l (the own key already went through the diagonal tile)
-            const int nall = ntx + ndx;
-            if (nall > 0) {
+            // ---- epilogue: the own value (self term) is fetched before waiting for O
+            uint4 vr[D / 8];
+            {
+                const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + base);
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) vr[c] = self ? __ldg(v4 + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (ntx > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(o_full + x, no & 1, ctl));
                 if (!ok) break;
                 ++no;
                 tc_fence_after_sync();
             }
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            float a = 1.f, b = 0.f, inv = 0.f;
+            if (row_valid && !split_mode) {
+                const float m_fin = fmaxf(m, ss);
+                a = (m == -INFINITY) ? 0.f : ex2_approx(m - m_fin);
+                b = self ? ex2_approx(ss - m_fin) : 0.f;
+                const float denom = l * a + b;
+                inv = denom > 0.f ? 1.f / denom : 0.f;
+            }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
-                if (nall > 0) {
+                if (ntx > 0) {
                     tmem_ld32(tO + c * 32, o);   // warp-collective: every lane loads
                 } else {
 #pragma unroll
@@ -759,7 +724,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (row_valid && !split_mode) {
                     float res[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) res[e] = __uint_as_float(o[e]) * inv;
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 va = vr[c * 4 + q];
+                        const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&va);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 vf = __bfloat1622float2(vh[e]);
+                            res[q * 8 + 2 * e] = (__uint_as_float(o[q * 8 + 2 * e]) * a + b * vf.x) * inv;
+                            res[q * 8 + 2 * e + 1] = (__uint_as_float(o[q * 8 + 2 * e + 1]) * a + b * vf.y) * inv;
+                        }
+                    }
                     if (p.out_fp32) {
                         float* dst = reinterpret_cast<float*>(p.out) + base + c * 32;
 #pragma unroll
@@ -807,24 +781,40 @@ __global__ void exp2_poly_selftest_kernel(const float* __restrict__ x, float* __
 }
 
 // Split-n merge for the rank decode: each (candidate, head) row combines the
-// nsplit partial results (O relative to 2^m, m in log2 units, l) of its key
-// sweep; the candidate's own key was in the last split's diagonal tile.
+// nsplit partial (O, m, l) of its pool sweep with its own key (self term).
+// One warp per row; the self dot product is reduced with warp shuffles.
 template <int D>
 __global__ void __launch_bounds__(256)
-    decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml, void* out,
-                        int out_fp32, int total_rows, int H, int nsplit)
+    decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
+                        const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_self,
+                        const __nv_bfloat16* __restrict__ v_self, void* out, int out_fp32, int total_rows, int H,
+                        int nsplit, float sl2)
 {
     constexpr int E = D / 32;   // elements per lane
     const int lane = threadIdx.x % 32;
     const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;   // tok * H + h
     if (row >= (long long)total_rows * H) return;
     const size_t base = (size_t)row * D + lane * E;
-    float m_fin = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) m_fin = fmaxf(m_fin, part_ml[((size_t)s * total_rows * H + row) * 2]);
-    float acc[E];
+    float dot = 0.f;
+    float vv[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    float den = 0.f;
+    for (int e = 0; e < E; ++e) {
+        dot = fmaf(__bfloat162float(q[base + e]), __bfloat162float(k_self[base + e]), dot);
+        vv[e] = __bfloat162float(v_self[base + e]);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    const float ss = dot * sl2;
+    float m_fin = ss;
+    for (int s = 0; s < nsplit; ++s) {
+        const float ms = part_ml[((size_t)s * total_rows * H + row) * 2];
+        m_fin = fmaxf(m_fin, ms);
+    }
+    float acc[E];
+    const float bself = ex2_approx(ss - m_fin);
+    float den = bself;
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = bself * vv[e];
     for (int s = 0; s < nsplit; ++s) {
         const float ms = part_ml[((size_t)s * total_rows * H + row) * 2];
         const float ls = part_ml[((size_t)s * total_rows * H + row) * 2 + 1];
@@ -835,7 +825,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = fmaf(w, po[e], acc[e]);
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
+    const float inv = 1.f / den;
     if (out_fp32) {
         float* dst = reinterpret_cast<float*>(out) + base;
 #pragma unroll

@@ -150,17 +150,17 @@ bool supported_d(int D) { return D == 32 || D == 64 || D == 128; }
 
 template <bool kDecode>
 int launch_attn(int D, dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const CUtensorMap& tks, const CUtensorMap& tvs, const AttnParams& p, cudaStream_t s)
+                const AttnParams& p, cudaStream_t s)
 {
     switch (D) {
     case 32:
-        attn_fwd_kernel<32, kDecode><<<grid, kThreads, AttnCfg<32>::kSmemBytes, s>>>(tq, tk, tv, tks, tvs, p);
+        attn_fwd_kernel<32, kDecode><<<grid, kThreads, AttnCfg<32>::kSmemBytes, s>>>(tq, tk, tv, p);
         break;
     case 64:
-        attn_fwd_kernel<64, kDecode><<<grid, kThreads, AttnCfg<64>::kSmemBytes, s>>>(tq, tk, tv, tks, tvs, p);
+        attn_fwd_kernel<64, kDecode><<<grid, kThreads, AttnCfg<64>::kSmemBytes, s>>>(tq, tk, tv, p);
         break;
     case 128:
-        attn_fwd_kernel<128, kDecode><<<grid, kThreads, AttnCfg<128>::kSmemBytes, s>>>(tq, tk, tv, tks, tvs, p);
+        attn_fwd_kernel<128, kDecode><<<grid, kThreads, AttnCfg<128>::kSmemBytes, s>>>(tq, tk, tv, p);
         break;
     default:
         return UNIPIN_ERR_UNSUPPORTED;
@@ -315,6 +315,9 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     if ((rc = make_token_map(&tv, v, total_tokens, H, D)) != UNIPIN_OK) return rc;
 
     AttnParams p = {};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k_self = static_cast<const __nv_bfloat16*>(k);
+    p.v_self = static_cast<const __nv_bfloat16*>(v);
     p.out = out;
     p.cu = cu_seqlens;
     p.past = past_lens;
@@ -331,7 +334,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.sched = sched;
     const long long bound = (long long)B * H * ((max_seqlen + kPairRows - 1) / kPairRows);
     dim3 grid(persistent_blocks(bound), 1, 1);
-    return launch_attn<false>(D, grid, tq, tk, tv, tk, tv, p, s);   // own keys: the same K/V
+    return launch_attn<false>(D, grid, tq, tk, tv, p, s);
 }
 
 int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, const void* v, const int* cu_seqlens,
@@ -386,14 +389,15 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
         if (cudaMemsetAsync(sched, 0, sizeof(unsigned long long), s) != cudaSuccess) return UNIPIN_ERR_CUDA;
     }
 
-    CUtensorMap tq, tk, tv, tks, tvs;
+    CUtensorMap tq, tk, tv;
     if ((rc = make_token_map(&tq, q_c, total_cand, H, D)) != UNIPIN_OK) return rc;
     if ((rc = make_pool_map(&tk, pool->k, pool)) != UNIPIN_OK) return rc;
     if ((rc = make_pool_map(&tv, pool->v, pool)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tks, k_c, total_cand, H, D)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tvs, v_c, total_cand, H, D)) != UNIPIN_OK) return rc;
 
     AttnParams p = {};
+    p.q = static_cast<const __nv_bfloat16*>(q_c);
+    p.k_self = static_cast<const __nv_bfloat16*>(k_c);
+    p.v_self = static_cast<const __nv_bfloat16*>(v_c);
     p.out = out;
     p.cu = cu_seqlens_c;
     p.past = past_lens;
@@ -417,20 +421,23 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     }
     const long long bound = (long long)R * H * nsplit * ((max_k + kPairRows - 1) / kPairRows);
     dim3 grid(persistent_blocks(bound), 1, 1);
-    rc = launch_attn<true>(D, grid, tq, tk, tv, tks, tvs, p, s);
+    rc = launch_attn<true>(D, grid, tq, tk, tv, p, s);
     if (rc != UNIPIN_OK || nsplit == 1) return rc;
 
     const long long rows = (long long)total_cand * H;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
     switch (D) {
     case 32:
-        decode_merge_kernel<32><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, out, p.out_fp32, total_cand, H, nsplit);
+        decode_merge_kernel<32><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
+                                                       p.out_fp32, total_cand, H, nsplit, p.sl2);
         break;
     case 64:
-        decode_merge_kernel<64><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, out, p.out_fp32, total_cand, H, nsplit);
+        decode_merge_kernel<64><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
+                                                       p.out_fp32, total_cand, H, nsplit, p.sl2);
         break;
     default:
-        decode_merge_kernel<128><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, out, p.out_fp32, total_cand, H, nsplit);
+        decode_merge_kernel<128><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
+                                                        p.out_fp32, total_cand, H, nsplit, p.sl2);
         break;
     }
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
