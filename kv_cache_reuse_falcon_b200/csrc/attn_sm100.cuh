@@ -670,7 +670,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
                         pk[c] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st32(tS + half * 32, pk);
+                    if (half == 0)
+                        tmem_st32_nowait(tS, pk);    // its latency overlaps the second half
+                    else
+                        tmem_st32(tS + 32, pk);      // waits for both halves
                 }
                 {
                     const uint64_t a01 = f2_add(acc[0], acc[1]);
