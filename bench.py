@@ -381,6 +381,99 @@ def run_ours(args, rank, world, device, dist):
     return result
 
 
+def run_decode_only(args, rank, world, device, dist):
+    """Rank decode workload: R requests over an L-layer pool, one call per layer per step."""
+    import torch
+    from kv_cache_reuse_falcon_b200 import binding as ub
+
+    w = synth.workload(args.workload)
+    seed = rank_seed(w.seed, rank)
+    rng = np.random.Generator(np.random.PCG64(seed))
+    kk = args.k if args.k > 0 else w.k
+    past = np.full(w.B, w.n, np.int32)
+    cand = np.full(w.B, kk, np.int32)
+    H, D, L, S, n_cap = w.H, w.D, w.L, w.S, w.n_cap
+    slots = rng.permutation(S)[: w.B].astype(np.int32)
+
+    def dev_bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    pool_k = torch.full((L, S, H, n_cap, D), 0x7FC0, dtype=torch.int16, device=device).view(torch.bfloat16)
+    pool_v = torch.full((L, S, H, n_cap, D), 0x7FC0, dtype=torch.int16, device=device).view(torch.bfloat16)
+    for layer in range(L):                     # cached rows of every request, every layer
+        ks, vs = synth.pool_rows(rng, past, H, D)
+        for r in range(w.B):
+            pool_k[layer, int(slots[r]), :, : w.n] = dev_bf16(ks[r])
+            pool_v[layer, int(slots[r]), :, : w.n] = dev_bf16(vs[r])
+    Tc = int(cand.sum())
+    qs, kc, vc = [], [], []
+    for layer in range(L):                     # fresh candidate q/k/v per layer
+        qs.append(dev_bf16(synth.normal_bf16(rng, (Tc, H, D))))
+        kc.append(dev_bf16(synth.normal_bf16(rng, (Tc, H, D))))
+        vc.append(dev_bf16(synth.normal_bf16(rng, (Tc, H, D))))
+    cu = torch.from_numpy(synth.cu_from_lens(cand)).to(device)
+    pl = torch.from_numpy(past).to(device)
+    sl = torch.from_numpy(slots).to(device)
+    out = [torch.empty((Tc, H, D), dtype=torch.bfloat16, device=device) for _ in range(L)]
+    ws_bytes = ub.rank_decode_workspace_size(w.B, H, D, kk, Tc, n_cap)
+    ws = torch.empty(ws_bytes // 4 + 4, dtype=torch.float32, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(ev=None):
+        for layer in range(L):
+            if ev is not None and layer == 0:
+                ev[0].record(stream)
+            ub.rank_decode_attn(qs[layer], kc[layer], vc[layer], cu, sl, pl, pool_k, pool_v, layer, kk,
+                                out=out[layer], out_fp32=False, workspace=ws, dev_status=status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(device)
+    clk = clocks.stop() if clocks else None
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %s" % ub.status_string(int(status.item())))
+    ms_step = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    peaks = load_peaks()
+    flops = decode_flops(past, cand, H, D) * L
+    nbytes = decode_bytes(past, cand, H, D, 2) * L
+    tflops = flops / (ms_step * 1e-3) / 1e12
+    gbs = nbytes / (ms_step * 1e-3) / 1e9
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    roof = ({"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": gbs / peaks["hbm_gbs"]} if bound == "hbm" else
+            {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+             "frac": tflops / peaks["bf16_tflops"]})
+    roof.update({"kernel": "attn_fwd_kernel<%d,decode>" % D, "traffic": None,
+                 "peak_source": "%s (burst for tensor)" % peaks["source"]})
+    return {
+        "metric": METRIC, "value": float(cand.sum()) * L / (ms_step * 1e-3), "unit": "candidate tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
+                   "pool": [L, S, H, n_cap, D], "layers_per_step": L, "split_n": ws_bytes > 256,
+                   "l2": "pool slots read per step exceed L2 (no flush)"},
+        "phases": {"decode_tflops": tflops, "decode_gbs": gbs, "decode_frac_hbm": gbs / peaks["hbm_gbs"],
+                   "decode_frac_tensor": tflops / peaks["bf16_tflops"],
+                   "roof_time_ms": 1e3 * max(t_hbm, t_tc)},
+        "roofline": roof, "gpu_launches": args.steps * L * (2 if ws_bytes > 256 else 1), "clocks": clk,
+    }
+
+
 def run_reference(args, rank, world):
     """The oracle (fp64 CPU) timed on the host cores, a bounded sample of the same workload per step."""
     if rank != 0:
@@ -430,6 +523,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--users", type=int, default=0, help="smaller case: this many users (profiling)")
+    ap.add_argument("--k", type=int, default=0, help="decode workloads: candidates per request")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -454,7 +548,10 @@ def main(argv=None):
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=device)
         dist = tdist
     try:
-        res = run_ours(args, rank, world, device, dist)
+        if synth.workload(args.workload).kind == "decode":
+            res = run_decode_only(args, rank, world, device, dist)
+        else:
+            res = run_ours(args, rank, world, device, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()
