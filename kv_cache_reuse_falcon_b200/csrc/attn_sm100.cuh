@@ -24,10 +24,13 @@
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r owns
 //              query row r = TMEM lane r, so the row max and row sum stay in
 //              one thread's registers; S is read from TMEM with one wide load,
-//              P (bf16) is written back into TMEM over S and consumed from
+//              P (bf16) is written to its own TMEM columns and consumed from
 //              there by the P.V MMA.  The O accumulator is rescaled in TMEM
 //              only when a row max grows by more than 2^8 (stale maxima keep
 //              P <= 2^8, exact after the final division).
+//              Because P does not overwrite S, the next key tile's S = Q K^T
+//              is computed while this tile's softmax runs: the tensor cores
+//              never wait for a softmax to finish before starting on the next S.
 //   warp 8     TMA producer: per item the Q tiles, then K_0, V_0, K_1, V_1, ...
 //              through a ring of shared-memory slots (the ring runs across items).
 //   warps 9, 10 the UMMA issuers of tile A and tile B (one elected thread each);
@@ -35,8 +38,10 @@
 //   warp 11    idle (it completes the third warpgroup for the register split).
 // Every warp walks the same item sequence (ItemWalker), so no queue is shared.
 //
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B [256+D, 256+2D);
-// P_X occupies the first 64 columns of S_X.
+// Key tiles are kN = 64 keys wide at D = 128 and 128 keys otherwise, so that
+// each query tile's S (kN columns), P (kN/2 columns of bf16 pairs) and O (D
+// columns) fit its half of the 512 TMEM columns:
+//   tile X: S at 256X, P at 256X + kN, O at 256X + 256 - D.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -46,36 +51,50 @@
 namespace unipin {
 
 constexpr int kBlockM = 128;     // query rows per tile = TMEM lanes
-constexpr int kBlockN = 128;     // keys per tile
 constexpr int kPairRows = 2 * kBlockM;
 constexpr int kThreads = 384;
 // Register split: the block launches with kLaunchRegs per thread (the most
 // 384 threads can have); the producer/MMA warpgroup gives registers back and
-// the two softmax warpgroups take them: 128*72 + 256*216 = 384*168.
+// the two softmax warpgroups take them (per head dim, in AttnCfg).
 constexpr int kLaunchRegs = 168;
 constexpr int kItemSlots = 4;        // items handed from the producer warp to the others
 constexpr int kItemConsumers = 10;   // the two MMA warps and the eight softmax warps
-constexpr int kRegsOther = 96;
-constexpr int kRegsSoftmax = 200;
-static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when a row max grows by > 2^8
 
+// Key tile width (keys per S tile) for head dim D.
+__host__ __device__ constexpr int key_tile_width(int D) { return D == 128 ? 64 : 128; }
+
 template <int D>
 struct AttnCfg {
     static_assert(D == 32 || D == 64 || D == 128, "head dim");
+    static constexpr int kN = key_tile_width(D);                // keys per K/V tile
     static constexpr int kBoxD = D >= 64 ? 64 : D;              // elements per TMA box row
     static constexpr int kChunks = D / kBoxD;                   // boxes across D
     static constexpr int kRowBytes = kBoxD * 2;                 // 128 (SW128) or 64 (SW64)
     static constexpr uint32_t kLayout = kRowBytes == 128 ? kLayoutSw128 : kLayoutSw64;
-    static constexpr int kAtomBytes = kBlockM * kRowBytes;      // one box of 128 rows
-    static constexpr int kTileBytes = kBlockM * D * 2;          // one Q, K or V tile
-    static constexpr int kStages = D == 128 ? 4 : 8;            // ring slots (each one K or one V tile)
+    static constexpr int kAtomQ = kBlockM * kRowBytes;          // one box of 128 query rows
+    static constexpr int kAtomKV = kN * kRowBytes;              // one box of kN key rows
+    static constexpr int kTileQ = kBlockM * D * 2;              // one Q tile
+    static constexpr int kTileKV = kN * D * 2;                  // one K or V tile
+    static constexpr int kStages = 8;                           // ring slots (each one K or one V tile)
     static constexpr int kOffQ = 0;                             // Q_A, Q_B
-    static constexpr int kOffRing = 2 * kTileBytes;
-    static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+    static constexpr int kOffRing = 2 * kTileQ;
+    static constexpr int kOffBar = kOffRing + kStages * kTileKV;
     static constexpr int kSmemBytes = kOffBar + 512;
+    // TMEM columns of tile X's S, P and O, relative to 256 X (O aligned to D)
+    static constexpr int kColS = 0;
+    static constexpr int kColP = kN;
+    static constexpr int kColO = 256 - D;
+    static_assert(kColP + kN / 2 <= kColO, "TMEM budget per query tile");
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+    // Registers per thread of the producer/MMA warpgroup and of the softmax
+    // warpgroups: a softmax thread holds a row of kN scores; 128 + 2*128
+    // threads share the launch's 384 * 168.
+    static constexpr int kRegsOther = kN == 64 ? 152 : 88;
+    static constexpr int kRegsSoftmax = kN == 64 ? 176 : 208;
+    static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 };
 
 struct AttnParams {
@@ -101,14 +120,15 @@ struct AttnParams {
     unsigned long long* sched;    // zeroed item counter (dynamic scheduling) or null (static striding)
 };
 
-// Key tile t of nt covering keys [0, kmax): tiles are 128 wide from key 0;
-// a ragged last tile is loaded right-aligned (start = kmax - 128, possibly
+// Key tile t of nt covering keys [0, kmax): tiles are kN wide from key 0;
+// a ragged last tile is loaded right-aligned (start = kmax - kN, possibly
 // negative: the TMA fills rows before 0 with zeros) so that it never reads
 // rows at or beyond kmax; keys below `lo` were already covered and are masked.
+template <int kN>
 __device__ __forceinline__ void key_tile(int t, int nt, int kmax, int& start, int& lo)
 {
-    lo = t * kBlockN;
-    start = (t == nt - 1 && (kmax % kBlockN) != 0) ? kmax - kBlockN : lo;
+    lo = t * kN;
+    start = (t == nt - 1 && (kmax % kN) != 0) ? kmax - kN : lo;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
@@ -202,7 +222,7 @@ struct Work {
     int nt_a, nt_b, nt;         // key tiles swept for A, B, and loaded
 };
 
-template <bool kDecode>
+template <bool kDecode, int kN>
 __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int local)
 {
     Work w;
@@ -233,12 +253,12 @@ __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int loca
     w.kmax_a = kDecode ? w.npast : min(w.qrow0 + w.nrows_a, w.npast);
     w.kmax_b = !w.has_b ? 0 : (kDecode ? w.npast : min(w.qrow0 + kBlockM + w.nrows_b, w.npast));
     // Tile A's range is a prefix of B's with identical tiles (kmax_a < kmax_b
-    // only when kmax_a is a multiple of 128).
+    // only when kmax_a is a multiple of 128, hence of kN).
     w.kmax = w.has_b ? w.kmax_b : w.kmax_a;
-    w.nt_all = (w.kmax + kBlockN - 1) / kBlockN;
+    w.nt_all = (w.kmax + kN - 1) / kN;
     w.t_begin = 0;
-    int t_end_a = (w.kmax_a + kBlockN - 1) / kBlockN;
-    int t_end_b = (w.kmax_b + kBlockN - 1) / kBlockN;
+    int t_end_a = (w.kmax_a + kN - 1) / kN;
+    int t_end_b = (w.kmax_b + kN - 1) / kN;
     if (kDecode && p.nsplit > 1) {
         const int per = (w.nt_all + p.nsplit - 1) / p.nsplit;
         w.t_begin = min(w.split * per, w.nt_all);
@@ -276,13 +296,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_q = bars + 0;           // Q tiles of the current item landed
     uint64_t* q_empty = bars + 1;         // every S MMA of an item finished with Q
-    uint64_t* s_full = bars + 2;          // [2]
-    uint64_t* p_full = bars + 4;          // [2]
-    uint64_t* o_full = bars + 6;          // [2]
+    uint64_t* s_full = bars + 2;          // [2] S_X computed
+    uint64_t* p_full = bars + 4;          // [2] P_X stored
+    uint64_t* pv_done = bars + 6;         // [2] O_X += P_X V finished (P_X free, O_X stable)
     uint64_t* bar_drain = bars + 8;       // [2] (bars + 8, bars + 9)
-    uint64_t* kv_full = bars + 10;        // [NS]
-    uint64_t* kv_empty = bars + 10 + NS;  // [NS]
-    uint64_t* item_full = bars + 10 + 2 * NS;      // [kItemSlots]
+    uint64_t* s_free = bars + 10;         // [2] S_X read into registers
+    uint64_t* kv_full = bars + 12;        // [NS]
+    uint64_t* kv_empty = bars + 12 + NS;  // [NS]
+    uint64_t* item_full = bars + 12 + 2 * NS;      // [kItemSlots]
     uint64_t* item_empty = item_full + kItemSlots;  // [kItemSlots]
     volatile long long* item_ring = reinterpret_cast<volatile long long*>(item_empty + kItemSlots);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 2 * kItemSlots);
@@ -293,8 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(q_empty, 2);            // one arrival from each MMA warp
         for (int x = 0; x < 2; ++x) {
             mbar_init(s_full + x, 1);
-            mbar_init(p_full + x, kBlockM);
-            mbar_init(o_full + x, 1);
+            mbar_init(s_free + x, 4);     // one arrival per softmax warp
+            mbar_init(p_full + x, 4);
+            mbar_init(pv_done + x, 1);
         }
         mbar_init(bar_drain + 0, 1);
         mbar_init(bar_drain + 1, 1);
@@ -341,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp-uniform, and only lane 0 issues copies, MMAs and commits.
     const bool leader = lane == 0;
     if (warp >= 8) {
-      setmaxnreg_dec<kRegsOther>();   // all four warps of the third warpgroup
+      setmaxnreg_dec<C::kRegsOther>();   // all four warps of the third warpgroup
       if (warp == 8) {
         // ------------------------------------------------------- producer
         if (leader) {
@@ -375,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ++n_items;
             if (!found) break;
-            const Work w = make_work<kDecode>(p, seg, local);
+            const Work w = make_work<kDecode, C::kN>(p, seg, local);
             if (!w.valid) {
                 if (leader) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
                 continue;
@@ -387,17 +409,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
             }
             if (leader) {
-                mbar_arrive_expect_tx(bar_q, (w.has_b ? 2 : 1) * C::kTileBytes);
+                mbar_arrive_expect_tx(bar_q, (w.has_b ? 2 : 1) * C::kTileQ);
                 for (int x = 0; x < (w.has_b ? 2 : 1); ++x)
                     for (int c = 0; c < C::kChunks; ++c)
-                        tma_load_3d(sQ + x * C::kTileBytes + c * C::kAtomBytes, &tm_q, bar_q, c * C::kBoxD, w.h,
+                        tma_load_3d(sQ + x * C::kTileQ + c * C::kAtomQ, &tm_q, bar_q, c * C::kBoxD, w.h,
                                     w.tok0 + w.qrow0 + x * kBlockM);
             }
             ++nq;
             const int pool_plane = (p.layer * p.S + w.slot) * p.H + w.h;
             for (int i = 0; ok && i < w.nt; ++i) {
                 int start, lo;
-                key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
+                key_tile<C::kN>(w.t_begin + i, w.nt_all, w.kmax, start, lo);
                 for (int kv = 0; kv < 2; ++kv) {          // K_i then V_i
                     const int st = u % NS;
                     if (u >= NS) {
@@ -405,15 +427,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!ok) break;
                     }
                     if (leader) {
-                        mbar_arrive_expect_tx(kv_full + st, C::kTileBytes);
+                        mbar_arrive_expect_tx(kv_full + st, C::kTileKV);
                         const CUtensorMap* map = kv == 0 ? &tm_k : &tm_v;
-                        uint8_t* dst = ring + st * C::kTileBytes;
+                        uint8_t* dst = ring + st * C::kTileKV;
                         for (int c = 0; c < C::kChunks; ++c) {
                             if (kDecode)
-                                tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, start,
+                                tma_load_3d(dst + c * C::kAtomKV, map, kv_full + st, c * C::kBoxD, start,
                                             pool_plane);
                             else
-                                tma_load_3d(dst + c * C::kAtomBytes, map, kv_full + st, c * C::kBoxD, w.h,
+                                tma_load_3d(dst + c * C::kAtomKV, map, kv_full + st, c * C::kBoxD, w.h,
                                             w.tok0 + start);
                         }
                     }
@@ -442,41 +464,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------- UMMA issuers
-        // Warp 9 issues the MMAs of tile A, warp 10 those of tile B, so each
-        // tile's next MMAs go out as soon as its own P is ready, never queued
-        // behind the other tile's issue.  Both release every K/V ring use and
-        // every Q load (arrival count 2); a use a warp does not need is still
-        // released, after its fill, so the two warps' arrivals stay in phase.
+        // Warp 9 issues the MMAs of tile A, warp 10 those of tile B.  Per key
+        // tile i of its query tile a warp issues
+        //   S_{i+1} = Q K_{i+1}^T  as soon as the softmax has read S_i out,
+        //   O += P_i V_i           as soon as the softmax has stored P_i,
+        // so S_{i+1} is being computed while the softmax works on S_i.  Both
+        // warps release every K/V ring use and every Q load (arrival count 2);
+        // a use a warp does not need is still released, after its fill, so
+        // the two warps' arrivals stay in phase.
         const int x = warp - 9;
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, false);
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(kBlockM, C::kN, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(kBlockM, D, true);
         // Descriptors are built once; a K-step moves only the start-address
         // field (low 14 bits, in 16-byte units), by compile-time offsets.
-        const uint64_t dq0 = smem_desc(smem_u32(sQ) + x * C::kTileBytes, 16, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dq0 = smem_desc(smem_u32(sQ) + x * C::kTileQ, 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dk0 = smem_desc(smem_u32(ring), 16, 8 * C::kRowBytes, C::kLayout);
-        const uint64_t dv0 = smem_desc(smem_u32(ring), C::kAtomBytes, 8 * C::kRowBytes, C::kLayout);
-        const uint32_t tS = tmem + x * 128;
-        const uint32_t tO = tmem + 256 + x * D;
-        // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16 elements.
+        const uint64_t dv0 = smem_desc(smem_u32(ring), C::kAtomKV, 8 * C::kRowBytes, C::kLayout);
+        const uint32_t tS = tmem + x * 256 + C::kColS;
+        const uint32_t tP = tmem + x * 256 + C::kColP;
+        const uint32_t tO = tmem + x * 256 + C::kColO;
+        // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16
+        // elements (32 bytes within a swizzle row, then the next box of D).
         auto issue_qk = [&](int st) {
-            const uint64_t b0 = dk0 + (uint64_t)((st * C::kTileBytes) >> 4);
+            const uint64_t b0 = dk0 + (uint64_t)((st * C::kTileKV) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 constexpr int kStep = 32;
-                const uint32_t off = ((kk * kStep / C::kRowBytes) * C::kAtomBytes + (kk * kStep) % C::kRowBytes) >> 4;
-                umma_bf16_ss(tS, dq0 + off, b0 + off, idesc_qk, kk > 0 ? 1u : 0u);
+                const uint32_t in_row = (kk * kStep) % C::kRowBytes;
+                const uint32_t box = kk * kStep / C::kRowBytes;
+                umma_bf16_ss(tS, dq0 + ((box * C::kAtomQ + in_row) >> 4), b0 + ((box * C::kAtomKV + in_row) >> 4),
+                             idesc_qk, kk > 0 ? 1u : 0u);
             }
             umma_commit(s_full + x);
         };
-        // O_x += P_x V: P from TMEM (first 64 columns of S_x, 8 columns per
-        // 16 keys), V read MN-major (D contiguous); K-steps of 16 keys.
+        // O_x += P_x V: P from TMEM (8 columns of bf16 pairs per 16 keys), V
+        // read MN-major (D contiguous); K-steps of 16 keys.
         auto issue_pv = [&](int st, bool acc) {
-            const uint64_t b0 = dv0 + (uint64_t)((st * C::kTileBytes) >> 4);
+            const uint64_t b0 = dv0 + (uint64_t)((st * C::kTileKV) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < kBlockN / 16; ++kk) {
+            for (int kk = 0; kk < C::kN / 16; ++kk) {
                 const uint32_t off = (kk * 16 * C::kRowBytes) >> 4;
-                umma_bf16_ts(tO, tS + kk * 8, b0 + off, idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                umma_bf16_ts(tO, tP + kk * 8, b0 + off, idesc_pv, (acc || kk > 0) ? 1u : 0u);
             }
+            umma_commit(pv_done + x);
         };
         auto wait_fill = [&](int u) {
             return __all_sync(0xffffffffu, mbar_wait(kv_full + u % NS, (u / NS) & 1, ctl));
@@ -484,57 +514,65 @@ __global__ void __launch_bounds__(kThreads, 1)
         int u = 0;                 // ring uses consumed
         int nq = 0;                // items with MMAs
         int np = 0;                // p_full completions consumed
+        int nsq = 0;               // S tiles issued (each is read out once: one s_free completion)
         bool ok = true;
+        // S_x may be overwritten once the softmax has read out the previous S_x.
+        auto wait_s_free = [&]() {
+            if (nsq == 0) return true;
+            const bool r = __all_sync(0xffffffffu, mbar_wait(s_free + x, (nsq - 1) & 1, ctl));
+            tc_fence_after_sync();
+            return r;
+        };
         while (pop_item(ok)) {
-            const Work w = make_work<kDecode>(p, seg, local);
+            const Work w = make_work<kDecode, C::kN>(p, seg, local);
             if (w.nt == 0) continue;
             const int ntx = x == 0 ? w.nt_a : w.nt_b;
             // Q landed: this also means both warps released the previous Q.
             ok = __all_sync(0xffffffffu, mbar_wait(bar_q, nq & 1, ctl)) && wait_fill(u);
             if (!ok) break;
             tc_fence_after_sync();
-            if (leader) {
-                if (ntx > 0) {
+            if (ntx > 0) {
+                if (!(ok = wait_s_free())) break;
+                if (leader) {
                     issue_qk(u % NS);
                     umma_commit(kv_empty + u % NS);                 // K_0
                     if (ntx == 1) umma_commit(q_empty);            // no S MMA of this tile after this
-                } else {
-                    mbar_arrive(kv_empty + u % NS);
-                    mbar_arrive(q_empty);
                 }
+                ++nsq;
+            } else if (leader) {
+                mbar_arrive(kv_empty + u % NS);
+                mbar_arrive(q_empty);
             }
             for (int i = 0; ok && i < w.nt; ++i) {
                 const int uv = u + 1;          // V_i
                 const int uk = u + 2;          // K_{i+1}
+                if (i + 1 < ntx) {
+                    if (!(ok = wait_fill(uk))) break;
+                    if (!(ok = wait_s_free())) break;
+                    if (leader) {
+                        issue_qk(uk % NS);
+                        umma_commit(kv_empty + uk % NS);
+                        if (i + 2 == ntx) umma_commit(q_empty);   // that was this tile's last S MMA
+                    }
+                    ++nsq;
+                }
                 if (!(ok = wait_fill(uv))) break;
                 if (i < ntx) {
                     ok = __all_sync(0xffffffffu, mbar_wait(p_full + x, np & 1, ctl));
                     if (!ok) break;
                     ++np;
                     tc_fence_after_sync();
-                    if (leader) issue_pv(uv % NS, i > 0);
-                    if (i + 1 < ntx) {
-                        if (!(ok = wait_fill(uk))) break;
-                        tc_fence_after_sync();
-                        if (leader) {
-                            issue_qk(uk % NS);
-                            if (i + 2 == ntx) umma_commit(q_empty);   // that was this tile's last S MMA
-                        }
-                    } else if (leader) {
-                        umma_commit(o_full + x);
+                    if (leader) {
+                        issue_pv(uv % NS, i > 0);
+                        umma_commit(kv_empty + uv % NS);
                     }
-                    if (leader) umma_commit(kv_empty + uv % NS);
                 } else if (leader) {
                     mbar_arrive(kv_empty + uv % NS);
                 }
-                if (i + 1 < w.nt) {
-                    if (i + 1 >= ntx) {
-                        // K_{i+1} is only for the other tile: release it once it has landed
-                        if (!(ok = wait_fill(uk))) break;
-                        if (leader) mbar_arrive(kv_empty + uk % NS);
-                    } else if (leader) {
-                        umma_commit(kv_empty + uk % NS);
-                    }
+                if (i + 1 < w.nt && i + 1 >= ntx) {
+                    // K_{i+1} is only for the other tile: release it once it has landed
+                    if (!(ok = wait_fill(uk))) break;
+                    if (leader) mbar_arrive(kv_empty + uk % NS);
                 }
                 u += 2;
             }
@@ -547,20 +585,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     } else {
-        setmaxnreg_inc<kRegsSoftmax>();
+        setmaxnreg_inc<C::kRegsSoftmax>();
         // ------------------------------------------------ softmax + epilogue
         const int x = warp / 4;                            // 0: tile A, 1: tile B
         const int r = threadIdx.x - x * kBlockM;           // query row in the tile
         const uint32_t lane_off = static_cast<uint32_t>((warp % 4) * 32) << 16;
-        const uint32_t tS = tmem + x * 128 + lane_off;
-        const uint32_t tO = tmem + 256 + x * D + lane_off;
+        const uint32_t tS = tmem + x * 256 + C::kColS + lane_off;
+        const uint32_t tP = tmem + x * 256 + C::kColP + lane_off;
+        const uint32_t tO = tmem + x * 256 + C::kColO + lane_off;
         const float sl2 = p.sl2;
         const bool split_mode = kDecode && p.nsplit > 1;
+        constexpr int kN = C::kN;
         int ns = 0;          // s_full completions consumed
-        int no = 0;          // o_full completions consumed
+        int npv = 0;         // pv_done completions consumed
+        auto wait_pv = [&]() {
+            const bool r = __all_sync(0xffffffffu, mbar_wait(pv_done + x, npv & 1, ctl));
+            ++npv;
+            tc_fence_after_sync();
+            return r;
+        };
         bool ok = true;
         while (pop_item(ok)) {
-            const Work w = make_work<kDecode>(p, seg, local);
+            const Work w = make_work<kDecode, C::kN>(p, seg, local);
             if (!w.valid) continue;
             const int ntx = x == 0 ? w.nt_a : w.nt_b;
             const int nrows_x = x == 0 ? w.nrows_a : w.nrows_b;
@@ -598,25 +644,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             float l = 0.f;           // row sum relative to m
             for (int i = 0; i < ntx; ++i) {
                 int start, lo;
-                key_tile(w.t_begin + i, w.nt_all, w.kmax, start, lo);
-                const bool full_tile = (start == lo) && (start + kBlockN <= kmax_x) && (start + kBlockN - 1 <= posx0);
+                key_tile<C::kN>(w.t_begin + i, w.nt_all, w.kmax, start, lo);
+                const bool full_tile = (start == lo) && (start + kN <= kmax_x) && (start + kN - 1 <= posx0);
                 // warp-uniform: the TMEM accesses below are warp-collective
                 ok = __all_sync(0xffffffffu, mbar_wait(s_full + x, ns & 1, ctl));
                 if (!ok) break;
                 ++ns;
                 tc_fence_after_sync();
-                uint32_t s[kBlockN];
-                tmem_ld128(tS, s);
+                uint32_t s[kN];
+                if constexpr (kN == 128)
+                    tmem_ld128(tS, s);
+                else
+                    tmem_ld64(tS, s);
+                // S is in registers: the next S may be written over it.
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(s_free + x);
+                // P_x and O_x belong to the previous tile's P.V until it finishes
+                // (at tile 0 the previous item's last P.V was waited for before its epilogue).
+                bool pv_waited = i == 0;
                 if (!full_tile) {
 #pragma unroll
-                    for (int e = 0; e < kBlockN; ++e) {
+                    for (int e = 0; e < kN; ++e) {
                         const int j = start + e;
                         if (!(j >= lo && j < kmax_x && j <= irow)) s[e] = 0xff800000u;   // -inf
                     }
                 }
                 float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < kBlockN; e += 8) {
+                for (int e = 0; e < kN; e += 8) {
                     mx0 = max3f(mx0, __uint_as_float(s[e]), __uint_as_float(s[e + 1]));
                     mx1 = max3f(mx1, __uint_as_float(s[e + 2]), __uint_as_float(s[e + 3]));
                     mx2 = max3f(mx2, __uint_as_float(s[e + 4]), __uint_as_float(s[e + 5]));
@@ -630,7 +686,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float m_new = fmaxf(m, m_tile);
                     const float corr = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
                     if (i > 0) {
-                        // O_x is stable: the P.V of the previous tile completed before S of this one.
+                        if (!(ok = wait_pv())) break;
+                        pv_waited = true;
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
                             uint32_t o[32];
@@ -646,13 +703,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_use = (m == -INFINITY) ? 0.f : m;
                 // P = 2^(s * scale * log2e - m): packed fp32 pairs; one pair in four
                 // takes the polynomial exp2 on the FMA pipe, the rest the MUFU ex2,
-                // so the two pipes share the load.  P goes over the first 64
-                // columns of S, written in two halves of 64 keys.
+                // so the two pipes share the load.  P is written in pieces of 64 keys
+                // (32 columns of bf16 pairs).
                 const uint64_t sc2 = f2_pack(sl2, sl2);
                 const uint64_t nm2 = f2_pack(-m_use, -m_use);
                 uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                for (int half = 0; half < kN / 64; ++half) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int c = 0; c < 32; ++c) {
@@ -670,11 +727,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         acc[c & 3] = f2_add(acc[c & 3], f2_pack(p0, p1));
                         pk[c] = pack_bf16x2(p0, p1);
                     }
-                    if (half == 0)
-                        tmem_st32_nowait(tS, pk);    // its latency overlaps the second half
+                    if (half == 0 && !pv_waited) {
+                        if (!(ok = wait_pv())) break;
+                    }
+                    if (half + 1 < kN / 64)
+                        tmem_st32_nowait(tP + half * 32, pk);   // its latency overlaps the next piece
                     else
-                        tmem_st32(tS + 32, pk);      // waits for both halves
+                        tmem_st32(tP + half * 32, pk);          // waits for every piece
                 }
+                if (!ok) break;
                 {
                     const uint64_t a01 = f2_add(acc[0], acc[1]);
                     const uint64_t a23 = f2_add(acc[2], acc[3]);
@@ -683,7 +744,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     l += lo + hi;
                 }
                 tc_fence_before_sync();
-                mbar_arrive(p_full + x);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full + x);
             }
             if (!ok) break;
             // ---- epilogue: the own value (self term) is fetched before waiting for O
@@ -693,12 +755,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) vr[c] = self ? __ldg(v4 + c) : make_uint4(0u, 0u, 0u, 0u);
             }
-            if (ntx > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(o_full + x, no & 1, ctl));
-                if (!ok) break;
-                ++no;
-                tc_fence_after_sync();
-            }
+            if (ntx > 0 && !(ok = wait_pv())) break;   // the last P.V: O_x is final
             float a = 1.f, b = 0.f, inv = 0.f;
             if (row_valid && !split_mode) {
                 const float m_fin = fmaxf(m, ss);

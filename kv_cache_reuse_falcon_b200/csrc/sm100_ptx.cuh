@@ -312,6 +312,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+// Waits until every tcgen05.st of this thread has completed.
+__device__ __forceinline__ void tmem_wait_st()
+{
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // As tmem_st32 without the wait: a later tcgen05.wait::st (e.g. in the next
 // tmem_st32) covers it.
 __device__ __forceinline__ void tmem_st32_nowait(uint32_t taddr, const uint32_t (&r)[32])

@@ -118,22 +118,23 @@ int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
     return r == CUDA_SUCCESS ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 
-// Packed token tensor [T, H, D]: boxes of 128 tokens x 1 head x (D or 64) elements.
-int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D)
+// Packed token tensor [T, H, D]: boxes of `rows` tokens x 1 head x (D or 64)
+// elements (128 query rows, or one key tile).
+int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D, int rows)
 {
     const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
     return make_map(m, base, (uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)D * 2, (uint64_t)H * D * 2, box_d, 1,
-                    kBlockN, D);
+                    (uint32_t)rows, D);
 }
 
-// Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of 128 history rows.
+// Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of one key tile of history rows.
 int make_pool_map(CUtensorMap* m, const void* base, const unipin_kvpool* pool)
 {
     const int D = pool->D;
     const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
     const uint64_t planes = (uint64_t)pool->L * pool->S * pool->H;
     return make_map(m, base, (uint64_t)D, (uint64_t)pool->n_cap, planes, (uint64_t)D * 2,
-                    (uint64_t)pool->n_cap * D * 2, box_d, kBlockN, 1, D);
+                    (uint64_t)pool->n_cap * D * 2, box_d, (uint32_t)key_tile_width(D), 1, D);
 }
 
 int check_pool(const unipin_kvpool* pool, int H, int D, int layer)
@@ -202,7 +203,7 @@ int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
     const long long slots = (long long)kNumSmsHint;   // one block per SM (all of TMEM)
     const long long target = 4 * slots;
     if (units >= 2 * slots) return 1;   // two or more waves already: no split
-    const int key_tiles = (n_cap + kBlockN - 1) / kBlockN;
+    const int key_tiles = (n_cap + key_tile_width(D) - 1) / key_tile_width(D);
     long long ns = (target + units - 1) / units;
     const long long cap = key_tiles / 2 > 1 ? key_tiles / 2 : 1;   // at least two key tiles per split
     if (ns > cap) ns = cap;
@@ -310,9 +311,9 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
         if (rc != UNIPIN_OK) return rc;
     }
     CUtensorMap tq, tk, tv;
-    if ((rc = make_token_map(&tq, q, total_tokens, H, D)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tk, k, total_tokens, H, D)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tv, v, total_tokens, H, D)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tq, q, total_tokens, H, D, kBlockM)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tk, k, total_tokens, H, D, key_tile_width(D))) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tv, v, total_tokens, H, D, key_tile_width(D))) != UNIPIN_OK) return rc;
 
     AttnParams p = {};
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -390,7 +391,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     }
 
     CUtensorMap tq, tk, tv;
-    if ((rc = make_token_map(&tq, q_c, total_cand, H, D)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tq, q_c, total_cand, H, D, kBlockM)) != UNIPIN_OK) return rc;
     if ((rc = make_pool_map(&tk, pool->k, pool)) != UNIPIN_OK) return rc;
     if ((rc = make_pool_map(&tv, pool->v, pool)) != UNIPIN_OK) return rc;
 
