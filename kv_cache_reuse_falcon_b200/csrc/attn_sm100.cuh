@@ -78,10 +78,11 @@ struct AttnCfg {
     static constexpr int kAtomKV = kN * kRowBytes;              // one box of kN key rows
     static constexpr int kTileQ = kBlockM * D * 2;              // one Q tile
     static constexpr int kTileKV = kN * D * 2;                  // one K or V tile
-    static constexpr int kStages = 8;                           // ring slots (each one K or one V tile)
+    static constexpr int kSlotBytes = 2 * kTileKV;              // a ring slot: K and V of one key tile
+    static constexpr int kStages = (128 * 1024) / kSlotBytes;   // ring slots
     static constexpr int kOffQ = 0;                             // Q_A, Q_B
     static constexpr int kOffRing = 2 * kTileQ;
-    static constexpr int kOffBar = kOffRing + kStages * kTileKV;
+    static constexpr int kOffBar = kOffRing + kStages * kSlotBytes;
     static constexpr int kSmemBytes = kOffBar + 512;
     // TMEM columns of tile X's S, P and O, relative to 256 X (O aligned to D)
     static constexpr int kColS = 0;
@@ -417,19 +418,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             ++nq;
             const int pool_plane = (p.layer * p.S + w.slot) * p.H + w.h;
-            for (int i = 0; ok && i < w.nt; ++i) {
+            for (int i = 0; ok && i < w.nt; ++i) {      // K_i and V_i into one slot
                 int start, lo;
                 key_tile<C::kN>(w.t_begin + i, w.nt_all, w.kmax, start, lo);
-                for (int kv = 0; kv < 2; ++kv) {          // K_i then V_i
-                    const int st = u % NS;
-                    if (u >= NS) {
-                        ok = __all_sync(0xffffffffu, mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl));
-                        if (!ok) break;
-                    }
-                    if (leader) {
-                        mbar_arrive_expect_tx(kv_full + st, C::kTileKV);
+                const int st = u % NS;
+                if (u >= NS) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl));
+                    if (!ok) break;
+                }
+                if (leader) {
+                    mbar_arrive_expect_tx(kv_full + st, C::kSlotBytes);
+                    for (int kv = 0; kv < 2; ++kv) {
                         const CUtensorMap* map = kv == 0 ? &tm_k : &tm_v;
-                        uint8_t* dst = ring + st * C::kTileKV;
+                        uint8_t* dst = ring + st * C::kSlotBytes + kv * C::kTileKV;
                         for (int c = 0; c < C::kChunks; ++c) {
                             if (kDecode)
                                 tma_load_3d(dst + c * C::kAtomKV, map, kv_full + st, c * C::kBoxD, start,
@@ -439,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             w.tok0 + start);
                         }
                     }
-                    ++u;
                 }
+                ++u;
             }
         }
         if (!ok && leader) {
@@ -479,14 +480,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // field (low 14 bits, in 16-byte units), by compile-time offsets.
         const uint64_t dq0 = smem_desc(smem_u32(sQ) + x * C::kTileQ, 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dk0 = smem_desc(smem_u32(ring), 16, 8 * C::kRowBytes, C::kLayout);
-        const uint64_t dv0 = smem_desc(smem_u32(ring), C::kAtomKV, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dv0 = smem_desc(smem_u32(ring) + C::kTileKV, C::kAtomKV, 8 * C::kRowBytes, C::kLayout);
         const uint32_t tS = tmem + x * 256 + C::kColS;
         const uint32_t tP = tmem + x * 256 + C::kColP;
         const uint32_t tO = tmem + x * 256 + C::kColO;
         // S_x = Q_x K^T: both operands K-major in shared memory; K-steps of 16
         // elements (32 bytes within a swizzle row, then the next box of D).
         auto issue_qk = [&](int st) {
-            const uint64_t b0 = dk0 + (uint64_t)((st * C::kTileKV) >> 4);
+            const uint64_t b0 = dk0 + (uint64_t)((st * C::kSlotBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 constexpr int kStep = 32;
@@ -500,7 +501,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O_x += P_x V: P from TMEM (8 columns of bf16 pairs per 16 keys), V
         // read MN-major (D contiguous); K-steps of 16 keys.
         auto issue_pv = [&](int st, bool acc) {
-            const uint64_t b0 = dv0 + (uint64_t)((st * C::kTileKV) >> 4);
+            const uint64_t b0 = dv0 + (uint64_t)((st * C::kSlotBytes) >> 4);
 #pragma unroll
             for (int kk = 0; kk < C::kN / 16; ++kk) {
                 const uint32_t off = (kk * 16 * C::kRowBytes) >> 4;
@@ -535,46 +536,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = wait_s_free())) break;
                 if (leader) {
                     issue_qk(u % NS);
-                    umma_commit(kv_empty + u % NS);                 // K_0
                     if (ntx == 1) umma_commit(q_empty);            // no S MMA of this tile after this
                 }
                 ++nsq;
             } else if (leader) {
-                mbar_arrive(kv_empty + u % NS);
                 mbar_arrive(q_empty);
             }
             for (int i = 0; ok && i < w.nt; ++i) {
-                const int uv = u + 1;          // V_i
-                const int uk = u + 2;          // K_{i+1}
-                if (i + 1 < ntx) {
-                    if (!(ok = wait_fill(uk))) break;
-                    if (!(ok = wait_s_free())) break;
-                    if (leader) {
-                        issue_qk(uk % NS);
-                        umma_commit(kv_empty + uk % NS);
-                        if (i + 2 == ntx) umma_commit(q_empty);   // that was this tile's last S MMA
-                    }
-                    ++nsq;
-                }
-                if (!(ok = wait_fill(uv))) break;
+                // Slot u holds K_i and V_i; slot u + 1 holds K_{i+1}.
                 if (i < ntx) {
+                    if (i + 1 < ntx) {
+                        // s_free also says that slot u + 1 has landed: the softmax
+                        // checks it before it signals, off this warp's critical path
+                        // (a wait issued behind MMAs costs this warp until they drain).
+                        if (!(ok = wait_s_free())) break;
+                        if (leader) {
+                            issue_qk((u + 1) % NS);
+                            if (i + 2 == ntx) umma_commit(q_empty);   // that was this tile's last S MMA
+                        }
+                        ++nsq;
+                    }
                     ok = __all_sync(0xffffffffu, mbar_wait(p_full + x, np & 1, ctl));
                     if (!ok) break;
                     ++np;
                     tc_fence_after_sync();
                     if (leader) {
-                        issue_pv(uv % NS, i > 0);
-                        umma_commit(kv_empty + uv % NS);
+                        issue_pv(u % NS, i > 0);
+                        umma_commit(kv_empty + u % NS);
                     }
-                } else if (leader) {
-                    mbar_arrive(kv_empty + uv % NS);
+                } else {
+                    // K_i/V_i are only for the other tile: release the slot once it has landed
+                    if (!(ok = wait_fill(u))) break;
+                    if (leader) mbar_arrive(kv_empty + u % NS);
                 }
-                if (i + 1 < w.nt && i + 1 >= ntx) {
-                    // K_{i+1} is only for the other tile: release it once it has landed
-                    if (!(ok = wait_fill(uk))) break;
-                    if (leader) mbar_arrive(kv_empty + uk % NS);
-                }
-                u += 2;
+                ++u;
             }
             ++nq;
         }
@@ -598,6 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int kN = C::kN;
         int ns = 0;          // s_full completions consumed
         int npv = 0;         // pv_done completions consumed
+        int u_sm = 0;        // ring slot uses (key tiles loaded) before the current item
         auto wait_pv = [&]() {
             const bool r = __all_sync(0xffffffffu, mbar_wait(pv_done + x, npv & 1, ctl));
             ++npv;
@@ -607,6 +603,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         while (pop_item(ok)) {
             const Work w = make_work<kDecode, C::kN>(p, seg, local);
+            const int u_item = u_sm;
+            u_sm += w.nt;
             if (!w.valid) continue;
             const int ntx = x == 0 ? w.nt_a : w.nt_b;
             const int nrows_x = x == 0 ? w.nrows_a : w.nrows_b;
@@ -656,7 +654,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld128(tS, s);
                 else
                     tmem_ld64(tS, s);
-                // S is in registers: the next S may be written over it.
+                // S is in registers: the next S may be written over it.  The next S
+                // also needs K_{i+1}; the first warp of the group signals only once
+                // its ring slot has landed, so the MMA warp waits on s_free alone.
+                if (i + 1 < ntx && (warp % 4) == 0) {
+                    const int un = u_item + i + 1;
+                    ok = __all_sync(0xffffffffu, mbar_wait(kv_full + un % NS, (un / NS) & 1, ctl));
+                    if (!ok) break;
+                }
                 tc_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(s_free + x);
