@@ -65,6 +65,26 @@ def pool_write_bytes(past, H, D):
     return float(2 * 2 * np.asarray(past, dtype=np.float64).sum() * H * D * 2)   # K and V, read + write
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the prefill
+# attention kernel per query-side token, from one ncu capture of a 24-user cut
+# of the ragged batch (H=8, D=128; summary and command under profiles/), keyed
+# by the kernel source it was taken on.  A changed kernel reports null until
+# it is captured again.
+_PREFILL_TRAFFIC_PER_TOKEN = {
+    # sha256 prefix of csrc/attn_sm100.cuh, H, D: bytes per token
+    ("0f149fb896637dd4", 8, 128): (432.068096e6 + 123.416064e6) / 70236,
+}
+
+
+def prefill_traffic(T, H, D):
+    import hashlib
+    src = os.path.join(ROOT, "kv_cache_reuse_falcon_b200", "csrc", "attn_sm100.cuh")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    per = _PREFILL_TRAFFIC_PER_TOKEN.get((sha, H, D))
+    return None if per is None else per * T
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -367,7 +387,9 @@ def run_ours(args, rank, world, device, dist):
                    "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
                    "pool_write_frac_hbm": pool_gbs / peaks["hbm_gbs"]},
         "roofline": {"kernel": "attn_fwd_kernel<128,prefill>", "bound": "tensor", "achieved": pre_tflops,
-                     "peak": peak, "unit": "TFLOP/s", "frac": pre_tflops / peak, "traffic": None,
+                     "peak": peak, "unit": "TFLOP/s", "frac": pre_tflops / peak,
+                     "traffic": prefill_traffic(T, H, D),
+                     "traffic_note": "ncu DRAM bytes per token of a 24-user capture, scaled by tokens",
                      "peak_source": "%s bf16_tflops (burst)" % peaks["source"],
                      "work_per_launch": "4*D*H*sum_b[n_b(n_b+1)/2 + k_b(n_b+1)] = %.4g FLOP" % pf},
         "e2e": {"value": cand_total / (e2e_ms * 1e-3), "unit": "candidate tokens/s",
