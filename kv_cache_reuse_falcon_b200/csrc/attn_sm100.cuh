@@ -93,8 +93,8 @@ struct AttnCfg {
     // Registers per thread of the producer/MMA warpgroup and of the softmax
     // warpgroups: a softmax thread holds a row of kN scores; 128 + 2*128
     // threads share the launch's 384 * 168.
-    static constexpr int kRegsOther = kN == 64 ? 152 : 88;
-    static constexpr int kRegsSoftmax = kN == 64 ? 176 : 208;
+    static constexpr int kRegsOther = kN == 64 ? 152 : 136;
+    static constexpr int kRegsSoftmax = kN == 64 ? 176 : 184;
     static_assert(128 * kRegsOther + 256 * kRegsSoftmax <= kThreads * kLaunchRegs, "register split");
 };
 
@@ -693,13 +693,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (i > 0) {
                         if (!(ok = wait_pv())) break;
                         pv_waited = true;
+                        // in 8-column pieces: the scores of the tile stay live meanwhile
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t o[32];
-                            tmem_ld32(tO + c * 32, o);
+                        for (int c = 0; c < D / 8; ++c) {
+                            uint32_t o[8];
+                            tmem_ld8(tO + c * 8, o);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
-                            tmem_st32(tO + c * 32, o);
+                            for (int e = 0; e < 8; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * corr);
+                            tmem_st8(tO + c * 8, o);
                         }
                     }
                     l *= corr;
