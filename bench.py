@@ -72,7 +72,7 @@ def pool_write_bytes(past, H, D):
 # it is captured again.
 _PREFILL_TRAFFIC_PER_TOKEN = {
     # sha256 prefix of csrc/attn_sm100.cuh, H, D: bytes per token
-    ("0f149fb896637dd4", 8, 128): (432.068096e6 + 123.416064e6) / 70236,
+    ("f13854000651ad27", 8, 128): (431.669760e6 + 123.166208e6) / 70236,
 }
 
 
@@ -135,20 +135,40 @@ class ClockSampler:
         self.proc = None
         self.path = None
 
+    def _lines(self):
+        try:
+            with open(self.path) as f:
+                return [ln for ln in f.read().splitlines() if ln.count(",") >= 8]
+        except OSError:
+            return []
+
     def start(self):
+        """Start sampling every 50 ms; returns once the first sample is in (at most 5 s), so the
+        timed region that follows is covered from its start."""
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            self.fh = open(self.path, "w")
+            self.fh = open(self.path, "w", buffering=1)
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 5.0 and not self._lines():
+            time.sleep(0.01)
+        self.first = len(self._lines())   # samples before the timed region are not used
 
     def stop(self):
+        """Waits for one sample after the timed region (at most 1 s), then stops sampling and
+        summarises the samples taken from the start of the timed region on."""
         if self.proc is None:
             return None
+        n_end = len(self._lines())
+        t0 = time.time()
+        while time.time() - t0 < 1.0 and len(self._lines()) <= n_end:
+            time.sleep(0.01)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -157,19 +177,16 @@ class ClockSampler:
         self.fh.close()
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx.append(float(parts[2]))
-                except ValueError:
-                    continue
-                for nm, val in zip(names, parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(nm)
+        for line in self._lines()[self.first:]:
+            parts = [x.strip() for x in line.split(",")]
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
         os.unlink(self.path)
         if not sm:
             return None
