@@ -459,18 +459,36 @@ def run_decode_only(args, rank, world, device, dist):
     status = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
 
-    def step(ev=None):
+    def layers(s):
         for layer in range(L):
-            if ev is not None and layer == 0:
-                ev[0].record(stream)
             ub.rank_decode_attn(qs[layer], kc[layer], vc[layer], cu, sl, pl, pool_k, pool_v, layer, kk,
-                                out=out[layer], out_fp32=False, workspace=ws, dev_status=status, stream=stream)
+                                out=out[layer], out_fp32=False, workspace=ws, dev_status=status, stream=s)
+
+    graph = None
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        if graph is not None:
+            graph.replay()
+        else:
+            layers(stream)
         if ev is not None:
             ev[1].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(device)
+    if args.graph:
+        # the L layer calls of a step as one CUDA graph (every call is asynchronous, allocates
+        # nothing and syncs nothing, and the first calls above did the one-time set-up)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            layers(torch.cuda.current_stream(device))
+        torch.cuda.synchronize(device)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(device)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if clocks:
@@ -505,6 +523,7 @@ def run_decode_only(args, rank, world, device, dist):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": args.workload, "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
                    "pool": [L, S, H, n_cap, D], "layers_per_step": L, "split_n": ws_bytes > 256,
+                   "cuda_graph": bool(args.graph),
                    "l2": "pool slots read per step exceed L2 (no flush)"},
         "phases": {"decode_tflops": tflops, "decode_gbs": gbs, "decode_frac_hbm": gbs / peaks["hbm_gbs"],
                    "decode_frac_tensor": tflops / peaks["bf16_tflops"],
@@ -563,6 +582,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--users", type=int, default=0, help="smaller case: this many users (profiling)")
     ap.add_argument("--k", type=int, default=0, help="decode workloads: candidates per request")
+    ap.add_argument("--graph", action="store_true",
+                    help="decode workloads: replay each step's layer calls as one CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
