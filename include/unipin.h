@@ -176,6 +176,68 @@ int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void
 /* Size of the array behind unipin_rank_decode_attn_noalloc (32 MiB). */
 size_t unipin_rank_decode_noalloc_scratch_bytes(void);
 
+/*
+ * Cross-process sharing of a pool ([notes] §6 "serving: cross-process KV
+ * sharing": retrieval and ranking are separate OS processes with separate
+ * CUDA contexts; each retrieval replica preallocates its [L, S, H, n, D] pool
+ * and exports CUDA IPC handles for it, and the ranking process maps the same
+ * device memory and reads the KV without a trip through the host).
+ *
+ * unipin_kvpool_share is plain bytes and may be written to a file or a
+ * socket as it is: the IPC handles of the device allocations that hold
+ * pool.k and pool.v, the byte offsets of the pool inside them, and the shape.
+ */
+typedef struct {
+    unsigned char k_handle[64];       /* cudaIpcMemHandle_t of the allocation holding pool.k */
+    unsigned char v_handle[64];       /* same for pool.v */
+    unsigned long long k_offset;      /* byte offset of pool.k inside its allocation */
+    unsigned long long v_offset;
+    int L, S, H, n_cap, D;
+} unipin_kvpool_share;
+
+/* Exporter side: fill *out for `pool`.  The pool's tensors must lie in memory
+ * from cudaMalloc (not from virtual-memory mapping or cudaMallocAsync pools),
+ * and must stay allocated while any importer has it open.
+ * Returns UNIPIN_ERR_INVALID_ARG for a null or malformed pool or a pointer
+ * that is not device memory, UNIPIN_ERR_OUT_OF_RANGE if the pool extends past
+ * its allocation, UNIPIN_ERR_CUDA if the handle cannot be created. */
+int unipin_kvpool_share_export(const unipin_kvpool* pool, unipin_kvpool_share* out);
+
+/* Importer side (another process, on a device that can reach the exporter's):
+ * map the shared pool into this process; *out is then a pool usable by every
+ * call of this library.  A process cannot open a handle it exported itself
+ * (UNIPIN_ERR_CUDA). */
+int unipin_kvpool_share_open(const unipin_kvpool_share* in, unipin_kvpool* out);
+
+/* Importer side: unmap a pool opened from `in`; clears opened->k and ->v. */
+int unipin_kvpool_share_close(const unipin_kvpool_share* in, unipin_kvpool* opened);
+
+/*
+ * Slot assignment for the pool ([notes] §6: slots are reused in rotation;
+ * [review] §2.4: the retrieval stage hands the ranking node the slot id of
+ * each request).  Host-side and thread-safe.  acquire hands out n distinct
+ * free slots, scanning in round-robin order from the slot after the last one
+ * it handed out, so consecutive requests rotate through the pool; release
+ * returns slots once the ranking side is done with them.
+ */
+typedef struct unipin_slot_ring unipin_slot_ring;
+
+/* A ring over slots 0..S-1, all free.  UNIPIN_ERR_INVALID_ARG if S < 1. */
+int unipin_slot_ring_create(int S, unipin_slot_ring** out);
+
+/* Writes n free slot ids into the host array slot_ids and marks them in use.
+ * If fewer than n are free, takes none and returns UNIPIN_ERR_OUT_OF_RANGE. */
+int unipin_slot_ring_acquire(unipin_slot_ring* ring, int n, int* slot_ids);
+
+/* Marks the n slots free again.  All or nothing: an id out of range, not in
+ * use, or repeated in the list gives UNIPIN_ERR_INVALID_ARG and frees none. */
+int unipin_slot_ring_release(unipin_slot_ring* ring, int n, const int* slot_ids);
+
+/* Number of free slots (or UNIPIN_ERR_INVALID_ARG for a null ring). */
+int unipin_slot_ring_free_count(unipin_slot_ring* ring);
+
+void unipin_slot_ring_destroy(unipin_slot_ring* ring);
+
 /* Human-readable name of a unipin_status value. */
 const char* unipin_status_string(int status);
 

@@ -39,6 +39,14 @@ EXPORTS = (
     "unipin_selftest_exp2",
     "unipin_rank_decode_attn_noalloc",
     "unipin_rank_decode_noalloc_scratch_bytes",
+    "unipin_kvpool_share_export",
+    "unipin_kvpool_share_open",
+    "unipin_kvpool_share_close",
+    "unipin_slot_ring_create",
+    "unipin_slot_ring_acquire",
+    "unipin_slot_ring_release",
+    "unipin_slot_ring_free_count",
+    "unipin_slot_ring_destroy",
 )
 
 
@@ -51,6 +59,14 @@ class UnipinError(RuntimeError):
 class KVPool(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("L", ctypes.c_int), ("S", ctypes.c_int),
                 ("H", ctypes.c_int), ("n_cap", ctypes.c_int), ("D", ctypes.c_int)]
+
+
+class KVPoolShare(ctypes.Structure):
+    """unipin_kvpool_share: IPC handles, offsets and shape of a pool (plain bytes)."""
+    _fields_ = [("k_handle", ctypes.c_ubyte * 64), ("v_handle", ctypes.c_ubyte * 64),
+                ("k_offset", ctypes.c_ulonglong), ("v_offset", ctypes.c_ulonglong),
+                ("L", ctypes.c_int), ("S", ctypes.c_int), ("H", ctypes.c_int), ("n_cap", ctypes.c_int),
+                ("D", ctypes.c_int)]
 
 
 def _load(path: str = _LIB_PATH):
@@ -79,6 +95,22 @@ def _load(path: str = _LIB_PATH):
     lib.unipin_rank_decode_attn_noalloc.restype = I
     lib.unipin_rank_decode_noalloc_scratch_bytes.argtypes = []
     lib.unipin_rank_decode_noalloc_scratch_bytes.restype = SZ
+    lib.unipin_kvpool_share_export.argtypes = [P, P]
+    lib.unipin_kvpool_share_export.restype = I
+    lib.unipin_kvpool_share_open.argtypes = [P, P]
+    lib.unipin_kvpool_share_open.restype = I
+    lib.unipin_kvpool_share_close.argtypes = [P, P]
+    lib.unipin_kvpool_share_close.restype = I
+    lib.unipin_slot_ring_create.argtypes = [I, ctypes.POINTER(P)]
+    lib.unipin_slot_ring_create.restype = I
+    lib.unipin_slot_ring_acquire.argtypes = [P, I, ctypes.POINTER(I)]
+    lib.unipin_slot_ring_acquire.restype = I
+    lib.unipin_slot_ring_release.argtypes = [P, I, ctypes.POINTER(I)]
+    lib.unipin_slot_ring_release.restype = I
+    lib.unipin_slot_ring_free_count.argtypes = [P]
+    lib.unipin_slot_ring_free_count.restype = I
+    lib.unipin_slot_ring_destroy.argtypes = [P]
+    lib.unipin_slot_ring_destroy.restype = None
     return lib
 
 
@@ -268,3 +300,83 @@ def selftest_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
 
 def status_string(code: int) -> str:
     return LIB.unipin_status_string(int(code)).decode()
+
+
+# ------------------------------------------------- pool sharing and slot ring
+
+def kvpool_share_export(pool_k: torch.Tensor, pool_v: torch.Tensor) -> bytes:
+    """IPC description of a pool (bytes to hand to another process, e.g. through a file)."""
+    pool = _pool(pool_k, pool_v)
+    desc = KVPoolShare()
+    _check(LIB.unipin_kvpool_share_export(ctypes.byref(pool), ctypes.byref(desc)), "unipin_kvpool_share_export")
+    return bytes(desc)
+
+
+class _DeviceArray:
+    """A zero-copy view of device memory owned elsewhere, for torch.as_tensor."""
+
+    def __init__(self, ptr: int, shape):
+        self.__cuda_array_interface__ = {"shape": tuple(int(x) for x in shape), "typestr": "<i2",
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+class SharedPool:
+    """A pool exported by another process, mapped into this one.
+
+    ``k`` and ``v`` are bf16 tensors [L, S, H, n_cap, D] over the exporter's
+    memory, usable with every call of this module; ``close()`` unmaps them.
+    """
+
+    def __init__(self, desc: bytes, device=None):
+        if len(desc) != ctypes.sizeof(KVPoolShare):
+            raise ValueError("a pool description is %d bytes" % ctypes.sizeof(KVPoolShare))
+        self._desc = KVPoolShare.from_buffer_copy(desc)
+        self._pool = KVPool()
+        _check(LIB.unipin_kvpool_share_open(ctypes.byref(self._desc), ctypes.byref(self._pool)),
+               "unipin_kvpool_share_open")
+        d = self._desc
+        shape = (d.L, d.S, d.H, d.n_cap, d.D)
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.k = torch.as_tensor(_DeviceArray(self._pool.k, shape), device=dev).view(torch.bfloat16)
+        self.v = torch.as_tensor(_DeviceArray(self._pool.v, shape), device=dev).view(torch.bfloat16)
+
+    def close(self):
+        if self._pool.k:
+            self.k = self.v = None
+            _check(LIB.unipin_kvpool_share_close(ctypes.byref(self._desc), ctypes.byref(self._pool)),
+                   "unipin_kvpool_share_close")
+
+
+class SlotRing:
+    """Round-robin assignment of pool slots to requests (host side, thread-safe)."""
+
+    def __init__(self, S: int):
+        h = ctypes.c_void_p()
+        _check(LIB.unipin_slot_ring_create(int(S), ctypes.byref(h)), "unipin_slot_ring_create")
+        self._h = h
+        self._destroy = LIB.unipin_slot_ring_destroy
+        self.S = int(S)
+
+    def acquire(self, n: int):
+        ids = (ctypes.c_int * max(int(n), 1))()
+        _check(LIB.unipin_slot_ring_acquire(self._h, int(n), ids), "unipin_slot_ring_acquire")
+        return [ids[i] for i in range(int(n))]
+
+    def release(self, slot_ids):
+        slot_ids = [int(s) for s in slot_ids]
+        ids = (ctypes.c_int * max(len(slot_ids), 1))(*slot_ids)
+        _check(LIB.unipin_slot_ring_release(self._h, len(slot_ids), ids), "unipin_slot_ring_release")
+
+    def free_count(self) -> int:
+        n = LIB.unipin_slot_ring_free_count(self._h)
+        if n < 0:
+            raise UnipinError(n, "unipin_slot_ring_free_count")
+        return n
+
+    def close(self):
+        if getattr(self, "_h", None):
+            self._destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
