@@ -71,17 +71,26 @@ def pool_write_bytes(past, H, D):
 # by the kernel source it was taken on.  A changed kernel reports null until
 # it is captured again.
 _PREFILL_TRAFFIC_PER_TOKEN = {
-    # sha256 prefix of csrc/attn_sm100.cuh, H, D: bytes per token
-    ("f13854000651ad27", 8, 128): (431.669760e6 + 123.166208e6) / 70236,
+    # kernel_source_key() of csrc/attn_sm100.cuh, H, D: bytes per token
+    ("03012fff8e2df70c", 8, 128): (431.669760e6 + 123.166208e6) / 70236,
 }
 
 
-def prefill_traffic(T, H, D):
+def kernel_source_key(path=None):
+    """sha256 prefix of the attention kernel's code with comments and blank
+    space removed: what the captured counters depend on."""
     import hashlib
-    src = os.path.join(ROOT, "kv_cache_reuse_falcon_b200", "csrc", "attn_sm100.cuh")
-    with open(src, "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    per = _PREFILL_TRAFFIC_PER_TOKEN.get((sha, H, D))
+    import re
+    path = path or os.path.join(ROOT, "kv_cache_reuse_falcon_b200", "csrc", "attn_sm100.cuh")
+    with open(path) as f:
+        text = f.read()
+    code = re.sub(r"/\*.*?\*/", "", re.sub(r"//[^\n]*", "", text), flags=re.S)
+    code = "\n".join(" ".join(ln.split()) for ln in code.splitlines() if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
+
+
+def prefill_traffic(T, H, D):
+    per = _PREFILL_TRAFFIC_PER_TOKEN.get((kernel_source_key(), H, D))
     return None if per is None else per * T
 
 

@@ -1,10 +1,10 @@
 // M-FALCON masked attention engine for sm_100a.
 //
 // Work item = (segment, head, pair of 128-row query tiles A and B[, key split]).
-// The two tiles share every K/V tile and run as a ping-pong: while the
-// tensor cores work on one tile's S = Q K^T and O += P V, the other tile's
-// softmax warpgroup turns its scores into probabilities.  Blocks are
-// persistent (one per SM): each walks its share of the items, and the next
+// The two tiles share every K/V tile; each has its own softmax warpgroup and
+// its own MMA-issuing warp, and the next key tile's S = Q K^T of a tile is
+// computed while its softmax works on the current one.  Blocks are
+// persistent (one per SM) and take items from the producer warp; the next
 // item's Q and first K/V tiles load, and its first S MMAs run, while the
 // softmax warpgroups finish the previous item's epilogue.
 //
@@ -31,12 +31,19 @@
 //              Because P does not overwrite S, the next key tile's S = Q K^T
 //              is computed while this tile's softmax runs: the tensor cores
 //              never wait for a softmax to finish before starting on the next S.
-//   warp 8     TMA producer: per item the Q tiles, then K_0, V_0, K_1, V_1, ...
-//              through a ring of shared-memory slots (the ring runs across items).
+//   warp 8     TMA producer: claims work items (from a counter in the caller's
+//              workspace, or by a fixed stride) and hands them to the other
+//              warps through a small shared-memory ring; per item it loads the
+//              Q tiles, then K_i and V_i of key tile i together into one slot
+//              of a ring of shared-memory slots (the ring runs across items).
 //   warps 9, 10 the UMMA issuers of tile A and tile B (one elected thread each);
-//              warp 9 also allocates TMEM.
+//              warp 9 also allocates TMEM.  Per key tile each waits only for
+//              "S read out" (which also says the next slot has landed) and
+//              "P stored": a wait issued right behind MMAs stalls the issuing
+//              warp until they drain, so the fewer the better.
 //   warp 11    idle (it completes the third warpgroup for the register split).
-// Every warp walks the same item sequence (ItemWalker), so no queue is shared.
+// Every warp maps a global item index to its segment with the same
+// warp-cooperative walker (ItemWalker).
 //
 // Key tiles are kN = 64 keys wide at D = 128 and 128 keys otherwise, so that
 // each query tile's S (kN columns), P (kN/2 columns of bf16 pairs) and O (D
