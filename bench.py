@@ -246,8 +246,8 @@ def run_ours(args, rank, world, device, dist):
     import torch
     from kv_cache_reuse_falcon_b200 import binding as ub
 
-    name = args.workload
-    w = synth.workload(name)
+    w = synth.workload(args.workload)
+    name = w.name
     seed = rank_seed(w.seed, rank)
     w, batch, S, n_cap = make_workload(name, seed, args.users)
     H, D = batch.H, batch.D
@@ -530,7 +530,7 @@ def run_decode_only(args, rank, world, device, dist):
         "metric": METRIC, "value": float(cand.sum()) * L / (ms_step * 1e-3), "unit": "candidate tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
+        "config": {"workload": w.name, "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
                    "pool": [L, S, H, n_cap, D], "layers_per_step": L, "split_n": ws_bytes > 256,
                    "cuda_graph": bool(args.graph),
                    "l2": "pool slots read per step exceed L2 (no flush)"},
@@ -545,8 +545,8 @@ def run_reference(args, rank, world):
     """The oracle (fp64 CPU) timed on the host cores, a bounded sample of the same workload per step."""
     if rank != 0:
         return None
-    name = args.workload
-    w = synth.workload(name)
+    w = synth.workload(args.workload)
+    name = w.name
     _, batch, _, _ = make_workload(name, w.seed)
     for _ in range(args.warmup):
         cpu_oracle_sample(batch, budget_s=0.5, max_segments=1, seed=99)

@@ -59,3 +59,19 @@ def test_clock_sampler_without_nvidia_smi(tmp_path, monkeypatch):
     c = bench.ClockSampler(0)
     c.start()
     assert c.stop() is None
+
+
+def test_reference_arm_prints_one_oracle_line():
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    assert d["config"]["workload"].startswith("tiny_prefill_B2_H2_D32")
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
