@@ -441,6 +441,8 @@ def run_decode_only(args, rank, world, device, dist):
     past = np.full(w.B, w.n, np.int32)
     cand = np.full(w.B, kk, np.int32)
     H, D, L, S, n_cap = w.H, w.D, w.L, w.S, w.n_cap
+    if args.layers > 0:
+        L = args.layers        # smaller pool and fewer layer calls per step (profiler captures)
     slots = rng.permutation(S)[: w.B].astype(np.int32)
 
     def dev_bf16(bits):
@@ -530,7 +532,8 @@ def run_decode_only(args, rank, world, device, dist):
         "metric": METRIC, "value": float(cand.sum()) * L / (ms_step * 1e-3), "unit": "candidate tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
+        "config": {"workload": w.name if args.layers <= 0 else "%s[layers=%d]" % (w.name, L),
+                   "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
                    "pool": [L, S, H, n_cap, D], "layers_per_step": L, "split_n": ws_bytes > 256,
                    "cuda_graph": bool(args.graph),
                    "l2": "pool slots read per step exceed L2 (no flush)"},
@@ -591,6 +594,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--users", type=int, default=0, help="smaller case: this many users (profiling)")
     ap.add_argument("--k", type=int, default=0, help="decode workloads: candidates per request")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="decode workloads: pool layers and layer calls per step (smaller case)")
     ap.add_argument("--graph", action="store_true",
                     help="decode workloads: replay each step's layer calls as one CUDA graph")
     args = ap.parse_args(argv)

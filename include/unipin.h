@@ -29,8 +29,12 @@
  *     Errors the kernels find in device arrays (a length or slot id out of
  *     range) and bounded waits that ran out of time are stored into
  *     *dev_status (device int, may be NULL; 0 = no error, the first error
- *     wins) and the affected blocks exit without writing; a kernel never
- *     traps.  The caller clears *dev_status and reads it back when it likes.
+ *     wins); a kernel never traps.  The rows of a segment or request found
+ *     out of range are written as zeros when the segment's own rows lie
+ *     inside the tensors (rows of a segment whose cu_seqlens range is
+ *     itself out of bounds are not written).  After a timeout the output is
+ *     undefined.  The caller clears *dev_status and reads it back when it
+ *     likes.
  */
 #ifndef UNIPIN_H
 #define UNIPIN_H
@@ -127,15 +131,22 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
  * prefill returns for those rows.
  *   q_c, k_c, v_c  [T_c, H, D] bf16, T_c = total_cand = cu_seqlens_c[R]
  *   out            [T_c, H, D], fp32 if out_fp32 else bf16
- *   max_k          host int >= every k_r (sizes the grid)
+ *   max_k          host int >= every k_r (sizes the grid and picks the kernel: with
+ *                  max_k <= 128 and D in {64, 128} the pool keys are the tensor-core
+ *                  M dimension and a request's key range is swept by several thread
+ *                  blocks, the bandwidth-bound case; otherwise 128-candidate query
+ *                  tiles run through the prefill engine)
  *   workspace      optional device scratch, 16-byte aligned (NULL allowed).  With at
  *                  least 256 bytes the blocks take work items from a shared counter
  *                  (zeroed by the call on `stream`); with at least
  *                  unipin_rank_decode_workspace_size(...) bytes the pool sweep of
  *                  each request is also split over several thread blocks (split-n)
- *                  and merged by a second kernel when that helps.  The result is
- *                  the same either way up to fp32 rounding.  Two calls that overlap
- *                  in time must not share a workspace.
+ *                  when that helps, and the splits are merged (in the kernel for
+ *                  max_k <= 128, by a second kernel otherwise; the per-request
+ *                  arrival counters the in-kernel merge uses are zeroed by the call
+ *                  on `stream`).  The result is the same either way up to fp32
+ *                  rounding.  Two calls that overlap in time must not share a
+ *                  workspace.
  */
 int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
                             const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H,
@@ -144,7 +155,9 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
 
 /* Bytes of workspace unipin_rank_decode_attn uses at most for these sizes
  * (n_cap = the pool's rows per slot): 256 for the work counter, plus the
- * split-n partial results when it would split. */
+ * split-n partial results (and, for max_k <= 128, one arrival counter per
+ * request and head) when it would split.  The split grows with the device's
+ * SM count; the size returned covers the current device and a 148-SM B200. */
 size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap);
 
 /*
@@ -152,12 +165,12 @@ size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int tot
  * counterpart to this on the pages; it exists for callers that cannot call
  * cudaMalloc at decode time: a serving process whose device memory is already
  * handed to another framework's pool, or a loop that must not allocate after
- * start-up.  Arguments, results and errors are those of
- * unipin_rank_decode_attn; the scratch it needs (a work counter and, for
- * small candidate counts, the split-n partial results) lives in a device
- * array of unipin_rank_decode_noalloc_scratch_bytes() bytes (32 MiB) that the
- * library reserves on every device it is loaded on and keeps until the
- * process exits.
+ * start-up.  Arguments and results are those of unipin_rank_decode_attn,
+ * and so are its errors, with one more: the scratch it needs (a work counter
+ * and, when the pool sweep is split, the split-n partial results and arrival
+ * counters) lives in a device array of unipin_rank_decode_noalloc_scratch_bytes()
+ * bytes (32 MiB) that the library reserves on every device it is loaded on
+ * and keeps until the process exits.
  *   - If unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand,
  *     pool->n_cap) exceeds that size, nothing is launched and
  *     UNIPIN_ERR_OUT_OF_RANGE is returned.

@@ -139,17 +139,6 @@ __device__ __forceinline__ void key_tile(int t, int nt, int kmax, int& start, in
     start = (t == nt - 1 && (kmax % kN) != 0) ? kmax - kN : lo;
 }
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
-{
-    const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&b);
-}
-
-__device__ __forceinline__ void report(int* status, int code)
-{
-    if (status) atomicCAS(status, 0, code);
-}
-
 // Warp-cooperative map from a global item index g (segment-major: the items
 // of segment 0, then of segment 1, ...) to its segment.  Every lane of the
 // calling warp must call locate() together; all lanes get the same answer.
@@ -219,6 +208,7 @@ struct ItemWalker {
 // Everything about one item that every role derives identically.
 struct Work {
     bool valid;
+    bool rows_ok;               // the segment's rows lie inside the token tensors
     int seg, h, split;
     int tok0, npast, slot;
     int qrow0;                  // first row of tile A within the segment
@@ -244,7 +234,8 @@ __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int loca
     const int nrows_seg = p.cu[seg + 1] - w.tok0;
     w.npast = p.past[seg];
     w.slot = kDecode ? p.slots[seg] : 0;
-    bool bad = w.tok0 < 0 || w.npast < 0 || (long long)w.tok0 + nrows_seg > (long long)p.total_rows;
+    w.rows_ok = w.tok0 >= 0 && nrows_seg >= 0 && (long long)w.tok0 + nrows_seg <= (long long)p.total_rows;
+    bool bad = !w.rows_ok || w.npast < 0;
     if (kDecode)
         bad = bad || w.slot < 0 || w.slot >= p.S || w.npast > p.n_cap;
     else
@@ -612,7 +603,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             const Work w = make_work<kDecode, C::kN>(p, seg, local);
             const int u_item = u_sm;
             u_sm += w.nt;
-            if (!w.valid) continue;
+            if (!w.valid) {
+                // A segment whose history length or slot id is out of range: its rows get
+                // zeros (a split partial marked invalid, l = -1, which the merge turns into
+                // zeros), so no row is left holding another call's values.
+                const int nrows_x = x == 0 ? w.nrows_a : w.nrows_b;
+                if (w.rows_ok && r < nrows_x) {
+                    const size_t tok = (size_t)w.tok0 + w.qrow0 + x * kBlockM + r;
+                    if (split_mode) {
+                        float* ml = p.part_ml + (((size_t)w.split * p.total_rows + tok) * p.H + w.h) * 2;
+                        ml[0] = -INFINITY;
+                        ml[1] = -1.f;
+                    } else if (p.out_fp32) {
+                        float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + (tok * p.H + w.h) * D);
+#pragma unroll
+                        for (int c = 0; c < D / 4; ++c) dst[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    } else {
+                        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out) + (tok * p.H + w.h) * D);
+#pragma unroll
+                        for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+                continue;
+            }
             const int ntx = x == 0 ? w.nt_a : w.nt_b;
             const int nrows_x = x == 0 ? w.nrows_a : w.nrows_b;
             if (nrows_x <= 0) continue;
@@ -879,8 +892,10 @@ __global__ void __launch_bounds__(256)
     for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
     const float ss = dot * sl2;
     float m_fin = ss;
+    bool invalid = false;   // the request was rejected on the device: its rows are zeros
     for (int s = 0; s < nsplit; ++s) {
         const float ms = part_ml[((size_t)s * total_rows * H + row) * 2];
+        invalid |= part_ml[((size_t)s * total_rows * H + row) * 2 + 1] < 0.f;
         m_fin = fmaxf(m_fin, ms);
     }
     float acc[E];
@@ -898,7 +913,11 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = fmaf(w, po[e], acc[e]);
     }
-    const float inv = 1.f / den;
+    const float inv = invalid ? 0.f : 1.f / den;
+    if (invalid) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    }
     if (out_fp32) {
         float* dst = reinterpret_cast<float*>(out) + base;
 #pragma unroll

@@ -13,6 +13,7 @@
 #include "unipin.h"
 #include "sm100_ptx.cuh"
 #include "attn_sm100.cuh"
+#include "decode_smallk_sm100.cuh"
 #include "kvpool_sm100.cuh"
 
 using namespace unipin;
@@ -40,12 +41,23 @@ unsigned long long wait_limit_ns()
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Persistent grid: one block per SM, fewer if there cannot be that many items.
-unsigned persistent_blocks(long long item_bound)
+// SM count of the current device (queried once per device; the B200 count if
+// the query fails, e.g. on a machine without a device).
+int current_sms()
 {
     int dev = 0;
-    cudaGetDevice(&dev);
-    const int sms = (dev >= 0 && dev < kMaxDevices && g_num_sms[dev] > 0) ? g_num_sms[dev] : kNumSmsHint;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return kNumSmsHint;
+    if (g_num_sms[dev] > 0) return g_num_sms[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return kNumSmsHint;
+    g_num_sms[dev] = n;
+    return n;
+}
+
+// Persistent grid: `per_sm` blocks per SM, fewer if there cannot be that many items.
+unsigned persistent_blocks(long long item_bound, int per_sm = 1)
+{
+    const long long sms = (long long)current_sms() * per_sm;
     long long n = item_bound < sms ? item_bound : sms;
     return (unsigned)(n < 1 ? 1 : n);
 }
@@ -69,6 +81,25 @@ int set_attn_attrs()
     int rc = set_attn_attr(attn_fwd_kernel<D, false>, AttnCfg<D>::kSmemBytes);
     if (rc != UNIPIN_OK) return rc;
     return set_attn_attr(attn_fwd_kernel<D, true>, AttnCfg<D>::kSmemBytes);
+}
+
+template <int D, int N>
+int set_sk_attr()
+{
+    return cudaFuncSetAttribute(decode_smallk_kernel<D, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SkCfg<D, N>::kSmemBytes) == cudaSuccess
+               ? UNIPIN_OK
+               : UNIPIN_ERR_CUDA;
+}
+
+template <int D>
+int set_sk_attrs()
+{
+    int rc = set_sk_attr<D, 16>();
+    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 32>();
+    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 64>();
+    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 128>();
+    return rc;
 }
 
 // Once per device: check it is an sm_100 part, resolve the tensor-map
@@ -98,6 +129,8 @@ int ensure_device()
     int rc = set_attn_attrs<32>();
     if (rc == UNIPIN_OK) rc = set_attn_attrs<64>();
     if (rc == UNIPIN_OK) rc = set_attn_attrs<128>();
+    if (rc == UNIPIN_OK) rc = set_sk_attrs<64>();
+    if (rc == UNIPIN_OK) rc = set_sk_attrs<128>();
     if (rc != UNIPIN_OK) return rc;
     g_device_ready[dev] = true;
     return UNIPIN_OK;
@@ -127,14 +160,14 @@ int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D, int ro
                     (uint32_t)rows, D);
 }
 
-// Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of one key tile of history rows.
-int make_pool_map(CUtensorMap* m, const void* base, const unipin_kvpool* pool)
+// Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of `rows` history rows of one plane.
+int make_pool_map(CUtensorMap* m, const void* base, const unipin_kvpool* pool, int rows)
 {
     const int D = pool->D;
     const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
     const uint64_t planes = (uint64_t)pool->L * pool->S * pool->H;
     return make_map(m, base, (uint64_t)D, (uint64_t)pool->n_cap, planes, (uint64_t)D * 2,
-                    (uint64_t)pool->n_cap * D * 2, box_d, (uint32_t)key_tile_width(D), 1, D);
+                    (uint64_t)pool->n_cap * D * 2, box_d, (uint32_t)rows, 1, D);
 }
 
 int check_pool(const unipin_kvpool* pool, int H, int D, int layer)
@@ -196,11 +229,11 @@ int launch_pool_write(const unipin_kvpool* pool, int layer, const void* k, const
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 
-int decode_nsplit(int R, int H, int D, int max_k, int n_cap)
+int decode_nsplit(int R, int H, int D, int max_k, int n_cap, int sms)
 {
     if (R < 1 || H < 1 || max_k < 1 || n_cap < 1) return 1;
     const long long units = (long long)R * H * ((max_k + kPairRows - 1) / kPairRows);
-    const long long slots = (long long)kNumSmsHint;   // one block per SM (all of TMEM)
+    const long long slots = (long long)sms;   // one block per SM (all of TMEM)
     const long long target = 4 * slots;
     if (units >= 2 * slots) return 1;   // two or more waves already: no split
     const int key_tiles = (n_cap + key_tile_width(D) - 1) / key_tile_width(D);
@@ -218,6 +251,155 @@ size_t decode_workspace_bytes(int nsplit, int total_cand, int H, int D)
     if (nsplit <= 1) return kSchedBytes;
     const size_t rows = (size_t)nsplit * (size_t)total_cand * (size_t)H;
     return kSchedBytes + rows * (size_t)D * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+// ---- small-k rank decode (keys as the MMA's M; decode_smallk_sm100.cuh)
+
+// Requests with at most this many candidates take the small-k kernel (D 64 or 128).
+constexpr int kSmallKMax = 128;
+
+bool use_small_k(int D, int max_k) { return (D == 64 || D == 128) && max_k >= 1 && max_k <= kSmallKMax; }
+
+int sk_ctas_per_sm(int D, int N)
+{
+    if (D == 64) {
+        switch (N) {
+        case 16: return SkCfg<64, 16>::kCtasPerSm;
+        case 32: return SkCfg<64, 32>::kCtasPerSm;
+        case 64: return SkCfg<64, 64>::kCtasPerSm;
+        default: return SkCfg<64, 128>::kCtasPerSm;
+        }
+    }
+    switch (N) {
+    case 16: return SkCfg<128, 16>::kCtasPerSm;
+    case 32: return SkCfg<128, 32>::kCtasPerSm;
+    case 64: return SkCfg<128, 64>::kCtasPerSm;
+    default: return SkCfg<128, 128>::kCtasPerSm;
+    }
+}
+
+// Work items a resident block should get on average (load balance against
+// per-item overhead); UNIPIN_DECODE_ITEMS_PER_BLOCK overrides it.
+int sk_items_per_block()
+{
+    static int v = [] {
+        const char* s = std::getenv("UNIPIN_DECODE_ITEMS_PER_BLOCK");
+        int n = s ? std::atoi(s) : 0;
+        return n > 0 ? n : 4;
+    }();
+    return v;
+}
+
+struct SkPlan {
+    int N, nsplit, tiles_per_split, blocks_per_sm;
+};
+
+// Key splits per (request, head): cut the pool sweep into runs of whole
+// 128-key tiles so that the grid gets about sk_items_per_block() items per
+// resident block, at most kSkMaxSplit runs.
+SkPlan sk_plan(int R, int H, int D, int max_k, int n_cap, int sms)
+{
+    SkPlan pl;
+    pl.N = sk_pad_n(max_k);
+    pl.blocks_per_sm = sk_ctas_per_sm(D, pl.N);
+    const long long tiles = (n_cap + kSkKeys - 1) / kSkKeys;
+    const long long pairs = (long long)R * H;
+    const long long target = (long long)sk_items_per_block() * sms * pl.blocks_per_sm;
+    long long per = (pairs * tiles + target - 1) / target;
+    if (per < 1) per = 1;
+    if (per > tiles) per = tiles;
+    long long ns = (tiles + per - 1) / per;
+    if (ns > kSkMaxSplit) {
+        per = (tiles + kSkMaxSplit - 1) / kSkMaxSplit;
+        ns = (tiles + per - 1) / per;
+    }
+    pl.nsplit = (int)(ns < 1 ? 1 : ns);
+    pl.tiles_per_split = (int)(pl.nsplit == 1 ? (tiles < 1 ? 1 : tiles) : per);
+    return pl;
+}
+
+// Workspace of the small-k decode: work counter, per-(request, head) arrival
+// counters, then the split partials O [nsplit, T, H, D] and (m, l) [nsplit, T, H, 2].
+size_t sk_counter_bytes(int R, int H) { return ((size_t)R * H * sizeof(unsigned) + 255) / 256 * 256; }
+
+size_t sk_workspace_bytes(const SkPlan& pl, int R, int H, int D, int total_cand)
+{
+    if (pl.nsplit <= 1) return kSchedBytes;
+    const size_t rows = (size_t)pl.nsplit * (size_t)total_cand * (size_t)H;
+    return kSchedBytes + sk_counter_bytes(R, H) + rows * (size_t)D * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+template <int D, int N>
+int launch_sk_kernel(unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     const SkParams& p, cudaStream_t s)
+{
+    decode_smallk_kernel<D, N><<<grid, kSkThreads, SkCfg<D, N>::kSmemBytes, s>>>(tq, tk, tv, p);
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+template <int D>
+int launch_sk_d(int N, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const SkParams& p, cudaStream_t s)
+{
+    switch (N) {
+    case 16: return launch_sk_kernel<D, 16>(grid, tq, tk, tv, p, s);
+    case 32: return launch_sk_kernel<D, 32>(grid, tq, tk, tv, p, s);
+    case 64: return launch_sk_kernel<D, 64>(grid, tq, tk, tv, p, s);
+    default: return launch_sk_kernel<D, 128>(grid, tq, tk, tv, p, s);
+    }
+}
+
+int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
+                        const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H, int D,
+                        int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer,
+                        void* workspace, size_t workspace_bytes, int* dev_status, cudaStream_t s)
+{
+    SkPlan pl = sk_plan(R, H, D, max_k, pool->n_cap, current_sms());
+    if (pl.nsplit > 1 && (!workspace || workspace_bytes < sk_workspace_bytes(pl, R, H, D, total_cand))) {
+        pl.nsplit = 1;
+        pl.tiles_per_split = (pool->n_cap + kSkKeys - 1) / kSkKeys;
+    }
+    unsigned long long* sched = nullptr;
+    if (workspace && workspace_bytes >= kSchedBytes) {
+        sched = static_cast<unsigned long long*>(workspace);
+        const size_t zero = pl.nsplit > 1 ? kSchedBytes + sk_counter_bytes(R, H) : sizeof(unsigned long long);
+        if (cudaMemsetAsync(workspace, 0, zero, s) != cudaSuccess) return UNIPIN_ERR_CUDA;
+    }
+    CUtensorMap tq, tk, tv;
+    int rc;
+    if ((rc = make_token_map(&tq, q_c, total_cand, H, D, pl.N)) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tk, pool->k, pool, kSkKeys)) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tv, pool->v, pool, kSkKeys)) != UNIPIN_OK) return rc;
+
+    SkParams p = {};
+    p.q = static_cast<const __nv_bfloat16*>(q_c);
+    p.k_self = static_cast<const __nv_bfloat16*>(k_c);
+    p.v_self = static_cast<const __nv_bfloat16*>(v_c);
+    p.out = out;
+    p.cu = cu_seqlens_c;
+    p.past = past_lens;
+    p.slots = slot_ids;
+    p.R = R;
+    p.H = H;
+    p.total_rows = total_cand;
+    p.out_fp32 = out_fp32 ? 1 : 0;
+    p.layer = layer;
+    p.S = pool->S;
+    p.n_cap = pool->n_cap;
+    p.nsplit = pl.nsplit;
+    p.tiles_per_split = pl.tiles_per_split;
+    p.sl2 = scale * kLog2e;
+    p.status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+    p.sched = sched;
+    if (pl.nsplit > 1) {
+        char* ws = static_cast<char*>(workspace);
+        p.pair_cnt = reinterpret_cast<unsigned*>(ws + kSchedBytes);
+        p.part_o = reinterpret_cast<float*>(ws + kSchedBytes + sk_counter_bytes(R, H));
+        p.part_ml = p.part_o + (size_t)pl.nsplit * total_cand * H * D;
+    }
+    const unsigned grid = persistent_blocks((long long)R * H * pl.nsplit, pl.blocks_per_sm);
+    return D == 64 ? launch_sk_d<64>(pl.N, grid, tq, tk, tv, p, s) : launch_sk_d<128>(pl.N, grid, tq, tk, tv, p, s);
 }
 
 __global__ void bounded_wait_selftest_kernel(int* status, unsigned long long limit_ns)
@@ -361,7 +543,10 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
 size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap)
 {
     if (R < 1 || H < 1 || !supported_d(D) || max_k < 1 || total_cand < 1 || n_cap < 1) return 0;
-    return decode_workspace_bytes(decode_nsplit(R, H, D, max_k, n_cap), total_cand, H, D);
+    // The split grows with the SM count: size for the larger of this device's and a B200's.
+    const int sms = current_sms() > kNumSmsHint ? current_sms() : kNumSmsHint;
+    if (use_small_k(D, max_k)) return sk_workspace_bytes(sk_plan(R, H, D, max_k, n_cap, sms), R, H, D, total_cand);
+    return decode_workspace_bytes(decode_nsplit(R, H, D, max_k, n_cap, sms), total_cand, H, D);
 }
 
 int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
@@ -381,8 +566,11 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_small_k(D, max_k))
+        return rank_decode_small_k(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, slot_ids, past_lens, R, H, D, max_k,
+                                   total_cand, scale, pool, layer, workspace, workspace_bytes, dev_status, s);
 
-    int nsplit = decode_nsplit(R, H, D, max_k, pool->n_cap);
+    int nsplit = decode_nsplit(R, H, D, max_k, pool->n_cap, current_sms());
     if (nsplit > 1 && (!workspace || workspace_bytes < decode_workspace_bytes(nsplit, total_cand, H, D))) nsplit = 1;
     unsigned long long* sched = nullptr;
     if (workspace && workspace_bytes >= kSchedBytes) {
@@ -392,8 +580,8 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
 
     CUtensorMap tq, tk, tv;
     if ((rc = make_token_map(&tq, q_c, total_cand, H, D, kBlockM)) != UNIPIN_OK) return rc;
-    if ((rc = make_pool_map(&tk, pool->k, pool)) != UNIPIN_OK) return rc;
-    if ((rc = make_pool_map(&tv, pool->v, pool)) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tk, pool->k, pool, key_tile_width(D))) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tv, pool->v, pool, key_tile_width(D))) != UNIPIN_OK) return rc;
 
     AttnParams p = {};
     p.q = static_cast<const __nv_bfloat16*>(q_c);

@@ -40,3 +40,29 @@ def shard_segments(past_lens, cand_lens, world_size: int) -> List[np.ndarray]:
 def rank_seed(base_seed: int, rank: int) -> int:
     """Seed of rank `rank` in a weak-scaling run: every rank draws its own batch of users."""
     return int(base_seed) + 7919 * int(rank)
+
+
+def combine_rank_results(times, counts, group=None, device=None):
+    """Whole-job numbers of a weak-scaling run from every rank's own numbers.
+
+    times:  dict name -> this rank's duration (ms); the job takes as long as its
+            slowest rank, so each becomes the maximum over ranks.
+    counts: dict name -> this rank's work (candidates scored, FLOPs, bytes); each
+            becomes the sum over ranks.
+    group:  a torch.distributed process group (None: the default group), or
+            False for a single-process run (returned unchanged).
+    device: where the reduction tensors live (a CUDA device for NCCL, CPU for gloo).
+    Every rank must call this with the same keys, in the same order.
+    """
+    if group is False:
+        return dict(times), dict(counts)
+    import torch
+    import torch.distributed as dist
+    tk, ck = list(times), list(counts)
+    t = torch.tensor([float(times[k]) for k in tk], dtype=torch.float64, device=device)
+    c = torch.tensor([float(counts[k]) for k in ck], dtype=torch.float64, device=device)
+    if t.numel():
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    if c.numel():
+        dist.all_reduce(c, op=dist.ReduceOp.SUM, group=group)
+    return dict(zip(tk, t.tolist())), dict(zip(ck, c.tolist()))

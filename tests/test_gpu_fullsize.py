@@ -113,20 +113,22 @@ def test_rank_decode_from_pool_workload(ub):
     rows = sample_rows(d.cu_seqlens, np.zeros_like(past), 1500, 3)
     ref = oracle.decode(d.q, d.k, d.v, d.cu_seqlens, d.slot_ids, d.past_lens, hk, hv, 0, tokens=rows)
     parity(out[torch.from_numpy(rows).cuda()].cpu().numpy(), ref, "decode R32 k1000")
-    # small-k sweep over the same pool with the split-n path (k = 16 per request)
-    cand16 = np.full(w.B, 16, np.int32)
-    d16 = synth.make_decode(w.seed + 100, past, cand16, w.H, w.D, n_slots=w.S)
-    d16.slot_ids = d.slot_ids
-    dd16 = DevDecode(d16)
-    nbytes = ub.rank_decode_workspace_size(w.B, w.H, w.D, 16, int(d16.cu_seqlens[-1]), w.n_cap)
-    assert nbytes > 256
-    ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device="cuda")
-    o16 = ub.rank_decode_attn(dd16.q, dd16.k, dd16.v, dd16.cu, dd16.slots, dd16.past, pk, pv, layer, 16,
-                              out_fp32=True, workspace=ws, dev_status=status)
-    torch.cuda.synchronize()
-    assert int(status.item()) == 0
-    ref16 = oracle.decode(d16.q, d16.k, d16.v, d16.cu_seqlens, d16.slot_ids, d16.past_lens, hk, hv, 0)
-    parity(o16.cpu().numpy(), ref16, "decode R32 k16 split-n")
+    # candidate-count sweep over the same pool, as the benchmark runs it (split workspace):
+    # k = 1 is the retrieval stage's one-token step, k <= 128 takes the small-k kernel
+    for kk in (1, 16, 64, 128):
+        candk = np.full(w.B, kk, np.int32)
+        dk = synth.make_decode(w.seed + 100 + kk, past, candk, w.H, w.D, n_slots=w.S)
+        dk.slot_ids = d.slot_ids
+        ddk = DevDecode(dk)
+        nbytes = ub.rank_decode_workspace_size(w.B, w.H, w.D, kk, int(dk.cu_seqlens[-1]), w.n_cap)
+        assert nbytes > 256
+        ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device="cuda")
+        ok_ = ub.rank_decode_attn(ddk.q, ddk.k, ddk.v, ddk.cu, ddk.slots, ddk.past, pk, pv, layer, kk,
+                                  out_fp32=True, workspace=ws, dev_status=status)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        refk = oracle.decode(dk.q, dk.k, dk.v, dk.cu_seqlens, dk.slot_ids, dk.past_lens, hk, hv, 0)
+        parity(ok_.cpu().numpy(), refk, "decode R32 k%d" % kk)
 
 
 def test_ragged_mixed_batch_prefill_then_decode(ub):

@@ -80,3 +80,41 @@ def test_shard_plan_covers_every_user_once_and_balances():
 
 def test_rank_seeds_differ():
     assert len({rank_seed(5, r) for r in range(8)}) == 8
+
+
+def _report_worker(rank, world, port, q):
+    from kv_cache_reuse_falcon_b200.shard import combine_rank_results
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        times = {"step_ms": 10.0 + rank, "prefill_ms": 5.0 - rank, "e2e_ms": 20.0 * (rank + 1)}
+        counts = {"candidates": 1000.0 * (rank + 1), "flops": 1e12}
+        t, c = combine_rank_results(times, counts, device="cpu")
+        q.put((rank, t, c))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_cross_rank_report_takes_max_times_and_summed_work():
+    """The multi-GPU benchmark's reduction: the job's time is its slowest rank's, its work the sum."""
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_report_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, c in res:
+        assert t == {"step_ms": 11.0, "prefill_ms": 5.0, "e2e_ms": 40.0}
+        assert c == {"candidates": 3000.0, "flops": 2e12}
+
+
+def test_single_process_report_is_unchanged():
+    from kv_cache_reuse_falcon_b200.shard import combine_rank_results
+    t, c = combine_rank_results({"a": 1.5}, {"n": 3}, group=False)
+    assert t == {"a": 1.5} and c == {"n": 3}
