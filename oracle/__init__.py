@@ -1,4 +1,4 @@
-"""CPU oracle (fp64) for the masked prefill, the pool write and the rank decode.
+"""CPU oracle (fp64) for the masked prefill, its gradients, the pool write and the rank decode.
 
 TEST INFRASTRUCTURE ONLY.  The tests, the smoke check and the benchmark's
 CPU-baseline leg may call this package; the library under
@@ -52,6 +52,10 @@ def _load():
         lib.oracle_decode_rows.argtypes = [P, P, P, P, P, P, I, I, I, ctypes.c_double, I,
                                            P, P, I, I, I, I, P, I64, P, P]
         lib.oracle_decode_rows.restype = I
+        lib.oracle_prefill_bwd.argtypes = [P, P, P, P, P, P, I, I, I, ctypes.c_double, I, P, P, P]
+        lib.oracle_prefill_bwd.restype = I
+        lib.oracle_prefill_bwd_f64.argtypes = [P, P, P, P, P, P, I, I, I, ctypes.c_double, I, P, P, P]
+        lib.oracle_prefill_bwd_f64.restype = I
         lib.oracle_pool_write.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, I]
         lib.oracle_pool_write.restype = I
         lib.oracle_num_threads.restype = I
@@ -146,3 +150,34 @@ def pool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids
                                    _ptr(k), _ptr(v), _ptr(cu), _ptr(past), _ptr(slots), past.shape[0])
     if rc != 0:
         raise ValueError("oracle_pool_write rejected its arguments")
+
+
+def _bwd(fn, q, k, v, dout, cu_seqlens, past_lens, scale, cand_self):
+    T, H, D = q.shape
+    cu = _i32(cu_seqlens)
+    past = _i32(past_lens)
+    B = past.shape[0]
+    if cu.shape[0] != B + 1 or int(cu[-1]) != T:
+        raise ValueError("cu_seqlens does not match q")
+    for a in (k, v, dout):
+        if a.shape != q.shape:
+            raise ValueError("q, k, v and dout must have one shape")
+    scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
+    dq, dk, dv = (np.zeros((T, H, D), dtype=np.float64) for _ in range(3))
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(cu), _ptr(past), B, H, D, scale, int(bool(cand_self)),
+            _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc != 0:
+        raise ValueError("oracle backward rejected its arguments")
+    return dq, dk, dv
+
+
+def prefill_bwd(q, k, v, dout, cu_seqlens, past_lens, scale: Optional[float] = None, cand_self: bool = True):
+    """Gradients (dq, dk, dv), float64 [T, H, D], of the masked prefill for upstream gradient dout (bf16 bits)."""
+    q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
+    return _bwd(_load().oracle_prefill_bwd, q, k, v, dout, cu_seqlens, past_lens, scale, cand_self)
+
+
+def prefill_bwd_f64(q, k, v, dout, cu_seqlens, past_lens, scale: Optional[float] = None, cand_self: bool = True):
+    """As prefill_bwd on float64 inputs (e.g. for finite-difference checks)."""
+    q, k, v, dout = (np.ascontiguousarray(a, dtype=np.float64) for a in (q, k, v, dout))
+    return _bwd(_load().oracle_prefill_bwd_f64, q, k, v, dout, cu_seqlens, past_lens, scale, cand_self)

@@ -1,6 +1,6 @@
 /*
- * CPU oracle for the M-FALCON masked attention, the KV pool write and the
- * cross-stage rank decode.  TEST INFRASTRUCTURE ONLY: the tests, the smoke
+ * CPU oracle for the M-FALCON masked attention (forward and gradients), the
+ * KV pool write and the cross-stage rank decode.  TEST INFRASTRUCTURE ONLY: the tests, the smoke
  * check and the benchmark's CPU-baseline leg call it; the product path never
  * does.  It shares no code, header or constant with the CUDA library.
  *
@@ -252,6 +252,125 @@ int oracle_decode_rows(const uint16_t *qc, const uint16_t *kc, const uint16_t *v
         free((void *)vp);
     }
     return bad ? -1 : 0;
+}
+
+/*
+ * Gradients of the masked prefill attention.  [review] §2.2 trains the whole
+ * sequence [past || candidates] in one forward pass under this mask (the
+ * joint objective); the backward pass below is the plain chain rule of the
+ * forward defined above, over the same allowed (i, j) pairs:
+ *
+ *   P_ij  = softmax_j over allowed j of s_ij,  s_ij = scale * q_i . k_j
+ *   O_i   = sum_j P_ij v_j
+ *   given dO (the gradient of the loss with respect to O):
+ *   dV_j  = sum_i P_ij dO_i
+ *   dP_ij = dO_i . v_j
+ *   dS_ij = P_ij (dP_ij - sum_l P_il dP_il)
+ *   dQ_i  = scale * sum_j dS_ij k_j
+ *   dK_j  = scale * sum_i dS_ij q_i
+ *
+ * so a past key receives gradient from the later past rows and from every
+ * candidate row; a candidate's own key and value only from its own row.
+ * Inputs are doubles (bf16 inputs are widened exactly by the caller);
+ * dq, dk, dv are written in full.  Parallel over (segment, head): every
+ * gradient element belongs to exactly one of them.
+ */
+int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, const double *dout,
+                           const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int D,
+                           double scale, int cand_self, double *dq, double *dk, double *dv)
+{
+    if (B < 1 || H < 1 || D < 1) return -1;
+    int64_t max_len = 0;
+    for (int b = 0; b < B; ++b) {
+        int64_t len = (int64_t)cu_seqlens[b + 1] - cu_seqlens[b];
+        if (len < 0 || past_lens[b] < 0 || past_lens[b] > len) return -1;
+        if (len > max_len) max_len = len;
+    }
+    int64_t T = cu_seqlens[B];
+    memset(dq, 0, sizeof(double) * (size_t)(T * H * D));
+    memset(dk, 0, sizeof(double) * (size_t)(T * H * D));
+    memset(dv, 0, sizeof(double) * (size_t)(T * H * D));
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)(max_len + 1));
+        double *dp = (double *)malloc(sizeof(double) * (size_t)(max_len + 1));
+        int64_t *js = (int64_t *)malloc(sizeof(int64_t) * (size_t)(max_len + 1));
+        if (!p || !dp || !js) {
+#pragma omp atomic write
+            bad = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+            if (bad) continue;
+            int b = (int)(bh / H), h = (int)(bh % H);
+            int64_t start = cu_seqlens[b], len = (int64_t)cu_seqlens[b + 1] - start, n_past = past_lens[b];
+#define ROW(x, t) ((x) + (((start + (t)) * H + h) * (int64_t)D))
+            for (int64_t i = 0; i < len; ++i) {
+                int64_t nk = 0;
+                for (int64_t j = 0; j < len; ++j)
+                    if (allowed(i, j, n_past, cand_self)) js[nk++] = j;
+                if (nk == 0) continue;              /* no key: O_i = 0 carries no gradient */
+                /* forward of row i: P_ij */
+                double m = -INFINITY;
+                for (int64_t a = 0; a < nk; ++a) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += ROW(q, i)[d] * ROW(k, js[a])[d];
+                    p[a] = dot * scale;
+                    if (p[a] > m) m = p[a];
+                }
+                double den = 0.0;
+                for (int64_t a = 0; a < nk; ++a) {
+                    p[a] = exp(p[a] - m);
+                    den += p[a];
+                }
+                for (int64_t a = 0; a < nk; ++a) p[a] /= den;
+                /* dP_ij = dO_i . v_j and its P-weighted mean over the row */
+                double dmean = 0.0;
+                for (int64_t a = 0; a < nk; ++a) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += ROW(dout, i)[d] * ROW(v, js[a])[d];
+                    dp[a] = dot;
+                    dmean += p[a] * dot;
+                }
+                for (int64_t a = 0; a < nk; ++a) {
+                    int64_t j = js[a];
+                    double ds = p[a] * (dp[a] - dmean);
+                    for (int d = 0; d < D; ++d) {
+                        ROW(dv, j)[d] += p[a] * ROW(dout, i)[d];
+                        ROW(dq, i)[d] += scale * ds * ROW(k, j)[d];
+                        ROW(dk, j)[d] += scale * ds * ROW(q, i)[d];
+                    }
+                }
+            }
+#undef ROW
+        }
+        free(p);
+        free(dp);
+        free(js);
+    }
+    return bad ? -1 : 0;
+}
+
+/* As oracle_prefill_bwd_f64 for bf16 inputs (bit patterns), widened exactly. */
+int oracle_prefill_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                       const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int D,
+                       double scale, int cand_self, double *dq, double *dk, double *dv)
+{
+    if (B < 1 || H < 1 || D < 1) return -1;
+    size_t n = (size_t)cu_seqlens[B] * (size_t)H * (size_t)D;
+    double *w = (double *)malloc(sizeof(double) * (4 * n + 1));
+    if (!w) return -1;
+    for (size_t x = 0; x < n; ++x) {
+        w[x] = bf16_to_f64(q[x]);
+        w[n + x] = bf16_to_f64(k[x]);
+        w[2 * n + x] = bf16_to_f64(v[x]);
+        w[3 * n + x] = bf16_to_f64(dout[x]);
+    }
+    int rc = oracle_prefill_bwd_f64(w, w + n, w + 2 * n, w + 3 * n, cu_seqlens, past_lens, B, H, D, scale,
+                                    cand_self, dq, dk, dv);
+    free(w);
+    return rc;
 }
 
 /*
