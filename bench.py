@@ -30,7 +30,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from kv_cache_reuse_falcon_b200 import synth  # noqa: E402
-from kv_cache_reuse_falcon_b200.shard import rank_seed, segment_cost  # noqa: E402
+from kv_cache_reuse_falcon_b200.shard import combine_rank_results, rank_seed, segment_cost  # noqa: E402
 
 DEFAULT_WORKLOAD = "ragged_B256_H8_D128_n32-4096_k50-2000"
 METRIC = "candidate tokens scored/s + prefill TFLOP/s (mask-effective) & decode HBM GB/s"
@@ -283,13 +283,12 @@ def run_ours(args, rank, world, device, dist):
     layer = 0
 
     def step(ev=None):
+        # the prefill also writes every user's past K/V into its pool slot (one kernel)
         if ev is not None:
             ev[0].record(stream)
-        ub.kvpool_write(pool_k, pool_v, layer, k, v, cu, pl, sl, max_past, dev_status=status, stream=stream)
-        if ev is not None:
-            ev[1].record(stream)
         ub.masked_prefill_attn(q, k, v, cu, pl, max_seqlen, out=out_p, out_fp32=False, workspace=ws_pre,
-                               dev_status=status, stream=stream)
+                               pool_k=pool_k, pool_v=pool_v, slot_ids=sl, layer=layer, dev_status=status,
+                               stream=stream)
         if ev is not None:
             ev[2].record(stream)
         ub.rank_decode_attn(qc, kc, vc, cu_c, sl, pl, pool_k, pool_v, layer, max_k, out=out_d, out_fp32=False,
@@ -321,69 +320,90 @@ def run_ours(args, rank, world, device, dist):
         dist.barrier()
     clk = clocks.stop() if clocks else None
     elapsed_ms = start.elapsed_time(stop)
-    t_pool = [e[0].elapsed_time(e[1]) for e in evs]
-    t_pre = [e[1].elapsed_time(e[2]) for e in evs]
+    t_pre = [e[0].elapsed_time(e[2]) for e in evs]
     t_dec = [e[2].elapsed_time(e[3]) for e in evs]
     if int(status.item()) != 0:
         raise RuntimeError("device status %s in the timed region" % ub.status_string(int(status.item())))
 
     # ------------------------------------------------------ end to end (host buffers)
-    hq = torch.from_numpy(batch.q.view(np.int16)).pin_memory()
-    hk = torch.from_numpy(batch.k.view(np.int16)).pin_memory()
-    hv = torch.from_numpy(batch.v.view(np.int16)).pin_memory()
-    hqc = torch.from_numpy(np.ascontiguousarray(batch.q[cidx]).view(np.int16)).pin_memory()
-    hkc = torch.from_numpy(np.ascontiguousarray(batch.k[cidx]).view(np.int16)).pin_memory()
-    hvc = torch.from_numpy(np.ascontiguousarray(batch.v[cidx]).view(np.int16)).pin_memory()
-    hcu = torch.from_numpy(batch.cu_seqlens.astype(np.int32)).pin_memory()
-    hpl = torch.from_numpy(past.astype(np.int32)).pin_memory()
-    hsl = torch.from_numpy(batch.slot_ids.astype(np.int32)).pin_memory()
-    hcuc = torch.from_numpy(synth.cu_from_lens(cand)).pin_memory()
+    # Every step copies its inputs (Q, K, V, the length / slot arrays and the
+    # candidate row index) from pinned host memory on a copy stream into one of
+    # two device buffer sets, so step i+1's copies run while step i computes;
+    # the candidates' q/k/v are gathered on the device from the copied tensors,
+    # and the decode output is read back into pinned host memory.
+    hcidx = torch.from_numpy(cidx).pin_memory()
+    hin = [torch.from_numpy(batch.q.view(np.int16)).pin_memory(),
+           torch.from_numpy(batch.k.view(np.int16)).pin_memory(),
+           torch.from_numpy(batch.v.view(np.int16)).pin_memory(),
+           torch.from_numpy(batch.cu_seqlens.astype(np.int32)).pin_memory(),
+           torch.from_numpy(past.astype(np.int32)).pin_memory(),
+           torch.from_numpy(batch.slot_ids.astype(np.int32)).pin_memory(),
+           torch.from_numpy(synth.cu_from_lens(cand)).pin_memory(),
+           hcidx]
     hout = torch.empty((Tc, H, D), dtype=torch.bfloat16).pin_memory()
-    h2d = [(hq, q.view(torch.int16)), (hk, k.view(torch.int16)), (hv, v.view(torch.int16)),
-           (hqc, qc.view(torch.int16)), (hkc, kc.view(torch.int16)), (hvc, vc.view(torch.int16)),
-           (hcu, cu), (hpl, pl), (hsl, sl), (hcuc, cu_c)]
-    h2d_bytes = sum(h.numel() * h.element_size() for h, _ in h2d)
+    sets = [[q.view(torch.int16), k.view(torch.int16), v.view(torch.int16), cu, pl, sl, cu_c,
+             torch.empty_like(hcidx, device=device)],
+            [torch.empty_like(h, device=device) for h in hin]]
+    h2d_bytes = sum(h.numel() * h.element_size() for h in hin)
     d2h_bytes = hout.numel() * hout.element_size()
-    e2e_steps = max(1, min(args.steps, 3))
+    e2e_steps = max(2, min(args.steps, 4))
+    copy_stream = torch.cuda.Stream(device)
+    ev_copied = [torch.cuda.Event() for _ in range(e2e_steps)]
+    ev_used = [torch.cuda.Event() for _ in range(e2e_steps)]
+
+    def e2e_step(i):
+        dq, dk, dv, dcu, dpl, dsl, dcuc, dcidx = sets[i % 2]
+        with torch.cuda.stream(copy_stream):
+            if i >= 2:
+                copy_stream.wait_event(ev_used[i - 2])     # step i-2 is done with this set
+            for h, d in zip(hin, sets[i % 2]):
+                d.copy_(h, non_blocking=True)
+            ev_copied[i].record(copy_stream)
+        stream.wait_event(ev_copied[i])
+        torch.index_select(dq, 0, dcidx, out=qc.view(torch.int16))
+        torch.index_select(dk, 0, dcidx, out=kc.view(torch.int16))
+        torch.index_select(dv, 0, dcidx, out=vc.view(torch.int16))
+        bq, bk, bv = dq.view(torch.bfloat16), dk.view(torch.bfloat16), dv.view(torch.bfloat16)
+        ub.masked_prefill_attn(bq, bk, bv, dcu, dpl, max_seqlen, out=out_p, out_fp32=False, workspace=ws_pre,
+                               pool_k=pool_k, pool_v=pool_v, slot_ids=dsl, layer=layer, dev_status=status,
+                               stream=stream)
+        ub.rank_decode_attn(qc, kc, vc, dcuc, dsl, dpl, pool_k, pool_v, layer, max_k, out=out_d, out_fp32=False,
+                            workspace=ws, dev_status=status, stream=stream)
+        hout.copy_(out_d, non_blocking=True)
+        ev_used[i].record(stream)
+
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(device)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        for h, d in h2d:
-            d.copy_(h, non_blocking=True)
-        step()
-        hout.copy_(out_d, non_blocking=True)
+    copy_stream.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %s in the end-to-end steps" % ub.status_string(int(status.item())))
+    del sets
 
     # ---------------------------------------------------------- max over ranks
-    ms_step = elapsed_ms / args.steps
-    pre_ms = sum(t_pre) / len(t_pre)
-    dec_ms = sum(t_dec) / len(t_dec)
-    pool_ms = sum(t_pool) / len(t_pool)
-    cand_total = float(cand.sum())
-    if dist is not None:
-        import torch.distributed as tdist
-        t = torch.tensor([ms_step, e2e_ms, pre_ms, dec_ms, pool_ms], dtype=torch.float64, device=device)
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        ms_step, e2e_ms, pre_ms, dec_ms, pool_ms = [float(x) for x in t.tolist()]
-        c = torch.tensor([cand_total], dtype=torch.float64, device=device)
-        tdist.all_reduce(c, op=tdist.ReduceOp.SUM)
-        cand_total = float(c.item())
+    times, counts = combine_rank_results(
+        {"step": elapsed_ms / args.steps, "e2e": e2e_ms, "prefill": sum(t_pre) / len(t_pre),
+         "decode": sum(t_dec) / len(t_dec)},
+        {"candidates": float(cand.sum())}, group=dist.group.WORLD if dist is not None else False, device=device)
+    ms_step, e2e_ms, pre_ms, dec_ms = (times[k] for k in ("step", "e2e", "prefill", "decode"))
+    cand_total = counts["candidates"]
 
     peaks = load_peaks()
     pf = prefill_flops(past, cand, H, D)
     df = decode_flops(past, cand, H, D)
     db = decode_bytes(past, cand, H, D, 2)
-    pwb = pool_write_bytes(past, H, D)
     pre_tflops = pf / (pre_ms * 1e-3) / 1e12
     dec_tflops = df / (dec_ms * 1e-3) / 1e12
     dec_gbs = db / (dec_ms * 1e-3) / 1e9
-    pool_gbs = pwb / (pool_ms * 1e-3) / 1e9
+    dec_roof = roof_entry(dec_ms, df, db, peaks, "decode")   # the decode's own binding roof
     # The prefill kernel runs for milliseconds inside a sub-second timed region at
     # full clock, so the burst GEMM figure is its denominator (the stricter one).
     peak = peaks["bf16_tflops"]
@@ -405,13 +425,12 @@ def run_ours(args, rank, world, device, dist):
                    "tokens_per_gpu": T, "candidates_per_gpu": Tc, "pool": [L, S, H, n_cap, D],
                    "layers_per_step": 1, "parallelism": "users sharded across %d GPU(s), no collective" % world,
                    "l2": "inputs larger than L2 (no flush)", "seed_rank0": seed},
-        "phases": {"pool_write_ms": pool_ms, "prefill_ms": pre_ms, "decode_ms": dec_ms,
+        "phases": {"prefill_ms": pre_ms, "decode_ms": dec_ms, "prefill_writes_pool": True,
                    "prefill_tflops": pre_tflops, "decode_tflops": dec_tflops, "decode_gbs": dec_gbs,
-                   "pool_write_gbs": pool_gbs,
                    "prefill_frac_tensor": pre_tflops / peak,
                    "prefill_frac_tensor_sustained": pre_tflops / peaks["bf16_tflops_sustained"],
                    "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
-                   "pool_write_frac_hbm": pool_gbs / peaks["hbm_gbs"]},
+                   "decode_bound": dec_roof["bound"], "decode_frac_roof": dec_roof["frac_roof"]},
         "roofline": {"kernel": "attn_fwd_kernel<128,prefill>", "bound": "tensor", "achieved": pre_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": pre_tflops / peak,
                      "traffic": prefill_traffic(T, H, D),
@@ -420,13 +439,136 @@ def run_ours(args, rank, world, device, dist):
                      "work_per_launch": "4*D*H*sum_b[n_b(n_b+1)/2 + k_b(n_b+1)] = %.4g FLOP" % pf},
         "e2e": {"value": cand_total / (e2e_ms * 1e-3), "unit": "candidate tokens/s",
                 "h2d_bytes_per_step": int(h2d_bytes), "d2h_bytes_per_step": int(d2h_bytes),
-                "steps": e2e_steps},
-        "gpu_launches": args.steps * (3 + (1 if decode_split else 0)),
+                "steps": e2e_steps,
+                "note": "inputs copied from pinned host memory on a second stream (double-buffered), "
+                        "candidate rows gathered on the device, decode output read back"},
+        "gpu_launches": args.steps * (2 + (1 if decode_split else 0)),
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_oracle_sample(batch, budget_s=args.cpu_budget)
+    if world == 1 and not args.no_sweep:
+        del q, k, v, qc, kc, vc, pool_k, pool_v, out_p, out_d, ws, ws_pre
+        torch.cuda.empty_cache()
+        result["sweep"] = run_sweep(device, peaks)
     return result
+
+
+def roof_entry(ms, flops, nbytes, peaks, kernel):
+    """Rates of one timed call and its fraction of the roof that binds it (tensor or HBM)."""
+    tflops = flops / (ms * 1e-3) / 1e12
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+    bound = "tensor" if t_tc >= t_hbm else "hbm"
+    return {"kernel": kernel, "ms": ms, "tflops": tflops, "gbs": gbs, "bound": bound,
+            "frac_tensor": tflops / peaks["bf16_tflops"], "frac_hbm": gbs / peaks["hbm_gbs"],
+            "frac_roof": (t_tc if bound == "tensor" else t_hbm) * 1e3 / ms}
+
+
+def run_sweep(device, peaks, iters=10, warm=3):
+    """The other workloads, one GPU: the D=64 prefills and the rank decode from the L=12 pool
+    at candidate counts 1..1000.  Inputs are N(0,1) bf16 drawn on the device from a seeded
+    generator; L2 is flushed (a 256 MB write) before every timed call; each entry is the
+    median over `iters` calls timed with CUDA events on the launching stream."""
+    import torch
+    from kv_cache_reuse_falcon_b200 import binding as ub
+
+    stream = torch.cuda.current_stream(device)
+    gen = torch.Generator(device=device)
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=device)
+
+    def randn(shape, seed):
+        gen.manual_seed(seed)
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(statistics.median(ts))
+
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    out = {}
+    for key, wname in (("prefill_B64_n256_k128_D64", "prefill_B64"),
+                       ("prefill_pool_B128_n1024_k512_D64", "prefill_pool_B128"),
+                       ("table2_B8_n992_k656_D64", "table2_B8")):
+        w = synth.workload(wname)
+        past = np.full(w.B, w.n, np.int32)
+        cand = np.full(w.B, w.k, np.int32)
+        T = int((past + cand).sum())
+        q, k, v = randn((T, w.H, w.D), w.seed), randn((T, w.H, w.D), w.seed + 1), randn((T, w.H, w.D), w.seed + 2)
+        cu = torch.from_numpy(synth.cu_from_lens(past + cand)).to(device)
+        pl = torch.from_numpy(past).to(device)
+        o = torch.empty((T, w.H, w.D), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(ub.masked_prefill_workspace_size() // 4 + 4, dtype=torch.float32, device=device)
+        kw = {}
+        nbytes = prefill_bytes(T, w.H, w.D, 2)
+        if w.L:
+            pk = torch.zeros((w.L, w.S, w.H, w.n_cap, w.D), dtype=torch.bfloat16, device=device)
+            pv = torch.zeros_like(pk)
+            gen.manual_seed(w.seed + 3)
+            slots = torch.randperm(w.S, generator=gen, device=device)[: w.B].to(torch.int32)
+            kw = dict(pool_k=pk, pool_v=pv, slot_ids=slots, layer=0)
+            nbytes += pool_write_bytes(past, w.H, w.D)
+
+        def fn():
+            ub.masked_prefill_attn(q, k, v, cu, pl, int(w.n + w.k), out=o, out_fp32=False, workspace=ws,
+                                   dev_status=status, stream=stream, **kw)
+
+        ms = timed(fn)
+        e = roof_entry(ms, prefill_flops(past, cand, w.H, w.D), nbytes, peaks,
+                       "attn_fwd_kernel<%d,prefill>%s" % (w.D, " (pool write fused)" if w.L else ""))
+        e["candidates_per_s"] = float(cand.sum()) / (ms * 1e-3)
+        out[key] = e
+        del q, k, v, o, kw
+        torch.cuda.empty_cache()
+
+    # rank decode from the [12, 256, 8, 2048, 64] pool, 32 requests, every layer per step
+    w = synth.workload("decode_R32")
+    pk = randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed)
+    pv = randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed + 1)
+    gen.manual_seed(w.seed + 2)
+    slots = torch.randperm(w.S, generator=gen, device=device)[: w.B].to(torch.int32)
+    past = np.full(w.B, w.n, np.int32)
+    pl = torch.from_numpy(past).to(device)
+    for kk in (1, 16, 64, 128, 256, 1000):
+        cand = np.full(w.B, kk, np.int32)
+        Tc = int(cand.sum())
+        cu = torch.from_numpy(synth.cu_from_lens(cand)).to(device)
+        qkv = [[randn((Tc, w.H, w.D), w.seed + 10 * l + j) for j in range(3)] for l in range(w.L)]
+        outs = [torch.empty((Tc, w.H, w.D), dtype=torch.bfloat16, device=device) for _ in range(w.L)]
+        nws = ub.rank_decode_workspace_size(w.B, w.H, w.D, kk, Tc, w.n_cap)
+        ws = torch.empty(nws // 4 + 4, dtype=torch.float32, device=device)
+
+        def fn():
+            for l in range(w.L):
+                ub.rank_decode_attn(qkv[l][0], qkv[l][1], qkv[l][2], cu, slots, pl, pk, pv, l, kk, out=outs[l],
+                                    out_fp32=False, workspace=ws, dev_status=status, stream=stream)
+
+        ms = timed(fn) / w.L
+        kernel = ("decode_smallk_kernel<%d,%d>" % (w.D, 16 if kk <= 16 else 32 if kk <= 32 else 64 if kk <= 64
+                                                     else 128)) if kk <= 128 else "attn_fwd_kernel<%d,decode>" % w.D
+        e = roof_entry(ms, decode_flops(past, cand, w.H, w.D), decode_bytes(past, cand, w.H, w.D, 2), peaks, kernel)
+        e["candidates_per_s"] = float(Tc) / (ms * 1e-3)
+        e["ms_per_12_layers"] = ms * w.L
+        out["decode_R32_n2048_D64_k%d" % kk] = e
+        del qkv, outs, ws
+    torch.cuda.synchronize(device)
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %s in the sweep" % ub.status_string(int(status.item())))
+    del pk, pv, flush
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_decode_only(args, rank, world, device, dist):
@@ -540,7 +682,8 @@ def run_decode_only(args, rank, world, device, dist):
         "phases": {"decode_tflops": tflops, "decode_gbs": gbs, "decode_frac_hbm": gbs / peaks["hbm_gbs"],
                    "decode_frac_tensor": tflops / peaks["bf16_tflops"],
                    "roof_time_ms": 1e3 * max(t_hbm, t_tc)},
-        "roofline": roof, "gpu_launches": args.steps * L * (2 if ws_bytes > 256 else 1), "clocks": clk,
+        "roofline": roof, "gpu_launches": args.steps * L * (2 if (ws_bytes > 256 and kk > 128) else 1),
+        "clocks": clk,
     }
 
 
@@ -583,6 +726,17 @@ def run_reference(args, rank, world):
     }
 
 
+def relaunch_command(argv, nproc, port=None):
+    """torchrun command that runs this script once per GPU (rendezvous on 127.0.0.1)."""
+    if port is None:
+        import socket
+        with socket.socket() as so:
+            so.bind(("127.0.0.1", 0))
+            port = so.getsockname()[1]
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", str(nproc),
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -596,13 +750,25 @@ def main(argv=None):
     ap.add_argument("--k", type=int, default=0, help="decode workloads: candidates per request")
     ap.add_argument("--layers", type=int, default=0,
                     help="decode workloads: pool layers and layer calls per step (smaller case)")
+    ap.add_argument("--no-sweep", action="store_true", help="headline workload only (no per-config sweep)")
     ap.add_argument("--graph", action="store_true",
                     help="decode workloads: replay each step's layer calls as one CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        if args.impl == "reference":
+            args.gpus = 1   # the oracle runs on rank 0's host cores only
+        else:
+            # one process per GPU: start the ranks with torch's launcher; rank 0 prints the line
+            return subprocess.call(relaunch_command(argv if argv is not None else sys.argv[1:], args.gpus))
+    world = int(world_env or "1")
+    if args.impl != "reference" and world != args.gpus:
+        ap.error("--gpus %d but the launcher started %d ranks (WORLD_SIZE)" % (args.gpus, world))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 

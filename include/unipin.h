@@ -81,6 +81,11 @@ typedef struct {
  *
  *   q, k, v        [T, H, D] bf16, T = total_tokens = cu_seqlens[B]
  *   out            [T, H, D], fp32 if out_fp32 != 0 else bf16 (round to nearest even)
+ *   lse            optional fp32 [T, H] (NULL: not written): per row and head the
+ *                  log-sum-exp of its scores in base-2 units,
+ *                  lse_i = log2(sum_j 2^(scale * log2(e) * q_i . k_j)) over the allowed
+ *                  keys j, so the weight of key j is 2^(scale*log2(e)*q_i.k_j - lse_i).
+ *                  The backward pass (unipin_masked_prefill_bwd) takes it.
  *   cu_seqlens     device int32 [B+1]; past_lens device int32 [B], 0 <= n_b <= len_b
  *   max_seqlen     host int >= every len_b (sizes the grid; a longer segment is a device error)
  *   scale          softmax scale, normally 1/sqrt(D)
@@ -95,7 +100,7 @@ typedef struct {
  *                  must not share a workspace.
  * Returns UNIPIN_OK or a negative unipin_status.
  */
-int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32,
+int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32, float* lse,
                                const int* cu_seqlens, const int* past_lens, int B, int H, int D,
                                int max_seqlen, int total_tokens, float scale, const unipin_kvpool* pool,
                                const int* slot_ids, int layer, void* workspace, size_t workspace_bytes,
@@ -104,6 +109,40 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
 /* Bytes of scratch that let unipin_masked_prefill_attn hand out work
  * dynamically (a work counter the call zeroes on `stream` before its kernel). */
 size_t unipin_masked_prefill_workspace_size(void);
+
+/*
+ * Gradients of the masked prefill ([review] §2.2: the joint objective trains
+ * [past || candidates] in one forward pass under this mask, so the backward
+ * pass runs over the same allowed pairs).  With P_ij the forward's weights
+ * (rebuilt from lse) and dO the gradient of the loss with respect to out:
+ *   dV_j = sum_i P_ij dO_i
+ *   dS_ij = P_ij (dO_i . v_j - dO_i . O_i)
+ *   dQ_i = scale * sum_j dS_ij k_j,   dK_j = scale * sum_i dS_ij q_i
+ * over allowed (i, j) only: a past key collects gradient from the later past
+ * rows and from every candidate row of its segment, a candidate's own key and
+ * value only from its own row.  Scores, probabilities and accumulation are
+ * fp32; P and dS are rounded to bf16 as tensor-core operands.
+ *   q, k, v        [T, H, D] bf16, the forward's inputs
+ *   out            [T, H, D] bf16, the forward's output (bf16 mode)
+ *   dout           [T, H, D] bf16, the gradient with respect to out
+ *   lse            fp32 [T, H] as written by unipin_masked_prefill_attn
+ *   dq, dk, dv     fp32 [T, H, D] outputs, written in full (dq is accumulated
+ *                  across key tiles with atomic adds, so its low bits depend on
+ *                  their order)
+ *   D              32 or 64 (UNIPIN_ERR_UNSUPPORTED otherwise)
+ *   workspace      device scratch of at least
+ *                  unipin_masked_prefill_bwd_workspace_size(total_tokens, H) bytes
+ *                  (the per-row dO . O), 16-byte aligned; not shared by overlapping calls
+ * Other arguments and errors as unipin_masked_prefill_attn.  Rows of a segment
+ * found out of range on the device get zero gradients.
+ */
+int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                              const float* lse, float* dq, float* dk, float* dv, const int* cu_seqlens,
+                              const int* past_lens, int B, int H, int D, int max_seqlen, int total_tokens,
+                              float scale, void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+
+/* Bytes of workspace unipin_masked_prefill_bwd needs: 4 * total_tokens * H, rounded up to 16. */
+size_t unipin_masked_prefill_bwd_workspace_size(int total_tokens, int H);
 
 /*
  * Pool write ([review] §2.4: retrieval writes the past K/V of every layer

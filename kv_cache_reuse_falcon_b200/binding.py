@@ -30,6 +30,8 @@ STATUS_NAMES = {
 
 EXPORTS = (
     "unipin_masked_prefill_attn",
+    "unipin_masked_prefill_bwd",
+    "unipin_masked_prefill_bwd_workspace_size",
     "unipin_kvpool_write",
     "unipin_rank_decode_attn",
     "unipin_rank_decode_workspace_size",
@@ -75,7 +77,11 @@ def _load(path: str = _LIB_PATH):
                           "python kv_cache_reuse_falcon_b200/build.py): %s" % path)
     lib = ctypes.CDLL(path)
     P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, I, I, I, I, I, F, P, P, I, P, SZ, P, P]
+    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, F, P, P, I, P, SZ, P, P]
+    lib.unipin_masked_prefill_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P, P]
+    lib.unipin_masked_prefill_bwd.restype = I
+    lib.unipin_masked_prefill_bwd_workspace_size.argtypes = [I, I]
+    lib.unipin_masked_prefill_bwd_workspace_size.restype = SZ
     lib.unipin_masked_prefill_workspace_size.argtypes = []
     lib.unipin_masked_prefill_workspace_size.restype = SZ
     lib.unipin_masked_prefill_attn.restype = I
@@ -175,8 +181,9 @@ def masked_prefill_workspace_size() -> int:
 
 def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=None, out_fp32: bool = True,
                         scale: Optional[float] = None, pool_k=None, pool_v=None, slot_ids=None, layer: int = 0,
-                        workspace="auto", dev_status=None, stream=None):
-    """M-FALCON masked prefill; optionally also writes the past K/V into pool slots."""
+                        workspace="auto", dev_status=None, stream=None, lse=None):
+    """M-FALCON masked prefill; optionally also writes the past K/V into pool slots and the per-row
+    log-sum-exp (base 2, fp32 [T, H]) into `lse`."""
     _tokens(q, "q")
     T, H, D = q.shape
     _tokens(k, "k", D)
@@ -192,15 +199,52 @@ def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=Non
     if pool_k is not None:
         pool = _pool(pool_k, pool_v)
         _index(slot_ids, "slot_ids", B)
+    if lse is not None and (lse.dtype != torch.float32 or lse.shape != (T, H) or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 tensor [T, H]")
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     ws, ws_bytes = _workspace(workspace, masked_prefill_workspace_size(), q.device)
-    rc = LIB.unipin_masked_prefill_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(bool(out_fp32)),
+    rc = LIB.unipin_masked_prefill_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(bool(out_fp32)), _ptr(lse),
                                         _ptr(cu_seqlens), _ptr(past_lens), B, H, D, int(max_seqlen), T, scale,
                                         ctypes.byref(pool) if pool is not None else None,
                                         _ptr(slot_ids) if pool is not None else None, int(layer),
                                         _ptr(ws), ws_bytes, _ptr(dev_status), _stream(stream))
     _check(rc, "unipin_masked_prefill_attn")
     return out
+
+
+def masked_prefill_bwd_workspace_size(total_tokens: int, H: int) -> int:
+    return int(LIB.unipin_masked_prefill_bwd_workspace_size(int(total_tokens), int(H)))
+
+
+def masked_prefill_bwd(q, k, v, out, dout, lse, cu_seqlens, past_lens, max_seqlen: int, scale: Optional[float] = None,
+                       dq=None, dk=None, dv=None, workspace="auto", dev_status=None, stream=None):
+    """Gradients (dq, dk, dv), fp32 [T, H, D], of the masked prefill for the upstream gradient dout.
+
+    `out` is the forward's bf16 output and `lse` the row statistic the forward wrote."""
+    _tokens(q, "q")
+    T, H, D = q.shape
+    for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _tokens(t, name, D)
+    if lse.dtype != torch.float32 or lse.shape != (T, H) or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous float32 tensor [T, H]")
+    B = past_lens.shape[0]
+    _index(cu_seqlens, "cu_seqlens", B + 1)
+    _index(past_lens, "past_lens", B)
+    grads = []
+    for g in (dq, dk, dv):
+        if g is None:
+            g = torch.empty((T, H, D), dtype=torch.float32, device=q.device)
+        elif g.dtype != torch.float32 or g.shape != q.shape or not g.is_contiguous():
+            raise ValueError("gradient outputs must be contiguous float32 [T, H, D]")
+        grads.append(g)
+    ws, ws_bytes = _workspace(workspace, masked_prefill_bwd_workspace_size(T, H), q.device)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    rc = LIB.unipin_masked_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                                       _ptr(grads[0]), _ptr(grads[1]), _ptr(grads[2]), _ptr(cu_seqlens),
+                                       _ptr(past_lens), B, H, D, int(max_seqlen), T, scale, _ptr(ws), ws_bytes,
+                                       _ptr(dev_status), _stream(stream))
+    _check(rc, "unipin_masked_prefill_bwd")
+    return tuple(grads)
 
 
 def kvpool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids, max_past: int,

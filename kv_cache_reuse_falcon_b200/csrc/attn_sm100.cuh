@@ -41,7 +41,11 @@
 //              "S read out" (which also says the next slot has landed) and
 //              "P stored": a wait issued right behind MMAs stalls the issuing
 //              warp until they drain, so the fewer the better.
-//   warp 11    idle (it completes the third warpgroup for the register split).
+//   warp 11    pool writer (prefill with a pool): each segment's last query-tile
+//              pair loads every past K/V tile of its head exactly once, and this
+//              warp copies those tiles from the ring into the segment's pool
+//              slot; it releases every ring use as the third arrival of the
+//              slot's empty barrier.
 // Every warp maps a global item index to its segment with the same
 // warp-cooperative walker (ItemWalker).
 //
@@ -65,18 +69,21 @@ constexpr int kThreads = 384;
 // the two softmax warpgroups take them (per head dim, in AttnCfg).
 constexpr int kLaunchRegs = 168;
 constexpr int kItemSlots = 4;        // items handed from the producer warp to the others
-constexpr int kItemConsumers = 10;   // the two MMA warps and the eight softmax warps
+constexpr int kItemConsumers = 11;   // the two MMA warps, the eight softmax warps, the pool writer
 constexpr int kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;   // rescale O only when a row max grows by > 2^8
 
-// Key tile width (keys per S tile) for head dim D.
-__host__ __device__ constexpr int key_tile_width(int D) { return D == 128 ? 64 : 128; }
+// Key tile width (keys per S tile).  The prefill takes 64 keys at every head
+// dim: a shorter softmax loop per tile (less code for the instruction cache,
+// finer pipelining); the rank decode through this engine (many candidates)
+// takes 128 keys at D <= 64, which halves its per-tile synchronisation.
+__host__ __device__ constexpr int key_tile_width(int D, bool decode) { return (D == 128 || !decode) ? 64 : 128; }
 
-template <int D>
+template <int D, bool kDecode>
 struct AttnCfg {
     static_assert(D == 32 || D == 64 || D == 128, "head dim");
-    static constexpr int kN = key_tile_width(D);                // keys per K/V tile
+    static constexpr int kN = key_tile_width(D, kDecode);       // keys per K/V tile
     static constexpr int kBoxD = D >= 64 ? 64 : D;              // elements per TMA box row
     static constexpr int kChunks = D / kBoxD;                   // boxes across D
     static constexpr int kRowBytes = kBoxD * 2;                 // 128 (SW128) or 64 (SW64)
@@ -126,6 +133,10 @@ struct AttnParams {
     int* status;
     unsigned long long wait_limit_ns;
     unsigned long long* sched;    // zeroed item counter (dynamic scheduling) or null (static striding)
+    float* lse;                   // [T, H] row statistic log2(sum_j 2^(s_ij * sl2)) or null (prefill)
+    int store_pool;               // prefill: also write the past K/V into slots[seg] of the pool
+    void* pool_k;                 // [L, S, H, n_cap, D] (prefill pool write)
+    void* pool_v;
 };
 
 // Key tile t of nt covering keys [0, kmax): tiles are kN wide from key 0;
@@ -208,6 +219,7 @@ struct ItemWalker {
 // Everything about one item that every role derives identically.
 struct Work {
     bool valid;
+    bool store;                 // prefill: this item writes the segment's past K/V tiles to the pool
     bool rows_ok;               // the segment's rows lie inside the token tensors
     int seg, h, split;
     int tok0, npast, slot;
@@ -233,7 +245,7 @@ __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int loca
     w.tok0 = p.cu[seg];
     const int nrows_seg = p.cu[seg + 1] - w.tok0;
     w.npast = p.past[seg];
-    w.slot = kDecode ? p.slots[seg] : 0;
+    w.slot = (kDecode || p.store_pool) ? p.slots[seg] : 0;
     w.rows_ok = w.tok0 >= 0 && nrows_seg >= 0 && (long long)w.tok0 + nrows_seg <= (long long)p.total_rows;
     bool bad = !w.rows_ok || w.npast < 0;
     if (kDecode)
@@ -268,15 +280,19 @@ __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int loca
     w.nt_b = w.has_b ? max(t_end_b - w.t_begin, 0) : 0;
     w.nt = w.valid ? max(w.nt_a, w.nt_b) : 0;
     if (!w.valid) w.nt_a = w.nt_b = 0;
+    // The segment's last pair sees every past key (kmax = npast) and is its first item.
+    w.store = !kDecode && p.store_pool && w.valid && pair_rank == 0 && w.slot >= 0 && w.slot < p.S &&
+              w.npast <= p.n_cap;
     return w;
 }
 
 template <int D, bool kDecode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p)
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_pk,
+                    const __grid_constant__ CUtensorMap tm_pv, const AttnParams p)
 {
-    using C = AttnCfg<D>;
+    using C = AttnCfg<D, kDecode>;
     constexpr int NS = C::kStages;
     extern __shared__ __align__(1024) uint8_t smem[];
 
@@ -325,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < NS; ++s) {
             mbar_init(kv_full + s, 1);
-            mbar_init(kv_empty + s, 2);   // one arrival from each MMA warp
+            mbar_init(kv_empty + s, 3);   // each MMA warp and the pool writer
         }
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -461,6 +477,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int v = (u > NS ? u - NS : 0); v < u; ++v)
                 mbar_wait_drain(kv_empty + v % NS, (v / NS) & 1, p.wait_limit_ns);
         }
+    } else if (warp == 11) {
+        // ----------------------------------------------------- pool writer
+        if (p.store_pool && leader) {
+            tma_prefetch_map(&tm_pk);
+            tma_prefetch_map(&tm_pv);
+        }
+        int u = 0;
+        bool ok = true;
+        while (pop_item(ok)) {
+            const Work w = make_work<kDecode, C::kN>(p, seg, local);
+            if (!kDecode && p.store_pool && w.valid && (local / p.H) == 0 && !w.store && leader)
+                report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);   // slot id or history length beyond the pool
+            const int plane = (p.layer * p.S + w.slot) * p.H + w.h;
+            for (int i = 0; i < w.nt; ++i, ++u) {
+                const int st = u % NS;
+                ok = __all_sync(0xffffffffu, mbar_wait(kv_full + st, (u / NS) & 1, ctl));
+                if (!ok) break;
+                if (w.store) {
+                    int start, lo;
+                    key_tile<C::kN>(w.t_begin + i, w.nt_all, w.kmax, start, lo);
+                    const uint8_t* src[2] = {ring + st * C::kSlotBytes, ring + st * C::kSlotBytes + C::kTileKV};
+                    if (start >= 0) {
+                        // the whole tile is rows start .. start+kN-1 of the slot (all below npast)
+                        if (leader) {
+                            for (int c = 0; c < C::kChunks; ++c) {
+                                tma_store_3d(&tm_pk, src[0] + c * C::kAtomKV, c * C::kBoxD, start, plane);
+                                tma_store_3d(&tm_pv, src[1] + c * C::kAtomKV, c * C::kBoxD, start, plane);
+                            }
+                            bulk_commit_group();
+                            bulk_wait_read_all();
+                        }
+                    } else {
+                        // a history shorter than one tile: rows 0 .. kmax-1 sit at tile rows
+                        // -start .. kN-1; un-swizzle them with plain 16-byte copies
+                        constexpr int kVecs = C::kRowBytes / 16;
+                        const int units = w.kmax * C::kChunks * kVecs;
+                        for (int x = lane; x < units; x += 32) {
+                            const int j = x % kVecs;
+                            const int c = (x / kVecs) % C::kChunks;
+                            const int rr = x / (kVecs * C::kChunks);
+                            const int sr = rr - start;
+                            const int sw = C::kRowBytes == 128 ? (sr & 7) : ((sr >> 1) & 3);
+                            const size_t dst = (((size_t)plane * p.n_cap + rr) * (D * 2)) + c * C::kRowBytes + j * 16;
+                            const int so = c * C::kAtomKV + sr * C::kRowBytes + ((j ^ sw) << 4);
+                            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.pool_k) + dst) =
+                                *reinterpret_cast<const uint4*>(src[0] + so);
+                            *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.pool_v) + dst) =
+                                *reinterpret_cast<const uint4*>(src[1] + so);
+                        }
+                    }
+                }
+                __syncwarp();
+                if (leader) mbar_arrive(kv_empty + st);
+            }
+            if (!ok) break;
+        }
+        if (leader) bulk_wait_all();   // every pool store has landed before the block exits
     } else if (warp == 9 || warp == 10) {
         // ------------------------------------------------- UMMA issuers
         // Warp 9 issues the MMAs of tile A, warp 10 those of tile B.  Per key
@@ -789,6 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 b = self ? ex2_approx(ss - m_fin) : 0.f;
                 const float denom = l * a + b;
                 inv = denom > 0.f ? 1.f / denom : 0.f;
+                if (!kDecode && p.lse) p.lse[(size_t)tok * p.H + w.h] = m_fin + log2f(denom);
             }
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {

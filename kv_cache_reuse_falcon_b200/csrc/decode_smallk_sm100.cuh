@@ -8,18 +8,20 @@
 // dimension, so no tensor-core row and no softmax thread is spent on padding
 // candidates:
 //
-//   S^T = K Q^T     M = 128 keys, N = k padded to 16/32/64/128, K = D
-//   O^T += V^T P^T  M = 128 (head-dim rows d; at D = 64 the upper 64 rows are
-//                   discarded), N = padded candidates (at least 64), K = 128 keys
+//   S^T = K Q^T   M = 128 keys, N = k padded to 16/32/64/128, K = D
+//   O  += P V     M = 128 candidate rows (rows past the padded count are
+//                 discarded), N = D, K = 128 keys; P (bf16) is staged through
+//                 shared memory in the 128-byte-swizzled K-major layout of a
+//                 query tile, V is read MN-major as the prefill reads it
 //
 // Softmax thread t owns key t of a tile (TMEM lane t): it loads that key's N
 // scores, and the per-candidate statistics are reductions over threads.  The
 // reference maximum of each candidate moves only when some score would
 // exceed it by more than 2^8 (one vote per tile among the four softmax warps;
 // the exact column maxima are computed only then), so the common tile costs
-// N scalings, N exponentials and one warp reduce-scatter of the column sums.
-// P^T is written to shared memory in the same 128-byte-swizzled, key-major
-// layout a V tile has, and O^T accumulates in TMEM.
+// N scalings, N exponentials, N two-byte stores of P and one warp
+// reduce-scatter of the column sums.  O accumulates in TMEM with lane =
+// candidate, so the epilogue thread of candidate c reads its own row.
 //
 // Work item = (request, head, key split).  The key range of a request is cut
 // into `nsplit` runs of whole 128-key tiles so that every SM has several
@@ -31,8 +33,8 @@
 //
 // Warp roles (192 threads, two blocks per SM where shared memory and TMEM
 // allow, so one block's per-item latencies hide behind the other's stream):
-//   warps 0-3  softmax and epilogue (thread t: key t of a tile; head-dim row
-//              t of O^T in the epilogue)
+//   warps 0-3  softmax and epilogue (thread t: key t of a tile; candidate t's
+//              output row in the epilogue)
 //   warp 4     TMA producer: claims items, loads Q (N candidate rows) and the
 //              V and K tiles of each key tile into a ring of stages
 //   warp 5     MMA issuer (one elected thread), owns TMEM
@@ -67,15 +69,18 @@ struct SkCfg {
     static constexpr int kStageBytes = 2 * kTileKV;        // V tile, then K tile
     static constexpr int kAtomQ = N * 128;                 // N candidate rows of one 64-element box
     static constexpr int kQBytes = kChunks * kAtomQ;
-    static constexpr int kNpv = N < 64 ? 64 : N;           // candidate columns of the P.V MMA
-    static constexpr int kPBytes = (kNpv / 64) * kAtom;    // P^T: 128 keys x kNpv candidates, bf16
-    // TMEM columns: S^T buffers at 0 and N, O^T at 2N.
+    // P: N candidate rows x 128 keys bf16, two 64-key boxes of N rows x 128 bytes.
+    // The P.V MMA reads 128 rows from each box base; rows N..127 fall on
+    // whatever follows in shared memory and give discarded output rows.
+    static constexpr int kPBox = N * 128;
+    static constexpr int kPBytes = 2 * kPBox;
+    // TMEM columns: S^T buffers at 0 and N, O (D columns) at 2N.
     static constexpr int kColO = 2 * N;
-    static constexpr int kTmemCols = sk_tmem_cols(2 * N + kNpv);
+    static constexpr int kTmemCols = sk_tmem_cols(2 * N + D);
     static constexpr int kCtasPerSm = (D == 64 && kTmemCols <= 256) ? 2 : 1;
-    // Scratch floats: red[4][N], mref[N], corr[N], coef_a[N], coef_b[N], self[N],
-    // flags[2][4], lfin[N]; merge weights reuse a P buffer.
-    static constexpr int kScratchBytes = ((4 * N + 6 * N + 8) * 4 + 1023) / 1024 * 1024;
+    // Scratch floats: red[4][N], mref[N], corr[N], coef_b[N], flags[2][4]; merge
+    // weights reuse a P buffer.
+    static constexpr int kScratchBytes = ((4 * N + 3 * N + 8) * 4 + 1023) / 1024 * 1024;
     static constexpr int kBarBytes = 1024;
     static constexpr int kBudget = kCtasPerSm == 2 ? 112 * 1024 : 226 * 1024;
     // Double-buffer Q (the next item's Q loads during this item) and P^T (the
@@ -91,14 +96,15 @@ struct SkCfg {
     static constexpr int kStagesFit = (kBudget - fixed_bytes(kQBufs, kPBufs)) / kStageBytes;
     static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
     static_assert(kStages >= 2, "small-k decode: ring depth");
-    static constexpr int kOffRing = 0;
-    static constexpr int kOffQ = kStages * kStageBytes;
-    static constexpr int kOffP = kOffQ + kQBufs * kQBytes;
-    static constexpr int kOffScratch = kOffP + kPBufs * kPBytes;
+    static constexpr int kOffP = 0;                                  // first: the 128-row reads overhang
+    static constexpr int kOffRing = kPBufs * kPBytes;                // into the ring that follows
+    static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
+    static constexpr int kOffScratch = kOffQ + kQBufs * kQBytes;
     static constexpr int kOffBar = kOffScratch + kScratchBytes;
     static constexpr int kSmemBytes = kOffBar + kBarBytes;
     static_assert(kSmemBytes <= kBudget, "small-k decode: shared memory budget");
     static_assert(kSkMaxSplit * N * 4 <= kPBytes, "merge weights fit a P buffer");
+    static_assert((kPBufs - 1) * kPBytes + kPBox + kSkKeys * 128 <= kSmemBytes, "P box reads stay in shared memory");
 };
 
 struct SkParams {
@@ -203,17 +209,6 @@ __device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t (&r)[N])
     else tmem_ld128(taddr, r);
 }
 
-// Bounded barrier of the four softmax warps (an mbarrier with arrival count
-// 4): unlike bar.sync it gives up when the block aborts.
-__device__ __forceinline__ bool sk_group_sync(uint64_t* bar, uint32_t& n, const WaitCtl& ctl, int lane)
-{
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bar);
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, n & 1, ctl));
-    ++n;
-    return ok;
-}
-
 // q . k of one head row (D bf16 each), all loads issued before the sums.
 template <int D>
 __device__ __forceinline__ float sk_dot_bf16(const __nv_bfloat16* a, const __nv_bfloat16* b)
@@ -252,14 +247,6 @@ __device__ __forceinline__ void sk_store4(void* out, int out_fp32, size_t idx, f
             make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
 }
 
-__device__ __forceinline__ void sk_store_out(void* out, int out_fp32, size_t idx, float val)
-{
-    if (out_fp32)
-        reinterpret_cast<float*>(out)[idx] = val;
-    else
-        reinterpret_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(val);
-}
-
 template <int D, int N>
 __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     decode_smallk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -284,11 +271,8 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     float* red = reinterpret_cast<float*>(smem + C::kOffScratch);   // [4][N]
     float* mref = red + 4 * N;                                      // [N] reference max (log2 units)
     float* corr = mref + N;                                         // [N]
-    float* coef_a = corr + N;                                       // [N]
-    float* coef_b = coef_a + N;                                     // [N]
-    float* selfs = coef_b + N;                                      // [N] self score (log2 units)
-    float* lfin = selfs + N;                                        // [N]
-    volatile int* flags = reinterpret_cast<volatile int*>(lfin + N);   // [2][4]
+    float* coef_b = corr + N;                                       // [N] merge: weight of the own value
+    volatile int* flags = reinterpret_cast<volatile int*>(coef_b + N);   // [2][4]
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_q = bars + 0;            // [2] Q buffer landed
     uint64_t* q_empty = bars + 2;          // [2] the last S MMA of the item using Q buffer b finished
@@ -441,16 +425,16 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         // the softmax has written P_{i-1}; so S_{i+1} is computed while the
         // softmax works on S_i.
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kSkKeys, N, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::kNpv, true, true);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true, false);
         const uint32_t ring_a = smem_u32(ring);
         // K (A of S^T): K-major, 128-byte rows, 8-row groups 1024 bytes apart.
         const uint64_t dk0 = smem_desc(ring_a + C::kTileKV, 16, 1024, kLayoutSw128);
-        // V (A of O^T, MN-major): 64-element head-dim blocks 16 KB apart (at
-        // D = 64 the second block is the stage's K tile: rows 64-127 of O^T
-        // are not used), 8-key groups 1024 bytes apart.
+        // V (B of O += P V, MN-major): 64-element head-dim blocks 16 KB apart,
+        // 8-key groups 1024 bytes apart.
         const uint64_t dv0 = smem_desc(ring_a, C::kAtom, 1024, kLayoutSw128);
         const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, 1024, kLayoutSw128);
-        const uint64_t dp0 = smem_desc(smem_u32(sP), C::kAtom, 1024, kLayoutSw128);
+        // P (A of O += P V): K-major rows of 64 keys per box, 8-row groups 1024 bytes apart.
+        const uint64_t dp0 = smem_desc(smem_u32(sP), 16, 1024, kLayoutSw128);
         const uint32_t tO = tmem + C::kColO;
         int u = 0, nq = 0;
         int gs = 0;            // S tiles issued
@@ -459,10 +443,11 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         bool ok = true;
         long long g;
         auto issue_pv = [&](int st, int pb, bool acc) {
+            // K-steps of 16 keys: 32 bytes within a P row (then the second box), 16 V rows
 #pragma unroll
             for (int kk = 0; kk < kSkKeys / 16; ++kk) {
-                const uint64_t a = dv0 + (uint64_t)((st * C::kStageBytes + kk * 2048) >> 4);
-                const uint64_t b = dp0 + (uint64_t)((pb * C::kPBytes + kk * 2048) >> 4);
+                const uint64_t a = dp0 + (uint64_t)((pb * C::kPBytes + (kk / 4) * C::kPBox + (kk % 4) * 32) >> 4);
+                const uint64_t b = dv0 + (uint64_t)((st * C::kStageBytes + kk * 2048) >> 4);
                 umma_bf16_ss(tO, a, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
             }
             umma_commit(pv_done + pb);
@@ -487,32 +472,58 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             if (!ok) break;
             ++nq;
             for (int i = 0; ok && i < w.nt; ++i) {
+                // S_i needs K_i landed and an S buffer the softmax has read out; P.V of
+                // tile i-1 needs P_{i-1}.  Issue each as soon as its inputs are there: a
+                // P.V queued behind the next tile's data would hold its ring stage, and
+                // the ring would then have a single load in flight.
                 const int st = (u + i) % NS;
-                ok = __all_sync(0xffffffffu, mbar_wait(kv_full + st, ((u + i) / NS) & 1, ctl));
-                if (!ok) break;
                 const int sb = gs & 1;
-                if (gs >= 2) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(s_free + sb, ((gs >> 1) - 1) & 1, ctl));
-                    if (!ok) break;
-                }
-                tc_fence_after_sync();
-                if (leader) {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const int box = kk / 4;
-                        const int in_row = (kk % 4) * 32;
-                        const uint64_t a = dk0 + (uint64_t)((st * C::kStageBytes + box * C::kAtom + in_row) >> 4);
-                        const uint64_t b = dq0 + (uint64_t)((qb * C::kQBytes + box * C::kAtomQ + in_row) >> 4);
-                        umma_bf16_ss(tmem + sb * N, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                bool need_qk = true;
+                bool need_pv = i >= 1;
+                const uint64_t t0 = global_timer_ns();
+                for (uint32_t spin = 1; need_qk || need_pv; ++spin) {
+                    if (need_pv) {
+                        const int pb = gp % NP;
+                        if (__all_sync(0xffffffffu, mbar_test_wait(p_full + pb, pfull_seen[pb] & 1))) {
+                            ++pfull_seen[pb];
+                            tc_fence_after_sync();
+                            if (leader) issue_pv((u + i - 1) % NS, pb, i - 1 > 0);
+                            ++gp;
+                            need_pv = false;
+                        }
                     }
-                    umma_commit(s_full + sb);
-                    if (i == w.nt - 1) umma_commit(q_empty + qb);
-                }
-                ++gs;
-                if (i >= 1) {
-                    if (!(ok = wait_p(gp))) break;
-                    if (leader) issue_pv((u + i - 1) % NS, gp % NP, i - 1 > 0);
-                    ++gp;
+                    if (need_qk && __all_sync(0xffffffffu, mbar_test_wait(kv_full + st, ((u + i) / NS) & 1) &&
+                                                              (gs < 2 || mbar_test_wait(s_free + sb, ((gs >> 1) - 1) & 1)))) {
+                        tc_fence_after_sync();
+                        if (leader) {
+#pragma unroll
+                            for (int kk = 0; kk < D / 16; ++kk) {
+                                const int box = kk / 4;
+                                const int in_row = (kk % 4) * 32;
+                                const uint64_t a =
+                                    dk0 + (uint64_t)((st * C::kStageBytes + box * C::kAtom + in_row) >> 4);
+                                const uint64_t b = dq0 + (uint64_t)((qb * C::kQBytes + box * C::kAtomQ + in_row) >> 4);
+                                umma_bf16_ss(tmem + sb * N, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                            }
+                            umma_commit(s_full + sb);
+                            if (i == w.nt - 1) umma_commit(q_empty + qb);
+                        }
+                        ++gs;
+                        need_qk = false;
+                    }
+                    if ((spin & 31) == 0) {
+                        // warp-uniform: every lane leaves the loop together
+                        const bool aborted = *abort_flag != 0;
+                        const bool stop = __any_sync(0xffffffffu, aborted || global_timer_ns() - t0 > p.wait_limit_ns);
+                        if (stop) {
+                            if (leader && !aborted) {
+                                *abort_flag = 1;
+                                report(p.status, (int)UNIPIN_ERR_DEVICE_TIMEOUT);
+                            }
+                            ok = false;
+                            break;
+                        }
+                    }
                 }
             }
             if (!ok) break;
@@ -527,7 +538,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         }
     } else {
         // ------------------------------------------------- softmax + epilogue
-        const int t = threadIdx.x;                               // key of a tile / head-dim row of O^T
+        const int t = threadIdx.x;                               // key of a tile / candidate row of O
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const float sl2 = p.sl2;
         int gs = 0, gp = 0;
@@ -556,6 +567,11 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 continue;
             }
             if (!w.valid && t == 0 && w.split == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
+            // Candidate t's own score (log2 units), taken while the item's first tile is in flight.
+            float ss_own = -INFINITY;
+            if (t < w.kc && w.valid)
+                ss_own = sl2 * sk_dot_bf16<D>(p.q + ((size_t)(w.tok0 + t) * p.H + w.h) * D,
+                                              p.k_self + ((size_t)(w.tok0 + t) * p.H + w.h) * D);
             // per-thread partial column sums of P (owned columns), relative to mref
             constexpr int kOwn = N >= 32 ? N / 32 : 1;
             float lown[kOwn];
@@ -594,7 +610,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 const int fb = ngrp & 1;
                 const int warp_need = __any_sync(0xffffffffu, need) ? 1 : 0;
                 if (lane == 0) flags[fb * 4 + warp] = warp_need;
-                if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+                if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
                 const bool any_need = (flags[fb * 4 + 0] | flags[fb * 4 + 1] | flags[fb * 4 + 2] | flags[fb * 4 + 3]) != 0;
                 if (any_need) {
                     // exact column maxima of this tile; move every reference max to it
@@ -605,7 +621,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 #pragma unroll
                     for (int e = 0; e < kOwn; ++e)
                         if (N >= 32 || (lane & 1) == 0) red[warp * N + sk_owned_col<N>(lane, e)] = cm[e];
-                    if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+                    if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
                     if (t < N) {
                         const float mt = fmaxf(fmaxf(red[t], red[N + t]), fmaxf(red[2 * N + t], red[3 * N + t]));
                         const float mo = mref[t];
@@ -613,27 +629,26 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                         corr[t] = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mn);
                         mref[t] = mn;
                     }
-                    if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+                    if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
 #pragma unroll
                     for (int e = 0; e < kOwn; ++e) lown[e] *= corr[sk_owned_col<N>(lane, e)];
                     if (i > 0) {
-                        // rescale the columns of O^T accumulated so far (after the last P.V)
+                        // rescale the O rows accumulated so far (after the last P.V): row c is candidate c
                         if (!(ok = wait_pv(gp - 1))) break;
-                        if (warp * 32 < D) {
+                        if (warp * 32 < N) {
+                            const float cf = corr[t < N ? t : 0];
 #pragma unroll
-                            for (int c0 = 0; c0 < N; c0 += 16) {
+                            for (int c0 = 0; c0 < D; c0 += 16) {
                                 uint32_t o[16];
                                 tmem_ld16(lane_base + C::kColO + c0, o);
 #pragma unroll
-                                for (int e = 0; e < 16; ++e)
-                                    o[e] = __float_as_uint(__uint_as_float(o[e]) * corr[c0 + e]);
+                                for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * cf);
                                 tmem_st16(lane_base + C::kColO + c0, o);
                             }
                         }
                     }
                 }
-                // P = 2^(x - m), packed to bf16 pairs
-                uint32_t pk[N / 2];
+                // P = 2^(x - m)
                 float ps[N];
 #pragma unroll
                 for (int c = 0; c < N; c += 4) {
@@ -644,17 +659,18 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                         const float mu = mm[e] == -INFINITY ? 0.f : mm[e];
                         ps[c + e] = ex2_approx(x[c + e] - mu);
                     }
-                    pk[c / 2] = pack_bf16x2(ps[c], ps[c + 1]);
-                    pk[c / 2 + 1] = pack_bf16x2(ps[c + 2], ps[c + 3]);
                 }
                 // the P buffer is free once the P.V that last read it has finished
                 const int pb = gp % NP;
                 if (!(ok = wait_pv(gp - NP))) break;
-                uint8_t* prow = sP + pb * C::kPBytes + t * 128;
+                // column t of P: key t of the tile is element t % 64 of a 128-byte row of box t / 64
+                {
+                    uint8_t* pbox = sP + pb * C::kPBytes + (t / 64) * C::kPBox;
+                    const int kx = t % 64;
 #pragma unroll
-                for (int j = 0; j < N / 8; ++j) {
-                    uint4 v4 = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-                    *reinterpret_cast<uint4*>(prow + (j / 8) * C::kAtom + (((j % 8) ^ (t % 8)) << 4)) = v4;
+                    for (int c = 0; c < N; ++c)
+                        *reinterpret_cast<__nv_bfloat16*>(pbox + c * 128 + ((((kx >> 3) ^ (c & 7))) << 4) +
+                                                          (kx & 7) * 2) = __float2bfloat16_rn(ps[c]);
                 }
                 fence_proxy_async_smem();
                 tc_fence_before_sync();
@@ -671,77 +687,78 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 #pragma unroll
             for (int e = 0; e < kOwn; ++e)
                 if (N >= 32 || (lane & 1) == 0) red[warp * N + sk_owned_col<N>(lane, e)] = lown[e];
-            if (t < w.kc && p.nsplit == 1 && w.valid)
-                selfs[t] = sl2 * sk_dot_bf16<D>(p.q + ((size_t)(w.tok0 + t) * p.H + w.h) * D,
-                                                p.k_self + ((size_t)(w.tok0 + t) * p.H + w.h) * D);
-            if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+            if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
+            // thread t < N: candidate t's sum, max and output coefficients
+            float m_c = -INFINITY, l_c = 0.f, ca = 0.f, cb = 0.f;
             if (t < N) {
-                const float l = red[t] + red[N + t] + red[2 * N + t] + red[3 * N + t];
-                const float m = w.nt > 0 ? mref[t] : -INFINITY;
-                lfin[t] = l;
-                coef_a[t] = m;   // the partial's max, before mref is reset below
-                if (p.nsplit == 1 && t < w.kc) {
-                    // final: (a O + b v_self) / (a l + b)
-                    const float ss = selfs[t];
-                    const float mf = fmaxf(m, ss);
-                    const float a = (m == -INFINITY) ? 0.f : ex2_approx(m - mf);
-                    const float b = ex2_approx(ss - mf);
-                    const float inv = 1.f / (l * a + b);
-                    coef_a[t] = w.valid ? a * inv : 0.f;
-                    coef_b[t] = w.valid ? b * inv : 0.f;
-                }
+                l_c = red[t] + red[N + t] + red[2 * N + t] + red[3 * N + t];
+                m_c = w.nt > 0 ? mref[t] : -INFINITY;
                 mref[t] = -INFINITY;   // ready for the next item
+                if (p.nsplit == 1 && t < w.kc && w.valid) {
+                    // final: (a O + b v_self) / (a l + b)
+                    const float mf = fmaxf(m_c, ss_own);
+                    const float a = (m_c == -INFINITY) ? 0.f : ex2_approx(m_c - mf);
+                    const float b = ex2_approx(ss_own - mf);
+                    const float inv = 1.f / (l_c * a + b);
+                    ca = a * inv;
+                    cb = b * inv;
+                }
             }
-            if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
-            // O^T row t (head-dim element d = t) for every candidate column
-            uint32_t o[N];
-            if (w.nt > 0 && warp * 32 < D) {
-                tmem_ld_n<N>(lane_base + C::kColO, o);
+            // O row t = candidate t (warp-collective load where the warp holds candidate rows)
+            uint32_t o[D];
+            if (w.nt > 0 && warp * 32 < N) {
+                if constexpr (D == 64) tmem_ld64(lane_base + C::kColO, o);
+                else tmem_ld128(lane_base + C::kColO, o);
             } else {
 #pragma unroll
-                for (int c = 0; c < N; ++c) o[c] = 0u;
+                for (int d = 0; d < D; ++d) o[d] = 0u;
             }
             tc_fence_before_sync();
-            if (t < D) {
+            if (t < w.kc) {
+                const size_t row = (size_t)(w.tok0 + t) * p.H + w.h;
                 if (p.nsplit == 1) {
+                    const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + row * D);
 #pragma unroll
-                    for (int c = 0; c < N; ++c) {
-                        if (c < w.kc) {
-                            const size_t idx = ((size_t)(w.tok0 + c) * p.H + w.h) * D + t;
-                            const float vs = __bfloat162float(p.v_self[idx]);
-                            sk_store_out(p.out, p.out_fp32, idx, __uint_as_float(o[c]) * coef_a[c] + coef_b[c] * vs);
+                    for (int d8 = 0; d8 < D / 8; ++d8) {
+                        const uint4 vb = __ldg(v4 + d8);
+                        const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vb);
+                        float r[8];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 vf = __bfloat1622float2(vh[e]);
+                            r[2 * e] = __uint_as_float(o[d8 * 8 + 2 * e]) * ca + cb * vf.x;
+                            r[2 * e + 1] = __uint_as_float(o[d8 * 8 + 2 * e + 1]) * ca + cb * vf.y;
                         }
+                        sk_store4(p.out, p.out_fp32, row * D + d8 * 8, make_float4(r[0], r[1], r[2], r[3]));
+                        sk_store4(p.out, p.out_fp32, row * D + d8 * 8 + 4, make_float4(r[4], r[5], r[6], r[7]));
                     }
                 } else {
+                    float* po = p.part_o + ((size_t)w.split * p.total_rows * p.H + row) * D;
 #pragma unroll
-                    for (int c = 0; c < N; ++c) {
-                        if (c < w.kc)
-                            p.part_o[(((size_t)w.split * p.total_rows + w.tok0 + c) * p.H + w.h) * D + t] =
-                                __uint_as_float(o[c]);
-                    }
+                    for (int d = 0; d < D; d += 4)
+                        *reinterpret_cast<float4*>(po + d) =
+                            make_float4(__uint_as_float(o[d]), __uint_as_float(o[d + 1]), __uint_as_float(o[d + 2]),
+                                        __uint_as_float(o[d + 3]));
+                    float* ml = p.part_ml + ((size_t)w.split * p.total_rows * p.H + row) * 2;
+                    ml[0] = w.valid ? m_c : -INFINITY;
+                    ml[1] = w.valid ? l_c : 0.f;
                 }
             }
             if (p.nsplit > 1) {
-                if (t < w.kc) {
-                    float* ml = p.part_ml + (((size_t)w.split * p.total_rows + w.tok0 + t) * p.H + w.h) * 2;
-                    ml[0] = w.valid ? coef_a[t] : -INFINITY;
-                    ml[1] = w.valid ? lfin[t] : 0.f;
-                }
                 // publish the partial; the last split of this (request, head) to arrive merges
                 __threadfence();
-                if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+                if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
                 if (t == 0) {
                     const unsigned prev = atomicAdd(p.pair_cnt + w.pair, 1u);
                     *last_flag = prev == (unsigned)(p.nsplit - 1);
                 }
-                if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+                if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
                 if (*last_flag) {
                     __threadfence();
                     float* wts = reinterpret_cast<float*>(sP + (gp % NP) * C::kPBytes);   // [kSkMaxSplit][N]
                     if (t < w.kc) {
                         // weights of the splits and of the own key: LSE merge in log2 units
                         const size_t row = (size_t)(w.tok0 + t) * p.H + w.h;
-                        const float ss = sl2 * sk_dot_bf16<D>(p.q + row * D, p.k_self + row * D);
                         float ms[kSkMaxSplit], ls[kSkMaxSplit];
 #pragma unroll
                         for (int s = 0; s < kSkMaxSplit; ++s) {
@@ -752,10 +769,10 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                             ms[s] = ml.x;
                             ls[s] = ml.y;
                         }
-                        float mf = ss;
+                        float mf = ss_own;
 #pragma unroll
                         for (int s = 0; s < kSkMaxSplit; ++s) mf = fmaxf(mf, ms[s]);
-                        const float b = ex2_approx(ss - mf);
+                        const float b = ex2_approx(ss_own - mf);
                         float den = b;
                         float a[kSkMaxSplit];
 #pragma unroll
@@ -763,13 +780,14 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                             a[s] = (ms[s] == -INFINITY || !(ls[s] > 0.f)) ? 0.f : ex2_approx(ms[s] - mf);
                             den = fmaf(a[s], ls[s], den);
                         }
+                        // a rejected request (no own score: every term -inf) gets zero weights
                         const float inv = w.valid ? 1.f / den : 0.f;
 #pragma unroll
                         for (int s = 0; s < kSkMaxSplit; ++s)
-                            if (s < p.nsplit) wts[s * N + t] = a[s] * inv;
-                        coef_b[t] = b * inv;
+                            if (s < p.nsplit) wts[s * N + t] = w.valid ? a[s] * inv : 0.f;
+                        coef_b[t] = w.valid ? b * inv : 0.f;
                     }
-                    if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+                    if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
                     // out = b v_self + sum_s w_s O_s, four head-dim elements per thread and step;
                     // four steps' loads are issued before their sums
                     constexpr int kQ = D / 4;
@@ -791,8 +809,8 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                                 const uint2 vb = __ldg(reinterpret_cast<const uint2*>(p.v_self + idx[u]));
                                 const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.x));
                                 const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.y));
-                                const float cb = coef_b[c];
-                                acc[u] = make_float4(cb * v01.x, cb * v01.y, cb * v23.x, cb * v23.y);
+                                const float cbv = coef_b[c];
+                                acc[u] = make_float4(cbv * v01.x, cbv * v01.y, cbv * v23.x, cbv * v23.y);
                             }
                         }
 #pragma unroll
@@ -801,13 +819,13 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 #pragma unroll
                                 for (int u = 0; u < 4; ++u) {
                                     if (cc[u] >= 0) {
-                                        const float4 po =
+                                        const float4 pv =
                                             __ldcg(reinterpret_cast<const float4*>(p.part_o + s * split_stride + idx[u]));
                                         const float wv = wts[s * N + cc[u]];
-                                        acc[u].x = fmaf(wv, po.x, acc[u].x);
-                                        acc[u].y = fmaf(wv, po.y, acc[u].y);
-                                        acc[u].z = fmaf(wv, po.z, acc[u].z);
-                                        acc[u].w = fmaf(wv, po.w, acc[u].w);
+                                        acc[u].x = fmaf(wv, pv.x, acc[u].x);
+                                        acc[u].y = fmaf(wv, pv.y, acc[u].y);
+                                        acc[u].z = fmaf(wv, pv.z, acc[u].z);
+                                        acc[u].w = fmaf(wv, pv.w, acc[u].w);
                                     }
                                 }
                             }
@@ -818,8 +836,8 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                     }
                 }
             }
-            // scratch (red, coef, weights) is reused by the next item
-            if (!(ok = sk_group_sync(grp, ngrp, ctl, lane))) break;
+            // scratch (red, weights) is reused by the next item
+            if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
         }
     }
 

@@ -149,6 +149,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
     return done != 0;
 }
 
+// Non-blocking probe: has phase `parity` of `bar` completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Shared state every bounded wait of a CTA consults.  `abort` is set by the
 // first wait that runs out of time; the others then give up promptly, so the
 // whole CTA reaches its exit path instead of spinning.
@@ -177,6 +191,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
             }
         }
     }
+}
+
+// Bounded barrier among the warps that arrive on `bar` (an mbarrier whose
+// arrival count is their number; one arrival per warp).  Unlike bar.sync it
+// gives up when the block aborts.  `n` counts the barrier's completed phases.
+__device__ __forceinline__ bool warp_group_sync(uint64_t* bar, uint32_t& n, const WaitCtl& ctl, int lane)
+{
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, n & 1, ctl));
+    ++n;
+    return ok;
 }
 
 // Time-limited wait that ignores the abort flag: used on the exit path to
@@ -209,6 +235,23 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
 }
+
+// 3-D tiled store shared -> global (box as the map's), tracked by this thread's bulk group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Waits until the shared-memory sources of this thread's bulk stores have been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Waits until this thread's bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (UMMA operands).
 __device__ __forceinline__ void fence_proxy_async_smem()

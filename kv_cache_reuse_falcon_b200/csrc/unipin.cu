@@ -13,6 +13,7 @@
 #include "unipin.h"
 #include "sm100_ptx.cuh"
 #include "attn_sm100.cuh"
+#include "bwd_sm100.cuh"
 #include "decode_smallk_sm100.cuh"
 #include "kvpool_sm100.cuh"
 
@@ -78,18 +79,22 @@ int set_attn_attr(K kernel, int smem_bytes)
 template <int D>
 int set_attn_attrs()
 {
-    int rc = set_attn_attr(attn_fwd_kernel<D, false>, AttnCfg<D>::kSmemBytes);
+    int rc = set_attn_attr(attn_fwd_kernel<D, false>, AttnCfg<D, false>::kSmemBytes);
     if (rc != UNIPIN_OK) return rc;
-    return set_attn_attr(attn_fwd_kernel<D, true>, AttnCfg<D>::kSmemBytes);
+    return set_attn_attr(attn_fwd_kernel<D, true>, AttnCfg<D, true>::kSmemBytes);
 }
 
 template <int D, int N>
 int set_sk_attr()
 {
-    return cudaFuncSetAttribute(decode_smallk_kernel<D, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                SkCfg<D, N>::kSmemBytes) == cudaSuccess
-               ? UNIPIN_OK
-               : UNIPIN_ERR_CUDA;
+    if (cudaFuncSetAttribute(decode_smallk_kernel<D, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SkCfg<D, N>::kSmemBytes) != cudaSuccess)
+        return UNIPIN_ERR_CUDA;
+    // All of the SM's on-chip memory as shared memory, so that two blocks fit where they are meant to.
+    if (cudaFuncSetAttribute(decode_smallk_kernel<D, N>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+        return UNIPIN_ERR_CUDA;
+    return UNIPIN_OK;
 }
 
 template <int D>
@@ -131,6 +136,12 @@ int ensure_device()
     if (rc == UNIPIN_OK) rc = set_attn_attrs<128>();
     if (rc == UNIPIN_OK) rc = set_sk_attrs<64>();
     if (rc == UNIPIN_OK) rc = set_sk_attrs<128>();
+    if (rc == UNIPIN_OK &&
+        (cudaFuncSetAttribute(bwd_kv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              BwCfg<32>::kSmemBytes) != cudaSuccess ||
+         cudaFuncSetAttribute(bwd_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              BwCfg<64>::kSmemBytes) != cudaSuccess))
+        rc = UNIPIN_ERR_CUDA;
     if (rc != UNIPIN_OK) return rc;
     g_device_ready[dev] = true;
     return UNIPIN_OK;
@@ -182,19 +193,21 @@ int check_pool(const unipin_kvpool* pool, int H, int D, int layer)
 
 bool supported_d(int D) { return D == 32 || D == 64 || D == 128; }
 
+// tpk, tpv: the pool as the prefill's fused pool write stores into it (unused otherwise).
 template <bool kDecode>
 int launch_attn(int D, dim3 grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                const AttnParams& p, cudaStream_t s)
+                const CUtensorMap& tpk, const CUtensorMap& tpv, const AttnParams& p, cudaStream_t s)
 {
     switch (D) {
     case 32:
-        attn_fwd_kernel<32, kDecode><<<grid, kThreads, AttnCfg<32>::kSmemBytes, s>>>(tq, tk, tv, p);
+        attn_fwd_kernel<32, kDecode><<<grid, kThreads, AttnCfg<32, kDecode>::kSmemBytes, s>>>(tq, tk, tv, tpk, tpv, p);
         break;
     case 64:
-        attn_fwd_kernel<64, kDecode><<<grid, kThreads, AttnCfg<64>::kSmemBytes, s>>>(tq, tk, tv, p);
+        attn_fwd_kernel<64, kDecode><<<grid, kThreads, AttnCfg<64, kDecode>::kSmemBytes, s>>>(tq, tk, tv, tpk, tpv, p);
         break;
     case 128:
-        attn_fwd_kernel<128, kDecode><<<grid, kThreads, AttnCfg<128>::kSmemBytes, s>>>(tq, tk, tv, p);
+        attn_fwd_kernel<128, kDecode><<<grid, kThreads, AttnCfg<128, kDecode>::kSmemBytes, s>>>(tq, tk, tv, tpk, tpv,
+                                                                                               p);
         break;
     default:
         return UNIPIN_ERR_UNSUPPORTED;
@@ -236,7 +249,7 @@ int decode_nsplit(int R, int H, int D, int max_k, int n_cap, int sms)
     const long long slots = (long long)sms;   // one block per SM (all of TMEM)
     const long long target = 4 * slots;
     if (units >= 2 * slots) return 1;   // two or more waves already: no split
-    const int key_tiles = (n_cap + key_tile_width(D) - 1) / key_tile_width(D);
+    const int key_tiles = (n_cap + key_tile_width(D, true) - 1) / key_tile_width(D, true);
     long long ns = (target + units - 1) / units;
     const long long cap = key_tiles / 2 > 1 ? key_tiles / 2 : 1;   // at least two key tiles per split
     if (ns > cap) ns = cap;
@@ -305,14 +318,12 @@ SkPlan sk_plan(int R, int H, int D, int max_k, int n_cap, int sms)
     const long long tiles = (n_cap + kSkKeys - 1) / kSkKeys;
     const long long pairs = (long long)R * H;
     const long long target = (long long)sk_items_per_block() * sms * pl.blocks_per_sm;
-    long long per = (pairs * tiles + target - 1) / target;
-    if (per < 1) per = 1;
-    if (per > tiles) per = tiles;
-    long long ns = (tiles + per - 1) / per;
-    if (ns > kSkMaxSplit) {
-        per = (tiles + kSkMaxSplit - 1) / kSkMaxSplit;
-        ns = (tiles + per - 1) / per;
-    }
+    long long ns = (target + pairs - 1) / pairs;   // splits per (request, head) for the target item count
+    if (ns > tiles) ns = tiles;
+    if (ns > kSkMaxSplit) ns = kSkMaxSplit;
+    if (ns < 1) ns = 1;
+    long long per = (tiles + ns - 1) / ns;         // equal runs of tiles
+    ns = (tiles + per - 1) / per;
     pl.nsplit = (int)(ns < 1 ? 1 : ns);
     pl.tiles_per_split = (int)(pl.nsplit == 1 ? (tiles < 1 ? 1 : tiles) : per);
     return pl;
@@ -461,7 +472,7 @@ const char* unipin_status_string(int status)
 
 size_t unipin_masked_prefill_workspace_size(void) { return kSchedBytes; }
 
-int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32,
+int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32, float* lse,
                                const int* cu_seqlens, const int* past_lens, int B, int H, int D, int max_seqlen,
                                int total_tokens, float scale, const unipin_kvpool* pool, const int* slot_ids,
                                int layer, void* workspace, size_t workspace_bytes, int* dev_status, void* stream)
@@ -478,6 +489,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     if (!q || !k || !v || !out || !cu_seqlens || !past_lens) return UNIPIN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return UNIPIN_ERR_MISALIGNED;
     if (workspace && !aligned16(workspace)) return UNIPIN_ERR_MISALIGNED;
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u) != 0) return UNIPIN_ERR_MISALIGNED;
     int rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -487,15 +499,18 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
         if (cudaMemsetAsync(sched, 0, sizeof(unsigned long long), s) != cudaSuccess) return UNIPIN_ERR_CUDA;
     }
 
-    if (pool) {
-        rc = launch_pool_write(pool, layer, k, v, cu_seqlens, past_lens, slot_ids, B, H, D, max_seqlen, total_tokens,
-                               dev_status, s);
-        if (rc != UNIPIN_OK) return rc;
-    }
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tpk, tpv;
     if ((rc = make_token_map(&tq, q, total_tokens, H, D, kBlockM)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tk, k, total_tokens, H, D, key_tile_width(D))) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tv, v, total_tokens, H, D, key_tile_width(D))) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tk, k, total_tokens, H, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tv, v, total_tokens, H, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
+    if (pool) {
+        // the past K/V tiles the kernel loads are also stored into the pool (no second pass)
+        if ((rc = make_pool_map(&tpk, pool->k, pool, key_tile_width(D, false))) != UNIPIN_OK) return rc;
+        if ((rc = make_pool_map(&tpv, pool->v, pool, key_tile_width(D, false))) != UNIPIN_OK) return rc;
+    } else {
+        tpk = tk;
+        tpv = tv;
+    }
 
     AttnParams p = {};
     p.q = static_cast<const __nv_bfloat16*>(q);
@@ -515,9 +530,19 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
     p.sched = sched;
+    p.lse = lse;
+    if (pool) {
+        p.store_pool = 1;
+        p.pool_k = pool->k;
+        p.pool_v = pool->v;
+        p.slots = slot_ids;
+        p.layer = layer;
+        p.S = pool->S;
+        p.n_cap = pool->n_cap;
+    }
     const long long bound = (long long)B * H * ((max_seqlen + kPairRows - 1) / kPairRows);
     dim3 grid(persistent_blocks(bound), 1, 1);
-    return launch_attn<false>(D, grid, tq, tk, tv, p, s);
+    return launch_attn<false>(D, grid, tq, tk, tv, tpk, tpv, p, s);
 }
 
 int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, const void* v, const int* cu_seqlens,
@@ -580,8 +605,8 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
 
     CUtensorMap tq, tk, tv;
     if ((rc = make_token_map(&tq, q_c, total_cand, H, D, kBlockM)) != UNIPIN_OK) return rc;
-    if ((rc = make_pool_map(&tk, pool->k, pool, key_tile_width(D))) != UNIPIN_OK) return rc;
-    if ((rc = make_pool_map(&tv, pool->v, pool, key_tile_width(D))) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tk, pool->k, pool, key_tile_width(D, true))) != UNIPIN_OK) return rc;
+    if ((rc = make_pool_map(&tv, pool->v, pool, key_tile_width(D, true))) != UNIPIN_OK) return rc;
 
     AttnParams p = {};
     p.q = static_cast<const __nv_bfloat16*>(q_c);
@@ -610,7 +635,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     }
     const long long bound = (long long)R * H * nsplit * ((max_k + kPairRows - 1) / kPairRows);
     dim3 grid(persistent_blocks(bound), 1, 1);
-    rc = launch_attn<true>(D, grid, tq, tk, tv, p, s);
+    rc = launch_attn<true>(D, grid, tq, tk, tv, tk, tv, p, s);
     if (rc != UNIPIN_OK || nsplit == 1) return rc;
 
     const long long rows = (long long)total_cand * H;
@@ -651,6 +676,77 @@ int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void
 }
 
 size_t unipin_rank_decode_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+size_t unipin_masked_prefill_bwd_workspace_size(int total_tokens, int H)
+{
+    if (total_tokens < 0 || H < 1) return 0;
+    return ((size_t)total_tokens * H * sizeof(float) + 15) / 16 * 16;
+}
+
+int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                              const float* lse, float* dq, float* dk, float* dv, const int* cu_seqlens,
+                              const int* past_lens, int B, int H, int D, int max_seqlen, int total_tokens,
+                              float scale, void* workspace, size_t workspace_bytes, int* dev_status, void* stream)
+{
+    if (B < 0 || H < 1 || max_seqlen < 0 || total_tokens < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (D != 32 && D != 64) return UNIPIN_ERR_UNSUPPORTED;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return UNIPIN_ERR_INVALID_ARG;
+    if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !cu_seqlens || !past_lens || !workspace)
+        return UNIPIN_ERR_INVALID_ARG;
+    if (workspace_bytes < unipin_masked_prefill_bwd_workspace_size(total_tokens, H)) return UNIPIN_ERR_INVALID_ARG;
+    for (const void* ptr : {q, k, v, out, dout, (const void*)lse, (const void*)dq, (const void*)dk, (const void*)dv,
+                            (const void*)workspace})
+        if (!aligned16(ptr)) return UNIPIN_ERR_MISALIGNED;
+    const long long items = (long long)B * H * ((max_seqlen + kBwRows - 1) / kBwRows);
+    if (items >= (1ll << 31)) return UNIPIN_ERR_INVALID_ARG;
+    int rc = ensure_device();
+    if (rc != UNIPIN_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    BwParams p = {};
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.o = static_cast<const __nv_bfloat16*>(out);
+    p.dout = static_cast<const __nv_bfloat16*>(dout);
+    p.lse = lse;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dvec = static_cast<float*>(workspace);
+    p.cu = cu_seqlens;
+    p.past = past_lens;
+    p.B = B;
+    p.H = H;
+    p.total_rows = total_tokens;
+    p.max_rows = max_seqlen;
+    p.scale = scale;
+    p.sl2 = scale * kLog2e;
+    p.status = dev_status;
+    p.wait_limit_ns = wait_limit_ns();
+
+    const long long rows = (long long)total_tokens * H;
+    const unsigned prep_blocks = (unsigned)((rows + 7) / 8);
+    if (D == 32)
+        bwd_prep_kernel<32><<<prep_blocks, 256, 0, s>>>(p);
+    else
+        bwd_prep_kernel<64><<<prep_blocks, 256, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return UNIPIN_ERR_CUDA;
+
+    CUtensorMap tq, tk, tv, tdo;
+    if ((rc = make_token_map(&tq, q, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tk, k, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tv, v, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tdo, dout, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
+    if (D == 32)
+        bwd_kv_kernel<32><<<(unsigned)items, kBwThreads, BwCfg<32>::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    else
+        bwd_kv_kernel<64><<<(unsigned)items, kBwThreads, BwCfg<64>::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+}
+
+
 
 int unipin_selftest_exp2(const float* x, float* y, int n, void* stream)
 {

@@ -75,3 +75,36 @@ def test_reference_arm_prints_one_oracle_line():
     assert d["config"]["workload"].startswith("tiny_prefill_B2_H2_D32")
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_gpus_flag_relaunches_one_rank_per_gpu():
+    """--gpus N without a launcher starts N ranks through torch's launcher on 127.0.0.1."""
+    cmd = bench.relaunch_command(["--gpus", "4", "--steps", "5"], 4, port=29555)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert cmd[cmd.index("--nproc-per-node") + 1] == "4"
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[cmd.index("--master-port") + 1] == "29555"
+    assert cmd[cmd.index("--master-port") + 2].endswith("bench.py")
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "5"]
+
+
+def test_gpus_flag_must_match_the_launcher(monkeypatch):
+    """Under a launcher, --gpus that disagrees with WORLD_SIZE is an error, never ignored."""
+    import pytest
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "0")
+    with pytest.raises(SystemExit) as e:
+        bench.main(["--gpus", "4", "--workload", "tiny"])
+    assert e.value.code == 2
+
+
+def test_reference_arm_with_several_gpus_runs_once():
+    """The oracle arm under --gpus 2 without a launcher runs on the host once and prints one line."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, bench.__file__, "--impl", "reference", "--gpus", "2", "--workload", "tiny",
+                        "--steps", "1", "--warmup", "3"], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1 and json.loads(lines[0])["impl"] == "reference"

@@ -100,9 +100,13 @@ def test_kvpool_write_bit_exact_on_nan_poisoned_pool(ub):
     assert bf16_tensor_bits(pv).tobytes() == hv.tobytes()
 
 
-def test_fused_prefill_pool_write_bit_exact(ub):
-    past, cand = [100, 7, 260], [20, 3, 40]
-    H, D, L, S, n_cap = 2, 128, 2, 5, 300
+@pytest.mark.parametrize("D", [128, 64, 32])
+def test_fused_prefill_pool_write_bit_exact(ub, D):
+    """The prefill stores each segment's past K/V tiles into its slot as it loads them: whole
+    64-key tiles, the right-aligned last tile, and histories shorter than one tile (copied
+    row by row); nothing else in the pool changes."""
+    past, cand = [100, 7, 260, 0, 1, 63, 64, 65], [20, 3, 40, 5, 2, 1, 0, 9]
+    H, L, S, n_cap = 2, 2, 9, 300
     batch = synth.make_prefill(1400, past, cand, H, D, n_slots=S)
     dp = DevPrefill(batch)
     pk, pv = nan_pool(L, S, H, n_cap, D)
@@ -203,9 +207,13 @@ def test_k1_candidate_is_independent_of_its_batch(ub):
         assert np.array_equal(o[n], full[n + c])
 
 
-def test_prefill_candidate_rows_equal_decode_over_written_pool(ub):
+@pytest.mark.parametrize("D", [128, 64])
+def test_prefill_candidate_rows_equal_decode_over_written_pool(ub, D):
+    """Decode over the pool the prefill wrote gives the prefill's candidate rows: bit for bit at
+    D = 128 (both calls sweep 64-key tiles), within tolerance at D = 64 (the prefill sweeps 64-key
+    tiles, the many-candidate decode 128-key tiles)."""
     past, cand = [300, 0, 129, 1000], [50, 4, 130, 9]
-    H, D, L, S, n_cap = 2, 64, 2, 6, 1024
+    H, L, S, n_cap = 2, 2, 6, 1024
     batch = synth.make_prefill(3200, past, cand, H, D, n_slots=S)
     dp = DevPrefill(batch)
     pk, pv = nan_pool(L, S, H, n_cap, D)
@@ -217,7 +225,8 @@ def test_prefill_candidate_rows_equal_decode_over_written_pool(ub):
     pre_c = pre[torch.from_numpy(cidx).cuda()]
     assert torch.isfinite(dec).all()
     parity(dec.cpu().numpy(), pre_c.cpu().numpy().astype(np.float64), "prefill vs decode")
-    assert torch.equal(dec, pre_c), "decode rows differ from prefill candidate rows in some bits"
+    if D == 128:
+        assert torch.equal(dec, pre_c), "decode rows differ from prefill candidate rows in some bits"
 
 
 # ------------------------------------------------------------- error reporting
