@@ -47,14 +47,14 @@ def _load():
         P = ctypes.c_void_p
         I = ctypes.c_int
         I64 = ctypes.c_int64
-        lib.oracle_prefill_rows.argtypes = [P, P, P, P, P, I, I, I, ctypes.c_double, I, P, I64, P, P]
+        lib.oracle_prefill_rows.argtypes = [P, P, P, P, P, I, I, I, I, ctypes.c_double, I, P, I64, P, P]
         lib.oracle_prefill_rows.restype = I
-        lib.oracle_decode_rows.argtypes = [P, P, P, P, P, P, I, I, I, ctypes.c_double, I,
+        lib.oracle_decode_rows.argtypes = [P, P, P, P, P, P, I, I, I, I, ctypes.c_double, I,
                                            P, P, I, I, I, I, P, I64, P, P]
         lib.oracle_decode_rows.restype = I
-        lib.oracle_prefill_bwd.argtypes = [P, P, P, P, P, P, I, I, I, ctypes.c_double, I, P, P, P]
+        lib.oracle_prefill_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, ctypes.c_double, I, P, P, P]
         lib.oracle_prefill_bwd.restype = I
-        lib.oracle_prefill_bwd_f64.argtypes = [P, P, P, P, P, P, I, I, I, ctypes.c_double, I, P, P, P]
+        lib.oracle_prefill_bwd_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, ctypes.c_double, I, P, P, P]
         lib.oracle_prefill_bwd_f64.restype = I
         lib.oracle_pool_write.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, I]
         lib.oracle_pool_write.restype = I
@@ -79,6 +79,15 @@ def _i32(a) -> np.ndarray:
     return np.ascontiguousarray(a, dtype=np.int32)
 
 
+def _kv_heads(q, k, v) -> int:
+    """Key/value heads of grouped-query inputs: k and v share a shape whose head count divides q's."""
+    if k.shape != v.shape or k.shape[0] != q.shape[0] or k.shape[2] != q.shape[2]:
+        raise ValueError("k and v must be [T, Hkv, D] with q's T and D")
+    if q.shape[1] % k.shape[1] != 0:
+        raise ValueError("query heads must be a multiple of key/value heads")
+    return int(k.shape[1])
+
+
 def num_threads() -> int:
     return int(_load().oracle_num_threads())
 
@@ -89,9 +98,13 @@ def set_num_threads(n: int) -> None:
 
 def prefill(q, k, v, cu_seqlens, past_lens, scale: Optional[float] = None, cand_self: bool = True,
             tokens=None, return_lse: bool = False):
-    """M-FALCON masked attention of packed segments; returns float64 [ntok, H, D] (and lse [ntok, H])."""
+    """M-FALCON masked attention of packed segments; returns float64 [ntok, H, D] (and lse [ntok, H]).
+
+    k and v may have fewer heads than q (grouped-query attention: query head h reads kv head
+    h // (H // Hkv))."""
     q, k, v = _u16(q), _u16(k), _u16(v)
     T, H, D = q.shape
+    Hkv = _kv_heads(q, k, v)
     cu = _i32(cu_seqlens)
     past = _i32(past_lens)
     B = past.shape[0]
@@ -102,7 +115,7 @@ def prefill(q, k, v, cu_seqlens, past_lens, scale: Optional[float] = None, cand_
     ntok = T if tok is None else tok.shape[0]
     out = np.zeros((ntok, H, D), dtype=np.float64)
     lse = np.zeros((ntok, H), dtype=np.float64) if return_lse else None
-    rc = _load().oracle_prefill_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), _ptr(past), B, H, D, scale,
+    rc = _load().oracle_prefill_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(cu), _ptr(past), B, H, Hkv, D, scale,
                                      int(bool(cand_self)), _ptr(tok), ntok, _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_prefill_rows rejected its arguments")
@@ -115,8 +128,9 @@ def decode(qc, kc, vc, cu_c, slot_ids, past_lens, pool_k, pool_v, layer: int,
     qc, kc, vc = _u16(qc), _u16(kc), _u16(vc)
     pool_k, pool_v = _u16(pool_k), _u16(pool_v)
     Tc, H, D = qc.shape
+    Hkv = _kv_heads(qc, kc, vc)
     L, S, Hp, n_cap, Dp = pool_k.shape
-    if (Hp, Dp) != (H, D) or pool_v.shape != pool_k.shape:
+    if (Hp, Dp) != (Hkv, D) or pool_v.shape != pool_k.shape:
         raise ValueError("pool shape does not match candidates")
     cu = _i32(cu_c)
     slots = _i32(slot_ids)
@@ -130,7 +144,7 @@ def decode(qc, kc, vc, cu_c, slot_ids, past_lens, pool_k, pool_v, layer: int,
     out = np.zeros((ntok, H, D), dtype=np.float64)
     lse = np.zeros((ntok, H), dtype=np.float64) if return_lse else None
     rc = _load().oracle_decode_rows(_ptr(qc), _ptr(kc), _ptr(vc), _ptr(cu), _ptr(slots), _ptr(past),
-                                    R, H, D, scale, int(bool(cand_self)), _ptr(pool_k), _ptr(pool_v),
+                                    R, H, Hkv, D, scale, int(bool(cand_self)), _ptr(pool_k), _ptr(pool_v),
                                     L, S, n_cap, int(layer), _ptr(tok), ntok, _ptr(out), _ptr(lse))
     if rc != 0:
         raise ValueError("oracle_decode_rows rejected its arguments")
@@ -154,25 +168,27 @@ def pool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids
 
 def _bwd(fn, q, k, v, dout, cu_seqlens, past_lens, scale, cand_self):
     T, H, D = q.shape
+    Hkv = _kv_heads(q, k, v)
     cu = _i32(cu_seqlens)
     past = _i32(past_lens)
     B = past.shape[0]
     if cu.shape[0] != B + 1 or int(cu[-1]) != T:
         raise ValueError("cu_seqlens does not match q")
-    for a in (k, v, dout):
-        if a.shape != q.shape:
-            raise ValueError("q, k, v and dout must have one shape")
+    if dout.shape != q.shape:
+        raise ValueError("dout must have the shape of q")
     scale = 1.0 / np.sqrt(D) if scale is None else float(scale)
-    dq, dk, dv = (np.zeros((T, H, D), dtype=np.float64) for _ in range(3))
-    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(cu), _ptr(past), B, H, D, scale, int(bool(cand_self)),
-            _ptr(dq), _ptr(dk), _ptr(dv))
+    dq = np.zeros((T, H, D), dtype=np.float64)
+    dk, dv = (np.zeros((T, Hkv, D), dtype=np.float64) for _ in range(2))
+    rc = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(cu), _ptr(past), B, H, Hkv, D, scale,
+            int(bool(cand_self)), _ptr(dq), _ptr(dk), _ptr(dv))
     if rc != 0:
         raise ValueError("oracle backward rejected its arguments")
     return dq, dk, dv
 
 
 def prefill_bwd(q, k, v, dout, cu_seqlens, past_lens, scale: Optional[float] = None, cand_self: bool = True):
-    """Gradients (dq, dk, dv), float64 [T, H, D], of the masked prefill for upstream gradient dout (bf16 bits)."""
+    """Gradients of the masked prefill for upstream gradient dout (bf16 bits): dq float64 [T, H, D],
+    dk and dv [T, Hkv, D] (with grouped heads a kv head sums its query heads' contributions)."""
     q, k, v, dout = _u16(q), _u16(k), _u16(v), _u16(dout)
     return _bwd(_load().oracle_prefill_bwd, q, k, v, dout, cu_seqlens, past_lens, scale, cand_self)
 

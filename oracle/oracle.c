@@ -32,6 +32,10 @@
  * over allowed j, with m_i = max over allowed j.  Inputs are bfloat16 bit
  * patterns, widened exactly to double.
  *
+ * Heads ([notes] §6 calls the pool's H "KV heads"): queries may have more
+ * heads than keys and values, H = G * Hkv; query head h reads key/value head
+ * h / G (grouped-query attention).  G = 1 is plain multi-head attention.
+ *
  * Pool ([notes] §6; [review] §2.4): one preallocated tensor of shape
  * [L, S, H, n, D] (layer, slot, KV head, history length, head dim) for K and
  * one for V.  Rank decode of a request reads rows 0..n_r-1 of its slot at the
@@ -124,7 +128,8 @@ static void attend(const uint16_t *qrow, const uint16_t *const *keys,
 
 /*
  * Masked prefill attention over packed segments.
- *   q, k, v     : bf16 bits, [T, H, D] row-major, T = cu_seqlens[B]
+ *   q           : bf16 bits, [T, H, D] row-major, T = cu_seqlens[B]
+ *   k, v        : bf16 bits, [T, Hkv, D]; query head h reads kv head h / (H / Hkv)
  *   cu_seqlens  : [B+1], segment b spans tokens cu[b] .. cu[b+1]-1
  *   past_lens   : [B], n_b <= cu[b+1]-cu[b]; the rest of segment b are candidates
  *   tokens      : packed token indices to evaluate (NULL = all T)
@@ -132,11 +137,12 @@ static void attend(const uint16_t *qrow, const uint16_t *const *keys,
  * Returns 0, or -1 on inconsistent arguments.
  */
 int oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
-                        const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int D,
+                        const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int Hkv, int D,
                         double scale, int cand_self, const int64_t *tokens, int64_t ntok,
                         double *out, double *lse)
 {
-    if (B < 1 || H < 1 || D < 1) return -1;
+    if (B < 1 || H < 1 || D < 1 || Hkv < 1 || H % Hkv != 0) return -1;
+    const int G = H / Hkv;
     int64_t T = cu_seqlens[B];
     int64_t max_len = 0;
     for (int b = 0; b < B; ++b) {
@@ -171,8 +177,8 @@ int oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             int64_t nk = 0;
             for (int64_t j = 0; j < len; ++j) {
                 if (!allowed(i, j, n_past, cand_self)) continue;
-                kp[nk] = k + ((start + j) * H + h) * (int64_t)D;
-                vp[nk] = v + ((start + j) * H + h) * (int64_t)D;
+                kp[nk] = k + ((start + j) * Hkv + h / G) * (int64_t)D;
+                vp[nk] = v + ((start + j) * Hkv + h / G) * (int64_t)D;
                 ++nk;
             }
             attend(q + (t * H + h) * (int64_t)D, kp, vp, nk, D, scale, s,
@@ -187,22 +193,24 @@ int oracle_prefill_rows(const uint16_t *q, const uint16_t *k, const uint16_t *v,
 
 /*
  * Rank decode over the cached pool ([review] §2.4, [notes] §6).
- *   qc, kc, vc     : candidate bf16 bits, [Tc, H, D], Tc = cu_c[R]
+ *   qc             : candidate bf16 bits, [Tc, H, D], Tc = cu_c[R]
+ *   kc, vc         : candidate bf16 bits, [Tc, Hkv, D]
  *   cu_c           : [R+1] candidate offsets of each request
  *   slot_ids       : [R] pool slot of each request
  *   past_lens      : [R] cached rows n_r of each request (n_r <= n_cap)
- *   pool_k, pool_v : bf16 bits, [L, S, H, n_cap, D]
+ *   pool_k, pool_v : bf16 bits, [L, S, Hkv, n_cap, D]; query head h reads kv head h / (H / Hkv)
  *   tokens         : candidate indices to evaluate (NULL = all Tc)
  * Candidate c of request r attends to pool rows 0..n_r-1 of slot_ids[r] at
  * `layer`, and (cand_self) to its own key/value.
  */
 int oracle_decode_rows(const uint16_t *qc, const uint16_t *kc, const uint16_t *vc,
                        const int32_t *cu_c, const int32_t *slot_ids, const int32_t *past_lens,
-                       int R, int H, int D, double scale, int cand_self,
+                       int R, int H, int Hkv, int D, double scale, int cand_self,
                        const uint16_t *pool_k, const uint16_t *pool_v, int L, int S, int n_cap,
                        int layer, const int64_t *tokens, int64_t ntok, double *out, double *lse)
 {
-    if (R < 1 || H < 1 || D < 1 || layer < 0 || layer >= L) return -1;
+    if (R < 1 || H < 1 || D < 1 || layer < 0 || layer >= L || Hkv < 1 || H % Hkv != 0) return -1;
+    const int G = H / Hkv;
     for (int r = 0; r < R; ++r) {
         if (cu_c[r + 1] < cu_c[r]) return -1;
         if (slot_ids[r] < 0 || slot_ids[r] >= S) return -1;
@@ -232,7 +240,7 @@ int oracle_decode_rows(const uint16_t *qc, const uint16_t *kc, const uint16_t *v
             int64_t t = tokens ? tokens[x] : x;
             int r = find_segment(cu_c, R, t);
             int64_t n_r = past_lens[r];
-            int64_t row0 = (((int64_t)layer * S + slot_ids[r]) * H + h) * (int64_t)n_cap;
+            int64_t row0 = (((int64_t)layer * S + slot_ids[r]) * Hkv + h / G) * (int64_t)n_cap;
             int64_t nk = 0;
             for (int64_t j = 0; j < n_r; ++j) {
                 kp[nk] = pool_k + (row0 + j) * D;
@@ -240,8 +248,8 @@ int oracle_decode_rows(const uint16_t *qc, const uint16_t *kc, const uint16_t *v
                 ++nk;
             }
             if (cand_self) {
-                kp[nk] = kc + (t * H + h) * (int64_t)D;
-                vp[nk] = vc + (t * H + h) * (int64_t)D;
+                kp[nk] = kc + (t * Hkv + h / G) * (int64_t)D;
+                vp[nk] = vc + (t * Hkv + h / G) * (int64_t)D;
                 ++nk;
             }
             attend(qc + (t * H + h) * (int64_t)D, kp, vp, nk, D, scale, s,
@@ -271,15 +279,18 @@ int oracle_decode_rows(const uint16_t *qc, const uint16_t *kc, const uint16_t *v
  *
  * so a past key receives gradient from the later past rows and from every
  * candidate row; a candidate's own key and value only from its own row.
- * Inputs are doubles (bf16 inputs are widened exactly by the caller);
- * dq, dk, dv are written in full.  Parallel over (segment, head): every
- * gradient element belongs to exactly one of them.
+ * With grouped heads a key/value head's gradient sums the contributions of
+ * its G query heads.  Inputs are doubles (bf16 inputs are widened exactly by
+ * the caller); dq [T, H, D], dk and dv [T, Hkv, D] are written in full.
+ * Parallel over (segment, kv head): every gradient element belongs to
+ * exactly one of them.
  */
 int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, const double *dout,
-                           const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int D,
+                           const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int Hkv, int D,
                            double scale, int cand_self, double *dq, double *dk, double *dv)
 {
-    if (B < 1 || H < 1 || D < 1) return -1;
+    if (B < 1 || H < 1 || D < 1 || Hkv < 1 || H % Hkv != 0) return -1;
+    const int G = H / Hkv;
     int64_t max_len = 0;
     for (int b = 0; b < B; ++b) {
         int64_t len = (int64_t)cu_seqlens[b + 1] - cu_seqlens[b];
@@ -288,8 +299,8 @@ int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, co
     }
     int64_t T = cu_seqlens[B];
     memset(dq, 0, sizeof(double) * (size_t)(T * H * D));
-    memset(dk, 0, sizeof(double) * (size_t)(T * H * D));
-    memset(dv, 0, sizeof(double) * (size_t)(T * H * D));
+    memset(dk, 0, sizeof(double) * (size_t)(T * Hkv * D));
+    memset(dv, 0, sizeof(double) * (size_t)(T * Hkv * D));
     int bad = 0;
 #pragma omp parallel
     {
@@ -301,11 +312,13 @@ int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, co
             bad = 1;
         }
 #pragma omp for schedule(dynamic, 1)
-        for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        for (int64_t bh = 0; bh < (int64_t)B * Hkv; ++bh) {
             if (bad) continue;
-            int b = (int)(bh / H), h = (int)(bh % H);
+            int b = (int)(bh / Hkv), hk = (int)(bh % Hkv);
             int64_t start = cu_seqlens[b], len = (int64_t)cu_seqlens[b + 1] - start, n_past = past_lens[b];
+            for (int h = hk * G; h < (hk + 1) * G; ++h)
 #define ROW(x, t) ((x) + (((start + (t)) * H + h) * (int64_t)D))
+#define KROW(x, t) ((x) + (((start + (t)) * Hkv + hk) * (int64_t)D))
             for (int64_t i = 0; i < len; ++i) {
                 int64_t nk = 0;
                 for (int64_t j = 0; j < len; ++j)
@@ -315,7 +328,7 @@ int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, co
                 double m = -INFINITY;
                 for (int64_t a = 0; a < nk; ++a) {
                     double dot = 0.0;
-                    for (int d = 0; d < D; ++d) dot += ROW(q, i)[d] * ROW(k, js[a])[d];
+                    for (int d = 0; d < D; ++d) dot += ROW(q, i)[d] * KROW(k, js[a])[d];
                     p[a] = dot * scale;
                     if (p[a] > m) m = p[a];
                 }
@@ -329,7 +342,7 @@ int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, co
                 double dmean = 0.0;
                 for (int64_t a = 0; a < nk; ++a) {
                     double dot = 0.0;
-                    for (int d = 0; d < D; ++d) dot += ROW(dout, i)[d] * ROW(v, js[a])[d];
+                    for (int d = 0; d < D; ++d) dot += ROW(dout, i)[d] * KROW(v, js[a])[d];
                     dp[a] = dot;
                     dmean += p[a] * dot;
                 }
@@ -337,13 +350,14 @@ int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, co
                     int64_t j = js[a];
                     double ds = p[a] * (dp[a] - dmean);
                     for (int d = 0; d < D; ++d) {
-                        ROW(dv, j)[d] += p[a] * ROW(dout, i)[d];
-                        ROW(dq, i)[d] += scale * ds * ROW(k, j)[d];
-                        ROW(dk, j)[d] += scale * ds * ROW(q, i)[d];
+                        KROW(dv, j)[d] += p[a] * ROW(dout, i)[d];
+                        ROW(dq, i)[d] += scale * ds * KROW(k, j)[d];
+                        KROW(dk, j)[d] += scale * ds * ROW(q, i)[d];
                     }
                 }
             }
 #undef ROW
+#undef KROW
         }
         free(p);
         free(dp);
@@ -354,21 +368,24 @@ int oracle_prefill_bwd_f64(const double *q, const double *k, const double *v, co
 
 /* As oracle_prefill_bwd_f64 for bf16 inputs (bit patterns), widened exactly. */
 int oracle_prefill_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
-                       const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int D,
+                       const int32_t *cu_seqlens, const int32_t *past_lens, int B, int H, int Hkv, int D,
                        double scale, int cand_self, double *dq, double *dk, double *dv)
 {
-    if (B < 1 || H < 1 || D < 1) return -1;
-    size_t n = (size_t)cu_seqlens[B] * (size_t)H * (size_t)D;
-    double *w = (double *)malloc(sizeof(double) * (4 * n + 1));
+    if (B < 1 || H < 1 || D < 1 || Hkv < 1) return -1;
+    size_t n = (size_t)cu_seqlens[B] * (size_t)H * (size_t)D;       /* q, dout */
+    size_t m = (size_t)cu_seqlens[B] * (size_t)Hkv * (size_t)D;     /* k, v */
+    double *w = (double *)malloc(sizeof(double) * (2 * n + 2 * m + 1));
     if (!w) return -1;
     for (size_t x = 0; x < n; ++x) {
         w[x] = bf16_to_f64(q[x]);
-        w[n + x] = bf16_to_f64(k[x]);
-        w[2 * n + x] = bf16_to_f64(v[x]);
-        w[3 * n + x] = bf16_to_f64(dout[x]);
+        w[n + x] = bf16_to_f64(dout[x]);
     }
-    int rc = oracle_prefill_bwd_f64(w, w + n, w + 2 * n, w + 3 * n, cu_seqlens, past_lens, B, H, D, scale,
-                                    cand_self, dq, dk, dv);
+    for (size_t x = 0; x < m; ++x) {
+        w[2 * n + x] = bf16_to_f64(k[x]);
+        w[2 * n + m + x] = bf16_to_f64(v[x]);
+    }
+    int rc = oracle_prefill_bwd_f64(w, w + 2 * n, w + 2 * n + m, w + n, cu_seqlens, past_lens, B, H, Hkv, D,
+                                    scale, cand_self, dq, dk, dv);
     free(w);
     return rc;
 }
