@@ -533,6 +533,32 @@ def run_sweep(device, peaks, iters=10, warm=3):
         del q, k, v, o, kw
         torch.cuda.empty_cache()
 
+    # gradients of the prefill workload (B=64, n=256, k=128, D=64): forward with its row
+    # statistic once, then the backward call timed; FLOPs = 10*D per allowed pair (S, dP,
+    # dV, dK, dQ products)
+    w = synth.workload("prefill_B64")
+    past = np.full(w.B, w.n, np.int32)
+    cand = np.full(w.B, w.k, np.int32)
+    T = int((past + cand).sum())
+    q, k, v, g = (randn((T, w.H, w.D), w.seed + j) for j in range(4))
+    cu = torch.from_numpy(synth.cu_from_lens(past + cand)).to(device)
+    pl = torch.from_numpy(past).to(device)
+    lse = torch.empty((T, w.H), dtype=torch.float32, device=device)
+    o = ub.masked_prefill_attn(q, k, v, cu, pl, w.n + w.k, out_fp32=False, lse=lse, dev_status=status)
+    grads = [torch.empty((T, w.H, w.D), dtype=torch.float32, device=device) for _ in range(3)]
+    wsb = torch.empty(ub.masked_prefill_bwd_workspace_size(T, w.H) // 4 + 4, dtype=torch.float32, device=device)
+
+    def fn_bwd():
+        ub.masked_prefill_bwd(q, k, v, o, g, lse, cu, pl, w.n + w.k, dq=grads[0], dk=grads[1], dv=grads[2],
+                              workspace=wsb, dev_status=status, stream=stream)
+
+    ms = timed(fn_bwd)
+    flops = 2.5 * prefill_flops(past, cand, w.H, w.D)
+    nbytes = 5 * T * w.H * w.D * 2 + 3 * T * w.H * w.D * 4 + 2 * T * w.H * 4
+    e = roof_entry(ms, flops, nbytes, peaks, "bwd_prep_kernel<64> + bwd_kv_kernel<64>")
+    out["backward_B64_n256_k128_D64"] = e
+    del q, k, v, g, o, grads, lse
+
     # rank decode from the [12, 256, 8, 2048, 64] pool, 32 requests, every layer per step
     w = synth.workload("decode_R32")
     pk = randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed)
@@ -556,8 +582,9 @@ def run_sweep(device, peaks, iters=10, warm=3):
                                     out_fp32=False, workspace=ws, dev_status=status, stream=stream)
 
         ms = timed(fn) / w.L
-        kernel = ("decode_smallk_kernel<%d,%d>" % (w.D, 16 if kk <= 16 else 32 if kk <= 32 else 64 if kk <= 64
-                                                     else 128)) if kk <= 128 else "attn_fwd_kernel<%d,decode>" % w.D
+        # the library sends requests of at most 64 candidates (one query head per kv head) to the small-k kernel
+        kernel = ("decode_smallk_kernel<%d,%d>" % (w.D, 16 if kk <= 16 else 32 if kk <= 32 else 64)
+                  if kk <= 64 else "attn_fwd_kernel<%d,decode>" % w.D)
         e = roof_entry(ms, decode_flops(past, cand, w.H, w.D), decode_bytes(past, cand, w.H, w.D, 2), peaks, kernel)
         e["candidates_per_s"] = float(Tc) / (ms * 1e-3)
         e["ms_per_12_layers"] = ms * w.L

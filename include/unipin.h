@@ -20,6 +20,10 @@
  *   - Ragged batches use int32 offset arrays in device memory: cu_seqlens of
  *     length B+1 (segment b = tokens cu_seqlens[b] .. cu_seqlens[b+1]-1).
  *   - Supported head dims: D in {32, 64, 128}.
+ *   - Heads: queries have H heads, keys and values H_kv heads with H a multiple
+ *     of H_kv; query head h reads key/value head h / (H / H_kv) (grouped-query
+ *     attention; H_kv = H is plain multi-head attention).  [notes] §6 names the
+ *     pool's H "KV heads": the pool has H_kv heads.
  *   - Every call is asynchronous on `stream` (a cudaStream_t, NULL = the
  *     legacy default stream), does no host synchronisation, allocates
  *     nothing and keeps no pointer after it returns.  The first call of each
@@ -79,7 +83,8 @@ typedef struct {
  *   fp32 scores, fp32 online softmax and fp32 accumulation (P rounded to bf16
  *   for the P.V product).
  *
- *   q, k, v        [T, H, D] bf16, T = total_tokens = cu_seqlens[B]
+ *   q              [T, H, D] bf16, T = total_tokens = cu_seqlens[B]
+ *   k, v           [T, H_kv, D] bf16
  *   out            [T, H, D], fp32 if out_fp32 != 0 else bf16 (round to nearest even)
  *   lse            optional fp32 [T, H] (NULL: not written): per row and head the
  *                  log-sum-exp of its scores in base-2 units,
@@ -89,9 +94,10 @@ typedef struct {
  *   cu_seqlens     device int32 [B+1]; past_lens device int32 [B], 0 <= n_b <= len_b
  *   max_seqlen     host int >= every len_b (sizes the grid; a longer segment is a device error)
  *   scale          softmax scale, normally 1/sqrt(D)
- *   pool, slot_ids optional (pool == NULL: no pool write).  When given, the
- *                  past K/V of segment b is also written to pool rows
- *                  [layer, slot_ids[b], h, 0:n_b) exactly as unipin_kvpool_write does.
+ *   pool, slot_ids optional (pool == NULL: no pool write).  When given (pool->H ==
+ *                  H_kv), the past K/V of segment b is also written to pool rows
+ *                  [layer, slot_ids[b], h, 0:n_b) exactly as unipin_kvpool_write does,
+ *                  by the same kernel from the K/V tiles it loads anyway.
  *   workspace      optional device scratch, 16-byte aligned (NULL allowed).  With at
  *                  least unipin_masked_prefill_workspace_size() bytes, the persistent
  *                  thread blocks take (segment, head, query-tile pair) work items from
@@ -101,7 +107,7 @@ typedef struct {
  * Returns UNIPIN_OK or a negative unipin_status.
  */
 int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32, float* lse,
-                               const int* cu_seqlens, const int* past_lens, int B, int H, int D,
+                               const int* cu_seqlens, const int* past_lens, int B, int H, int H_kv, int D,
                                int max_seqlen, int total_tokens, float scale, const unipin_kvpool* pool,
                                const int* slot_ids, int layer, void* workspace, size_t workspace_bytes,
                                int* dev_status, void* stream);
@@ -122,11 +128,12 @@ size_t unipin_masked_prefill_workspace_size(void);
  * rows and from every candidate row of its segment, a candidate's own key and
  * value only from its own row.  Scores, probabilities and accumulation are
  * fp32; P and dS are rounded to bf16 as tensor-core operands.
- *   q, k, v        [T, H, D] bf16, the forward's inputs
+ *   q              [T, H, D] bf16; k, v [T, H_kv, D] bf16: the forward's inputs
  *   out            [T, H, D] bf16, the forward's output (bf16 mode)
  *   dout           [T, H, D] bf16, the gradient with respect to out
  *   lse            fp32 [T, H] as written by unipin_masked_prefill_attn
- *   dq, dk, dv     fp32 [T, H, D] outputs, written in full (dq is accumulated
+ *   dq             fp32 [T, H, D], dk and dv fp32 [T, H_kv, D] (a key/value head
+ *                  sums its query heads' gradients); written in full (dq is accumulated
  *                  across key tiles with atomic adds, so its low bits depend on
  *                  their order)
  *   D              32 or 64 (UNIPIN_ERR_UNSUPPORTED otherwise)
@@ -138,8 +145,9 @@ size_t unipin_masked_prefill_workspace_size(void);
  */
 int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                               const float* lse, float* dq, float* dk, float* dv, const int* cu_seqlens,
-                              const int* past_lens, int B, int H, int D, int max_seqlen, int total_tokens,
-                              float scale, void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
+                              const int* past_lens, int B, int H, int H_kv, int D, int max_seqlen,
+                              int total_tokens, float scale, void* workspace, size_t workspace_bytes,
+                              int* dev_status, void* stream);
 
 /* Bytes of workspace unipin_masked_prefill_bwd needs: 4 * total_tokens * H, rounded up to 16. */
 size_t unipin_masked_prefill_bwd_workspace_size(int total_tokens, int H);
@@ -168,13 +176,16 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
  * to pool rows 0..n_r-1 of that slot and to itself (its own k_c, v_c) - the
  * same mask as the candidate rows of the prefill, so it returns what the
  * prefill returns for those rows.
- *   q_c, k_c, v_c  [T_c, H, D] bf16, T_c = total_cand = cu_seqlens_c[R]
+ *   q_c            [T_c, H, D] bf16, T_c = total_cand = cu_seqlens_c[R]
+ *   k_c, v_c       [T_c, pool->H, D] bf16 (the candidates' own keys and values;
+ *                  H must be a multiple of the pool's key/value heads)
  *   out            [T_c, H, D], fp32 if out_fp32 else bf16
  *   max_k          host int >= every k_r (sizes the grid and picks the kernel: with
- *                  max_k <= 128 and D in {64, 128} the pool keys are the tensor-core
- *                  M dimension and a request's key range is swept by several thread
- *                  blocks, the bandwidth-bound case; otherwise 128-candidate query
- *                  tiles run through the prefill engine)
+ *                  max_k * G <= 128 (G = H / pool->H) and D in {64, 128} the pool keys
+ *                  are the tensor-core M dimension, the G query heads of a key/value
+ *                  head share one sweep of its history, and a request's key range is
+ *                  swept by several thread blocks, the bandwidth-bound case;
+ *                  otherwise 128-candidate query tiles run through the prefill engine)
  *   workspace      optional device scratch, 16-byte aligned (NULL allowed).  With at
  *                  least 256 bytes the blocks take work items from a shared counter
  *                  (zeroed by the call on `stream`); with at least
@@ -197,7 +208,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
  * split-n partial results (and, for max_k <= 128, one arrival counter per
  * request and head) when it would split.  The split grows with the device's
  * SM count; the size returned covers the current device and a 148-SM B200. */
-size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap);
+size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_k, int total_cand, int n_cap);
 
 /*
  * Rank decode that allocates nothing and takes no workspace.  There is no
@@ -210,8 +221,8 @@ size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int tot
  * counters) lives in a device array of unipin_rank_decode_noalloc_scratch_bytes()
  * bytes (32 MiB) that the library reserves on every device it is loaded on
  * and keeps until the process exits.
- *   - If unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand,
- *     pool->n_cap) exceeds that size, nothing is launched and
+ *   - If unipin_rank_decode_workspace_size(R, H, pool->H, D, max_k,
+ *     total_cand, pool->n_cap) exceeds that size, nothing is launched and
  *     UNIPIN_ERR_OUT_OF_RANGE is returned.
  *   - The first call on a device looks up the array's device address; make
  *     that first call before any stream capture.

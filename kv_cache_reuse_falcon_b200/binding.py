@@ -77,8 +77,8 @@ def _load(path: str = _LIB_PATH):
                           "python kv_cache_reuse_falcon_b200/build.py): %s" % path)
     lib = ctypes.CDLL(path)
     P, I, F, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, F, P, P, I, P, SZ, P, P]
-    lib.unipin_masked_prefill_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, SZ, P, P]
+    lib.unipin_masked_prefill_attn.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, I, F, P, P, I, P, SZ, P, P]
+    lib.unipin_masked_prefill_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, SZ, P, P]
     lib.unipin_masked_prefill_bwd.restype = I
     lib.unipin_masked_prefill_bwd_workspace_size.argtypes = [I, I]
     lib.unipin_masked_prefill_bwd_workspace_size.restype = SZ
@@ -89,7 +89,7 @@ def _load(path: str = _LIB_PATH):
     lib.unipin_kvpool_write.restype = I
     lib.unipin_rank_decode_attn.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, F, P, I, P, SZ, P, P]
     lib.unipin_rank_decode_attn.restype = I
-    lib.unipin_rank_decode_workspace_size.argtypes = [I, I, I, I, I, I]
+    lib.unipin_rank_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.unipin_rank_decode_workspace_size.restype = SZ
     lib.unipin_status_string.argtypes = [I]
     lib.unipin_status_string.restype = ctypes.c_char_p
@@ -145,6 +145,15 @@ def _tokens(t: torch.Tensor, name: str, D: Optional[int] = None):
         raise ValueError("%s has head dim %d, expected %d" % (name, t.shape[2], D))
 
 
+def _kv_heads(q, k, v) -> int:
+    """Key/value heads of grouped-query inputs (k and v [T, H_kv, D], H a multiple of H_kv)."""
+    if k.shape != v.shape or k.shape[0] != q.shape[0]:
+        raise ValueError("k and v must be [T, H_kv, D] with the tokens of q")
+    if q.shape[1] % k.shape[1] != 0:
+        raise ValueError("query heads (%d) must be a multiple of key/value heads (%d)" % (q.shape[1], k.shape[1]))
+    return int(k.shape[1])
+
+
 def _index(t: torch.Tensor, name: str, n: int):
     if t.dtype != torch.int32 or t.dim() != 1 or t.shape[0] != n or not t.is_contiguous() or not t.is_cuda:
         raise ValueError("%s must be a contiguous CUDA int32 tensor of length %d" % (name, n))
@@ -188,6 +197,7 @@ def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=Non
     T, H, D = q.shape
     _tokens(k, "k", D)
     _tokens(v, "v", D)
+    H_kv = _kv_heads(q, k, v)
     B = past_lens.shape[0]
     _index(cu_seqlens, "cu_seqlens", B + 1)
     _index(past_lens, "past_lens", B)
@@ -204,7 +214,7 @@ def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=Non
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     ws, ws_bytes = _workspace(workspace, masked_prefill_workspace_size(), q.device)
     rc = LIB.unipin_masked_prefill_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), int(bool(out_fp32)), _ptr(lse),
-                                        _ptr(cu_seqlens), _ptr(past_lens), B, H, D, int(max_seqlen), T, scale,
+                                        _ptr(cu_seqlens), _ptr(past_lens), B, H, H_kv, D, int(max_seqlen), T, scale,
                                         ctypes.byref(pool) if pool is not None else None,
                                         _ptr(slot_ids) if pool is not None else None, int(layer),
                                         _ptr(ws), ws_bytes, _ptr(dev_status), _stream(stream))
@@ -225,23 +235,24 @@ def masked_prefill_bwd(q, k, v, out, dout, lse, cu_seqlens, past_lens, max_seqle
     T, H, D = q.shape
     for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout)):
         _tokens(t, name, D)
+    H_kv = _kv_heads(q, k, v)
     if lse.dtype != torch.float32 or lse.shape != (T, H) or not lse.is_contiguous():
         raise ValueError("lse must be a contiguous float32 tensor [T, H]")
     B = past_lens.shape[0]
     _index(cu_seqlens, "cu_seqlens", B + 1)
     _index(past_lens, "past_lens", B)
     grads = []
-    for g in (dq, dk, dv):
+    for g, heads in ((dq, H), (dk, H_kv), (dv, H_kv)):
         if g is None:
-            g = torch.empty((T, H, D), dtype=torch.float32, device=q.device)
-        elif g.dtype != torch.float32 or g.shape != q.shape or not g.is_contiguous():
-            raise ValueError("gradient outputs must be contiguous float32 [T, H, D]")
+            g = torch.empty((T, heads, D), dtype=torch.float32, device=q.device)
+        elif g.dtype != torch.float32 or tuple(g.shape) != (T, heads, D) or not g.is_contiguous():
+            raise ValueError("gradient outputs must be contiguous float32: dq [T, H, D], dk and dv [T, H_kv, D]")
         grads.append(g)
     ws, ws_bytes = _workspace(workspace, masked_prefill_bwd_workspace_size(T, H), q.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     rc = LIB.unipin_masked_prefill_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
                                        _ptr(grads[0]), _ptr(grads[1]), _ptr(grads[2]), _ptr(cu_seqlens),
-                                       _ptr(past_lens), B, H, D, int(max_seqlen), T, scale, _ptr(ws), ws_bytes,
+                                       _ptr(past_lens), B, H, H_kv, D, int(max_seqlen), T, scale, _ptr(ws), ws_bytes,
                                        _ptr(dev_status), _stream(stream))
     _check(rc, "unipin_masked_prefill_bwd")
     return tuple(grads)
@@ -263,8 +274,11 @@ def kvpool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_i
     _check(rc, "unipin_kvpool_write")
 
 
-def rank_decode_workspace_size(R: int, H: int, D: int, max_k: int, total_cand: int, n_cap: int) -> int:
-    return int(LIB.unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand, n_cap))
+def rank_decode_workspace_size(R: int, H: int, D: int, max_k: int, total_cand: int, n_cap: int,
+                               H_kv: Optional[int] = None) -> int:
+    """Workspace bytes of rank_decode_attn; H are query heads, H_kv the pool's key/value heads (default H)."""
+    return int(LIB.unipin_rank_decode_workspace_size(R, H, H if H_kv is None else int(H_kv), D, max_k, total_cand,
+                                                      n_cap))
 
 
 def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, pool_v, layer: int, max_k: int,
@@ -276,6 +290,8 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
     _tokens(k_c, "k_c", D)
     _tokens(v_c, "v_c", D)
     pool = _pool(pool_k, pool_v)
+    if _kv_heads(q_c, k_c, v_c) != pool.H:
+        raise ValueError("k_c and v_c must have the pool's %d key/value heads" % pool.H)
     R = past_lens.shape[0]
     _index(cu_seqlens_c, "cu_seqlens_c", R + 1)
     _index(slot_ids, "slot_ids", R)
@@ -284,7 +300,7 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
         out = torch.empty((T, H, D), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q_c.device)
     elif out.dtype != (torch.float32 if out_fp32 else torch.bfloat16) or out.shape != q_c.shape or not out.is_contiguous():
         raise ValueError("out has the wrong dtype or shape")
-    ws, ws_bytes = _workspace(workspace, rank_decode_workspace_size(R, H, D, int(max_k), T, pool.n_cap)
+    ws, ws_bytes = _workspace(workspace, rank_decode_workspace_size(R, H, D, int(max_k), T, pool.n_cap, pool.H)
                               if isinstance(workspace, str) else 0, q_c.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     rc = LIB.unipin_rank_decode_attn(_ptr(q_c), _ptr(k_c), _ptr(v_c), _ptr(out), int(bool(out_fp32)),
@@ -309,6 +325,8 @@ def rank_decode_attn_noalloc(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, p
     _tokens(k_c, "k_c", D)
     _tokens(v_c, "v_c", D)
     pool = _pool(pool_k, pool_v)
+    if _kv_heads(q_c, k_c, v_c) != pool.H:
+        raise ValueError("k_c and v_c must have the pool's %d key/value heads" % pool.H)
     R = past_lens.shape[0]
     _index(cu_seqlens_c, "cu_seqlens_c", R + 1)
     _index(slot_ids, "slot_ids", R)

@@ -123,7 +123,8 @@ struct AttnParams {
     const int* past;              // [nseg]
     const int* slots;             // [nseg] (decode)
     int nseg;
-    int H;
+    int H;                        // query heads
+    int G;                        // query heads per key/value head (H = G * key/value heads)
     int max_rows;                 // host bound on rows per segment
     int total_rows;               // T
     int out_fp32;
@@ -281,8 +282,8 @@ __device__ __forceinline__ Work make_work(const AttnParams& p, int seg, int loca
     w.nt = w.valid ? max(w.nt_a, w.nt_b) : 0;
     if (!w.valid) w.nt_a = w.nt_b = 0;
     // The segment's last pair sees every past key (kmax = npast) and is its first item.
-    w.store = !kDecode && p.store_pool && w.valid && pair_rank == 0 && w.slot >= 0 && w.slot < p.S &&
-              w.npast <= p.n_cap;
+    w.store = !kDecode && p.store_pool && w.valid && pair_rank == 0 && (w.h % p.G) == 0 && w.slot >= 0 &&
+              w.slot < p.S && w.npast <= p.n_cap;
     return w;
 }
 
@@ -431,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     w.tok0 + w.qrow0 + x * kBlockM);
             }
             ++nq;
-            const int pool_plane = (p.layer * p.S + w.slot) * p.H + w.h;
+            const int hkv = w.h / p.G;   // the key/value head query head w.h reads
+            const int pool_plane = (p.layer * p.S + w.slot) * (p.H / p.G) + hkv;
             for (int i = 0; ok && i < w.nt; ++i) {      // K_i and V_i into one slot
                 int start, lo;
                 key_tile<C::kN>(w.t_begin + i, w.nt_all, w.kmax, start, lo);
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 tma_load_3d(dst + c * C::kAtomKV, map, kv_full + st, c * C::kBoxD, start,
                                             pool_plane);
                             else
-                                tma_load_3d(dst + c * C::kAtomKV, map, kv_full + st, c * C::kBoxD, w.h,
+                                tma_load_3d(dst + c * C::kAtomKV, map, kv_full + st, c * C::kBoxD, hkv,
                                             w.tok0 + start);
                         }
                     }
@@ -487,9 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         while (pop_item(ok)) {
             const Work w = make_work<kDecode, C::kN>(p, seg, local);
-            if (!kDecode && p.store_pool && w.valid && (local / p.H) == 0 && !w.store && leader)
+            if (!kDecode && p.store_pool && w.valid && (local / p.H) == 0 && (w.h % p.G) == 0 && !w.store &&
+                leader)
                 report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);   // slot id or history length beyond the pool
-            const int plane = (p.layer * p.S + w.slot) * p.H + w.h;
+            const int plane = (p.layer * p.S + w.slot) * (p.H / p.G) + w.h / p.G;
             for (int i = 0; i < w.nt; ++i, ++u) {
                 const int st = u % NS;
                 ok = __all_sync(0xffffffffu, mbar_wait(kv_full + st, (u / NS) & 1, ctl));
@@ -708,13 +711,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool row_valid = r < nrows_x;
             const long long tok = (long long)w.tok0 + w.qrow0 + x * kBlockM + r;
             const size_t base = ((size_t)tok * p.H + w.h) * D;
+            const size_t base_kv = ((size_t)tok * (p.H / p.G) + w.h / p.G) * D;   // the row's own key/value
             // self term: a candidate row's own key (prefill rows i >= n_b; every decode row)
             const bool self = row_valid && !split_mode && (kDecode || irow >= w.npast);
             float ss = -INFINITY;
             if (self) {
                 // issued before the first S wait so its latency overlaps the MMAs
                 const uint4* q4 = reinterpret_cast<const uint4*>(p.q + base);
-                const uint4* k4 = reinterpret_cast<const uint4*>(p.k_self + base);
+                const uint4* k4 = reinterpret_cast<const uint4*>(p.k_self + base_kv);
                 float dot0 = 0.f, dot1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
@@ -850,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // ---- epilogue: the own value (self term) is fetched before waiting for O
             uint4 vr[D / 8];
             {
-                const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + base);
+                const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + base_kv);
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) vr[c] = self ? __ldg(v4 + c) : make_uint4(0u, 0u, 0u, 0u);
             }
@@ -948,19 +952,21 @@ __global__ void __launch_bounds__(256)
     decode_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_ml,
                         const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k_self,
                         const __nv_bfloat16* __restrict__ v_self, void* out, int out_fp32, int total_rows, int H,
-                        int nsplit, float sl2)
+                        int G, int nsplit, float sl2)
 {
     constexpr int E = D / 32;   // elements per lane
     const int lane = threadIdx.x % 32;
     const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;   // tok * H + h
     if (row >= (long long)total_rows * H) return;
     const size_t base = (size_t)row * D + lane * E;
+    // the row's own key/value: token row / H, key/value head (row % H) / G
+    const size_t base_kv = ((size_t)(row / H) * (H / G) + (row % H) / G) * D + lane * E;
     float dot = 0.f;
     float vv[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        dot = fmaf(__bfloat162float(q[base + e]), __bfloat162float(k_self[base + e]), dot);
-        vv[e] = __bfloat162float(v_self[base + e]);
+        dot = fmaf(__bfloat162float(q[base + e]), __bfloat162float(k_self[base_kv + e]), dot);
+        vv[e] = __bfloat162float(v_self[base_kv + e]);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);

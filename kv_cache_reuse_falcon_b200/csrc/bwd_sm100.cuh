@@ -10,12 +10,15 @@
 //   dK_j   = scale * sum_i dS_ij q_i
 //   dQ_i   = scale * sum_j dS_ij k_j
 // over the allowed pairs.  Two kernels:
-//   bwd_prep_kernel  one warp per (token, head): Dvec_i, and for a candidate
-//       row its own key (the diagonal of the candidate block) entirely - it is
-//       the only row that sees that key, so dK and dV of a candidate come
-//       from here alone - plus that term's share of dQ; a past row's dQ
-//       starts at zero.
-//   bwd_kv_kernel    one block per (segment, head, tile of 128 past keys):
+//   bwd_prep_kernel  one warp per (token, key/value head): Dvec_i of each of
+//       its G query heads, and for a candidate row its own key (the diagonal
+//       of the candidate block) entirely - it is the only row that sees that
+//       key, so dK and dV of a candidate come from here alone, summed over
+//       the group - plus that term's share of dQ; a past row's dQ starts at
+//       zero.
+//   bwd_kv_kernel    one block per (segment, key/value head, tile of 128 past
+//       keys), sweeping the query tiles of each of the G query heads in turn
+//       (dK and dV of the tile accumulate over all of them):
 //       K and V of the tile stay in shared memory while the block sweeps the
 //       128-row query tiles that see them (from the tile's own rows to the
 //       segment end; past rows causally, every candidate row fully), with
@@ -79,7 +82,8 @@ struct BwParams {
     float* dvec;                // [T, H] workspace
     const int* cu;
     const int* past;
-    int B, H, total_rows, max_rows;
+    int B, H, total_rows, max_rows;   // H: query heads
+    int G;                            // query heads per key/value head
     float scale, sl2;
     int* status;
     unsigned long long wait_limit_ns;
@@ -95,15 +99,17 @@ __device__ __forceinline__ bool bw_segment_ok(const BwParams& p, int b, int& tok
            npast >= 0 && npast <= len;
 }
 
-// One warp per (token, head): Dvec, the candidate self term, dQ initialisation.
+// One warp per (token, key/value head): Dvec, the candidate self term, dQ initialisation.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwParams p)
 {
     constexpr int E = D / 32;
     const int lane = threadIdx.x % 32;
-    const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;   // token * H + head
-    if (row >= (long long)p.total_rows * p.H) return;
-    const long long t = row / p.H;
+    const int hkv = p.H / p.G;
+    const long long row = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;   // token * hkv + kv head
+    if (row >= (long long)p.total_rows * hkv) return;
+    const long long t = row / hkv;
+    const int hk = (int)(row - t * hkv);
     // segment of token t: the last b with cu[b] <= t
     int lo = 0, hi = p.B - 1;
     while (lo < hi) {
@@ -112,39 +118,54 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const BwParams p)
     }
     int tok0, len, npast;
     const bool ok = bw_segment_ok(p, lo, tok0, len, npast) && t >= tok0 && t < (long long)tok0 + len;
-    const size_t base = (size_t)row * D + lane * E;
-    float o[E], g[E], qv[E], kv[E], vv[E];
-    float dvec = 0.f, qk = 0.f, gv = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-        o[e] = __bfloat162float(p.o[base + e]);
-        g[e] = __bfloat162float(p.dout[base + e]);
-        qv[e] = __bfloat162float(p.q[base + e]);
-        kv[e] = __bfloat162float(p.k[base + e]);
-        vv[e] = __bfloat162float(p.v[base + e]);
-        dvec = fmaf(g[e], o[e], dvec);
-        qk = fmaf(qv[e], kv[e], qk);
-        gv = fmaf(g[e], vv[e], gv);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        dvec += __shfl_xor_sync(0xffffffffu, dvec, off);
-        qk += __shfl_xor_sync(0xffffffffu, qk, off);
-        gv += __shfl_xor_sync(0xffffffffu, gv, off);
-    }
-    if (lane == 0) p.dvec[row] = dvec;
     const bool cand = ok && (t - tok0) >= npast;
-    float pq = 0.f, ds = 0.f;
-    if (cand) {
-        pq = ex2_approx(qk * p.sl2 - p.lse[row]);   // the row's weight on its own key
-        ds = pq * (gv - dvec);
-    }
+    const size_t kbase = (size_t)row * D + lane * E;
+    float kv[E], vv[E], dk[E], dv[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-        p.dq[base + e] = cand ? p.scale * ds * kv[e] : 0.f;
-        if (cand || !ok) {                            // past keys of a valid segment: bwd_kv_kernel
-            p.dk[base + e] = cand ? p.scale * ds * qv[e] : 0.f;
-            p.dv[base + e] = cand ? pq * g[e] : 0.f;
+        kv[e] = __bfloat162float(p.k[kbase + e]);
+        vv[e] = __bfloat162float(p.v[kbase + e]);
+        dk[e] = 0.f;
+        dv[e] = 0.f;
+    }
+    for (int g = 0; g < p.G; ++g) {
+        const long long qr = t * p.H + (long long)hk * p.G + g;   // query row (token, query head)
+        const size_t base = (size_t)qr * D + lane * E;
+        float o[E], gd[E], qv[E];
+        float dvec = 0.f, qk = 0.f, gv = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            o[e] = __bfloat162float(p.o[base + e]);
+            gd[e] = __bfloat162float(p.dout[base + e]);
+            qv[e] = __bfloat162float(p.q[base + e]);
+            dvec = fmaf(gd[e], o[e], dvec);
+            qk = fmaf(qv[e], kv[e], qk);
+            gv = fmaf(gd[e], vv[e], gv);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            dvec += __shfl_xor_sync(0xffffffffu, dvec, off);
+            qk += __shfl_xor_sync(0xffffffffu, qk, off);
+            gv += __shfl_xor_sync(0xffffffffu, gv, off);
+        }
+        if (lane == 0) p.dvec[qr] = dvec;
+        float pq = 0.f, ds = 0.f;
+        if (cand) {
+            pq = ex2_approx(qk * p.sl2 - p.lse[qr]);   // the row's weight on its own key
+            ds = pq * (gv - dvec);
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            p.dq[base + e] = cand ? p.scale * ds * kv[e] : 0.f;
+            dk[e] = fmaf(p.scale * ds, qv[e], dk[e]);
+            dv[e] = fmaf(pq, gd[e], dv[e]);
+        }
+    }
+    if (cand || !ok) {                            // past keys of a valid segment: bwd_kv_kernel
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            p.dk[kbase + e] = dk[e];
+            p.dv[kbase + e] = dv[e];
         }
     }
     if (!ok && lane == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
@@ -167,11 +188,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
 
-    // item: key tile kt of (segment b, head h); key-tile-major so the longest sweeps start first
-    const int bh_count = p.B * p.H;
+    // item: key tile kt of (segment b, key/value head h); key-tile-major so the longest sweeps start first
+    const int hkv = p.H / p.G;
+    const int bh_count = p.B * hkv;
     const int kt = blockIdx.x / bh_count;
     const int bh = blockIdx.x - kt * bh_count;
-    const int b = bh / p.H, h = bh - (bh / p.H) * p.H;
+    const int b = bh / hkv, h = bh - (bh / hkv) * hkv;
     int tok0, len, npast;
     if (!bw_segment_ok(p, b, tok0, len, npast)) return;   // bwd_prep_kernel zeroed and reported it
     const int j0 = kt * kBwRows;
@@ -181,7 +203,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         if (threadIdx.x == 0) report(p.status, (int)UNIPIN_ERR_CUDA);
         return;
     }
-    const int nq = (len - j0 + kBwRows - 1) / kBwRows;   // query tiles kt .. kt + nq - 1
+    const int nqt = (len - j0 + kBwRows - 1) / kBwRows;   // query tiles kt .. kt + nqt - 1 of one query head
+    const int nq = nqt * p.G;                             // swept for each of the G query heads in turn
 
     uint8_t* sK = smem + C::kOffK;
     uint8_t* sV = smem + C::kOffV;
@@ -246,10 +269,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                 if (!ok) break;
             }
             if (leader) {
-                const int row0 = tok0 + j0 + qi * kBwRows;
+                const int row0 = tok0 + j0 + (qi % nqt) * kBwRows;
+                const int hq = h * p.G + qi / nqt;
                 mbar_arrive_expect_tx(bar_qdo + qb, 2 * C::kTile);
-                tma_load_3d(sQ + qb * C::kTile, &tm_q, bar_qdo + qb, 0, h, row0);
-                tma_load_3d(sDO + qb * C::kTile, &tm_do, bar_qdo + qb, 0, h, row0);
+                tma_load_3d(sQ + qb * C::kTile, &tm_q, bar_qdo + qb, 0, hq, row0);
+                tma_load_3d(sDO + qb * C::kTile, &tm_do, bar_qdo + qb, 0, hq, row0);
             }
         }
         if (leader) {
@@ -327,10 +351,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         bool ok = true;
         for (int qi = 0; qi < nq; ++qi) {
             const int sb = qi & 1;
-            const int qrow0 = j0 + qi * kBwRows;   // first query row of the tile (segment position)
+            const int qrow0 = j0 + (qi % nqt) * kBwRows;   // first query row of the tile (segment position)
+            const int hq = h * p.G + qi / nqt;              // its query head
             {
                 const int r = qrow0 + t;
-                const size_t idx = (size_t)(tok0 + r) * p.H + h;
+                const size_t idx = (size_t)(tok0 + r) * p.H + hq;
                 s_lse[sb * kBwRows + t] = r < len ? p.lse[idx] : 0.f;
                 s_dvec[sb * kBwRows + t] = r < len ? p.dvec[idx] : 0.f;
             }
@@ -389,7 +414,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             tc_fence_before_sync();
             const int row = qrow0 + t;
             if (row < len) {
-                float* dst = p.dq + ((size_t)(tok0 + row) * p.H + h) * D;
+                float* dst = p.dq + ((size_t)(tok0 + row) * p.H + hq) * D;
 #pragma unroll
                 for (int e = 0; e < D; e += 4)
                     red_add_v4(dst + e, p.scale * __uint_as_float(dqr[e]), p.scale * __uint_as_float(dqr[e + 1]),
@@ -403,7 +428,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             if constexpr (D == 64) tmem_ld64(lane_base + C::kColDK, g);
             else tmem_ld32(lane_base + C::kColDK, g);
             if (key_ok) {
-                float* dkd = p.dk + ((size_t)(tok0 + key) * p.H + h) * D;
+                float* dkd = p.dk + ((size_t)(tok0 + key) * hkv + h) * D;
 #pragma unroll
                 for (int e = 0; e < D; e += 4)
                     *reinterpret_cast<float4*>(dkd + e) =
@@ -413,7 +438,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             if constexpr (D == 64) tmem_ld64(lane_base + C::kColDV, g);
             else tmem_ld32(lane_base + C::kColDV, g);
             if (key_ok) {
-                float* dvd = p.dv + ((size_t)(tok0 + key) * p.H + h) * D;
+                float* dvd = p.dv + ((size_t)(tok0 + key) * hkv + h) * D;
 #pragma unroll
                 for (int e = 0; e < D; e += 4)
                     *reinterpret_cast<float4*>(dvd + e) = make_float4(__uint_as_float(g[e]), __uint_as_float(g[e + 1]),

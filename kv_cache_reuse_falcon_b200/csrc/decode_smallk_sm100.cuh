@@ -78,9 +78,9 @@ struct SkCfg {
     static constexpr int kColO = 2 * N;
     static constexpr int kTmemCols = sk_tmem_cols(2 * N + D);
     static constexpr int kCtasPerSm = (D == 64 && kTmemCols <= 256) ? 2 : 1;
-    // Scratch floats: red[4][N], mref[N], corr[N], coef_b[N], flags[2][4]; merge
-    // weights reuse a P buffer.
-    static constexpr int kScratchBytes = ((4 * N + 3 * N + 8) * 4 + 1023) / 1024 * 1024;
+    // Scratch floats: red[4][N], mref[N], corr[N], coef_b[N], flags[2][4],
+    // selfs[kSkItemSlots][N]; merge weights reuse a P buffer.
+    static constexpr int kScratchBytes = ((4 * N + 3 * N + 8 + kSkItemSlots * N) * 4 + 1023) / 1024 * 1024;
     static constexpr int kBarBytes = 1024;
     static constexpr int kBudget = kCtasPerSm == 2 ? 112 * 1024 : 226 * 1024;
     // Double-buffer Q (the next item's Q loads during this item) and P^T (the
@@ -118,7 +118,8 @@ struct SkParams {
     const int* cu;                 // [R + 1]
     const int* past;               // [R]
     const int* slots;              // [R]
-    int R, H;
+    int R, H;                      // requests, query heads
+    int G;                         // query heads per key/value head
     int total_rows;                // T
     int out_fp32;
     int layer, S, n_cap;
@@ -129,12 +130,15 @@ struct SkParams {
     unsigned long long* sched;     // zeroed item counter or null (static striding)
 };
 
-// What every role derives identically from an item index.
+// What every role derives identically from an item index.  An item is a
+// (request, key/value head, run of key tiles); its candidate columns are the
+// pairs (candidate c, query head g of the group) in the order n = c * G + g.
 struct SkWork {
-    bool rows_ok;   // the request's candidate rows are addressable (cu in range, k <= N)
+    bool rows_ok;   // the request's candidate rows are addressable (cu in range, k * G <= N)
     bool valid;     // rows_ok and slot / history length in range
-    int r, h, split, pair;
+    int r, h, split, pair;   // h: the key/value head
     int tok0, kc, npast, slot;
+    int ncol;                // valid candidate columns, kc * G
     int nt_all;     // key tiles covering [0, npast)
     int t_begin, nt;
 };
@@ -145,13 +149,15 @@ __device__ __forceinline__ SkWork sk_make_work(const SkParams& p, long long g)
     SkWork w;
     w.pair = (int)(g / p.nsplit);
     w.split = (int)(g - (long long)w.pair * p.nsplit);
-    w.r = w.pair / p.H;
-    w.h = w.pair - w.r * p.H;
+    const int hkv = p.H / p.G;
+    w.r = w.pair / hkv;
+    w.h = w.pair - w.r * hkv;
     w.tok0 = p.cu[w.r];
     w.kc = p.cu[w.r + 1] - w.tok0;
     w.npast = p.past[w.r];
     w.slot = p.slots[w.r];
-    w.rows_ok = w.tok0 >= 0 && w.kc >= 0 && w.kc <= N && (long long)w.tok0 + w.kc <= (long long)p.total_rows;
+    w.ncol = w.kc * p.G;
+    w.rows_ok = w.tok0 >= 0 && w.kc >= 0 && w.ncol <= N && (long long)w.tok0 + w.kc <= (long long)p.total_rows;
     w.valid = w.rows_ok && w.slot >= 0 && w.slot < p.S && w.npast >= 0 && w.npast <= p.n_cap;
     w.nt_all = w.valid ? (w.npast + kSkKeys - 1) / kSkKeys : 0;
     w.t_begin = min(w.split * p.tiles_per_split, w.nt_all);
@@ -273,6 +279,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     float* corr = mref + N;                                         // [N]
     float* coef_b = corr + N;                                       // [N] merge: weight of the own value
     volatile int* flags = reinterpret_cast<volatile int*>(coef_b + N);   // [2][4]
+    float* selfs = coef_b + N + 8;                                  // [kSkItemSlots][N] own scores, per item slot
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_q = bars + 0;            // [2] Q buffer landed
     uint64_t* q_empty = bars + 2;          // [2] the last S MMA of the item using Q buffer b finished
@@ -324,13 +331,16 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     const uint32_t tmem = *tmem_slot;
 
     WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
-    const long long total_items = (long long)p.R * p.H * p.nsplit;
+    const long long total_items = (long long)p.R * (p.H / p.G) * p.nsplit;
     int n_items = 0;
-    auto pop_item = [&](bool& ok, long long& g) -> bool {
+    // Consumers: the next item (warp-uniform); `own` receives selfs[slot][own_col] read
+    // before the slot is released (the producer may refill it right after).
+    auto pop_item = [&](bool& ok, long long& g, int own_col, float& own) -> bool {
         const int si = n_items % kSkItemSlots;
         ok = __all_sync(0xffffffffu, mbar_wait(item_full + si, (n_items / kSkItemSlots) & 1, ctl));
         if (!ok) return false;
         g = item_ring[si];
+        own = (own_col >= 0 && own_col < N) ? selfs[si * N + own_col] : -INFINITY;
         __syncwarp();
         if (lane == 0) mbar_arrive(item_empty + si);
         ++n_items;
@@ -363,13 +373,26 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 g_static += gridDim.x;
             }
             const bool found = g < total_items;
+            SkWork w;
+            if (found) {
+                // the own score of every candidate column (log2 units), off the softmax warps' path
+                w = sk_make_work<N>(p, g);
+                if (w.valid) {
+                    const int hkv = p.H / p.G;
+                    for (int n = lane; n < w.ncol; n += 32) {
+                        const size_t qrow = (size_t)(w.tok0 + n / p.G) * p.H + w.h * p.G + n % p.G;
+                        const size_t kvrow = (size_t)(w.tok0 + n / p.G) * hkv + w.h;
+                        selfs[si * N + n] = p.sl2 * sk_dot_bf16<D>(p.q + qrow * D, p.k_self + kvrow * D);
+                    }
+                }
+                __syncwarp();
+            }
             if (leader) {
                 item_ring[si] = found ? g : -1;
-                mbar_arrive(item_full + si);
+                mbar_arrive(item_full + si);   // release: the consumers see selfs[si] with the item
             }
             ++n_items;
             if (!found) break;
-            const SkWork w = sk_make_work<N>(p, g);
             if (w.nt == 0) continue;
             const int qb = nq % NQ;
             if (nq >= NQ) {
@@ -379,10 +402,11 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             if (leader) {
                 mbar_arrive_expect_tx(bar_q + qb, C::kQBytes);
                 for (int c = 0; c < C::kChunks; ++c)
-                    tma_load_3d(sQ + qb * C::kQBytes + c * C::kAtomQ, &tm_q, bar_q + qb, c * 64, w.h, w.tok0);
+                    // N / G candidate tokens x the G query heads of key/value head w.h
+                    tma_load_3d(sQ + qb * C::kQBytes + c * C::kAtomQ, &tm_q, bar_q + qb, c * 64, w.h * p.G, w.tok0);
             }
             ++nq;
-            const int plane = (p.layer * p.S + w.slot) * p.H + w.h;
+            const int plane = (p.layer * p.S + w.slot) * (p.H / p.G) + w.h;
             for (int i = 0; ok && i < w.nt; ++i) {
                 const int start = sk_tile_start(w.t_begin + i, w.nt_all, w.npast);
                 const int st = u % NS;
@@ -464,7 +488,8 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             tc_fence_after_sync();
             return r;
         };
-        while (pop_item(ok, g)) {
+        float unused_own;
+        while (pop_item(ok, g, -1, unused_own)) {
             const SkWork w = sk_make_work<N>(p, g);
             if (w.nt == 0) continue;
             const int qb = nq % NQ;
@@ -560,18 +585,20 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             tc_fence_after_sync();
             return r;
         };
-        while (pop_item(ok, g)) {
+        float own_popped;
+        while (pop_item(ok, g, threadIdx.x, own_popped)) {
             const SkWork w = sk_make_work<N>(p, g);
             if (!w.rows_ok) {
                 if (t == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
                 continue;
             }
             if (!w.valid && t == 0 && w.split == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
-            // Candidate t's own score (log2 units), taken while the item's first tile is in flight.
-            float ss_own = -INFINITY;
-            if (t < w.kc && w.valid)
-                ss_own = sl2 * sk_dot_bf16<D>(p.q + ((size_t)(w.tok0 + t) * p.H + w.h) * D,
-                                              p.k_self + ((size_t)(w.tok0 + t) * p.H + w.h) * D);
+            // Column t = (candidate t / G, query head w.h * G + t % G): its output row, its own
+            // key/value row, and its own score (log2 units), taken while the first tile is in flight.
+            const int hkv = p.H / p.G;
+            const size_t qrow = (size_t)(w.tok0 + t / p.G) * p.H + w.h * p.G + t % p.G;
+            const size_t kvrow = (size_t)(w.tok0 + t / p.G) * hkv + w.h;
+            const float ss_own = (t < w.ncol && w.valid) ? own_popped : -INFINITY;
             // per-thread partial column sums of P (owned columns), relative to mref
             constexpr int kOwn = N >= 32 ? N / 32 : 1;
             float lown[kOwn];
@@ -596,7 +623,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 float x[N];
 #pragma unroll
                 for (int c = 0; c < N; ++c)
-                    x[c] = (key_ok && c < w.kc) ? __uint_as_float(sraw[c]) * sl2 : -INFINITY;
+                    x[c] = (key_ok && c < w.ncol) ? __uint_as_float(sraw[c]) * sl2 : -INFINITY;
                 // vote: does any score exceed its candidate's reference max by > 2^8?
                 bool need = false;
 #pragma unroll
@@ -683,6 +710,15 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             }
             if (!ok) break;
             // ------------------------------------------------------ epilogue
+            // the own value row is fetched before the last wait, so its latency overlaps it
+            // (where registers allow: the widest variant keeps it in the store loop)
+            constexpr bool kPrefetchV = N <= 32;
+            uint4 vrow[kPrefetchV ? D / 8 : 1];
+            if (kPrefetchV && p.nsplit == 1 && t < w.ncol) {
+                const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + kvrow * D);
+#pragma unroll
+                for (int d8 = 0; d8 < D / 8; ++d8) vrow[d8] = __ldg(v4 + d8);
+            }
             if (w.nt > 0 && !(ok = wait_pv(gp - 1))) break;
 #pragma unroll
             for (int e = 0; e < kOwn; ++e)
@@ -694,7 +730,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 l_c = red[t] + red[N + t] + red[2 * N + t] + red[3 * N + t];
                 m_c = w.nt > 0 ? mref[t] : -INFINITY;
                 mref[t] = -INFINITY;   // ready for the next item
-                if (p.nsplit == 1 && t < w.kc && w.valid) {
+                if (p.nsplit == 1 && t < w.ncol && w.valid) {
                     // final: (a O + b v_self) / (a l + b)
                     const float mf = fmaxf(m_c, ss_own);
                     const float a = (m_c == -INFINITY) ? 0.f : ex2_approx(m_c - mf);
@@ -714,13 +750,14 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 for (int d = 0; d < D; ++d) o[d] = 0u;
             }
             tc_fence_before_sync();
-            if (t < w.kc) {
-                const size_t row = (size_t)(w.tok0 + t) * p.H + w.h;
+            if (t < w.ncol) {
+                const size_t row = qrow;
                 if (p.nsplit == 1) {
-                    const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + row * D);
 #pragma unroll
                     for (int d8 = 0; d8 < D / 8; ++d8) {
-                        const uint4 vb = __ldg(v4 + d8);
+                        uint4 vb;
+                        if constexpr (kPrefetchV) vb = vrow[d8];
+                        else vb = __ldg(reinterpret_cast<const uint4*>(p.v_self + kvrow * D) + d8);
                         const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vb);
                         float r[8];
 #pragma unroll
@@ -756,9 +793,9 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 if (*last_flag) {
                     __threadfence();
                     float* wts = reinterpret_cast<float*>(sP + (gp % NP) * C::kPBytes);   // [kSkMaxSplit][N]
-                    if (t < w.kc) {
+                    if (t < w.ncol) {
                         // weights of the splits and of the own key: LSE merge in log2 units
-                        const size_t row = (size_t)(w.tok0 + t) * p.H + w.h;
+                        const size_t row = qrow;
                         float ms[kSkMaxSplit], ls[kSkMaxSplit];
 #pragma unroll
                         for (int s = 0; s < kSkMaxSplit; ++s) {
@@ -791,7 +828,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                     // out = b v_self + sum_s w_s O_s, four head-dim elements per thread and step;
                     // four steps' loads are issued before their sums
                     constexpr int kQ = D / 4;
-                    const int total = w.kc * kQ;
+                    const int total = w.ncol * kQ;
                     const size_t split_stride = (size_t)p.total_rows * p.H * D;
                     for (int base = 0; base < total; base += 4 * 128) {
                         float4 acc[4];
@@ -803,10 +840,12 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                             const bool act = q < total;
                             cc[u] = act ? q / kQ : -1;
                             const int c = act ? cc[u] : 0;
-                            idx[u] = ((size_t)(w.tok0 + c) * p.H + w.h) * D + (q % kQ) * 4;
+                            // column c: candidate c / G, query head w.h * G + c % G
+                            idx[u] = ((size_t)(w.tok0 + c / p.G) * p.H + w.h * p.G + c % p.G) * D + (q % kQ) * 4;
+                            const size_t vidx = ((size_t)(w.tok0 + c / p.G) * hkv + w.h) * D + (q % kQ) * 4;
                             acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                             if (act) {
-                                const uint2 vb = __ldg(reinterpret_cast<const uint2*>(p.v_self + idx[u]));
+                                const uint2 vb = __ldg(reinterpret_cast<const uint2*>(p.v_self + vidx));
                                 const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.x));
                                 const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.y));
                                 const float cbv = coef_b[c];

@@ -103,7 +103,6 @@ int set_sk_attrs()
     int rc = set_sk_attr<D, 16>();
     if (rc == UNIPIN_OK) rc = set_sk_attr<D, 32>();
     if (rc == UNIPIN_OK) rc = set_sk_attr<D, 64>();
-    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 128>();
     return rc;
 }
 
@@ -162,13 +161,14 @@ int make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_
     return r == CUDA_SUCCESS ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 
-// Packed token tensor [T, H, D]: boxes of `rows` tokens x 1 head x (D or 64)
-// elements (128 query rows, or one key tile).
-int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D, int rows)
+// Packed token tensor [T, H, D]: boxes of `rows` tokens x `heads` heads x (D or
+// 64) elements (128 query rows, one key tile, or the candidates of a request
+// for a group of query heads).
+int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D, int rows, int heads = 1)
 {
     const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
-    return make_map(m, base, (uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)D * 2, (uint64_t)H * D * 2, box_d, 1,
-                    (uint32_t)rows, D);
+    return make_map(m, base, (uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)D * 2, (uint64_t)H * D * 2, box_d,
+                    (uint32_t)heads, (uint32_t)rows, D);
 }
 
 // Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of `rows` history rows of one plane.
@@ -181,10 +181,12 @@ int make_pool_map(CUtensorMap* m, const void* base, const unipin_kvpool* pool, i
                     (uint64_t)pool->n_cap * D * 2, box_d, (uint32_t)rows, 1, D);
 }
 
+// The pool's heads are key/value heads: H (query heads) must be a multiple of them.
 int check_pool(const unipin_kvpool* pool, int H, int D, int layer)
 {
     if (!pool || !pool->k || !pool->v) return UNIPIN_ERR_INVALID_ARG;
-    if (pool->L < 1 || pool->S < 1 || pool->n_cap < 1 || pool->H != H || pool->D != D) return UNIPIN_ERR_INVALID_ARG;
+    if (pool->L < 1 || pool->S < 1 || pool->n_cap < 1 || pool->H < 1 || H % pool->H != 0 || pool->D != D)
+        return UNIPIN_ERR_INVALID_ARG;
     if (!aligned16(pool->k) || !aligned16(pool->v)) return UNIPIN_ERR_MISALIGNED;
     if (layer < 0 || layer >= pool->L) return UNIPIN_ERR_OUT_OF_RANGE;
     if ((uint64_t)pool->L * pool->S * pool->H >= (1ull << 31)) return UNIPIN_ERR_INVALID_ARG;
@@ -268,10 +270,15 @@ size_t decode_workspace_bytes(int nsplit, int total_cand, int H, int D)
 
 // ---- small-k rank decode (keys as the MMA's M; decode_smallk_sm100.cuh)
 
-// Requests with at most this many candidates take the small-k kernel (D 64 or 128).
-constexpr int kSmallKMax = 128;
+// Requests with at most this many candidate columns (candidates x query heads per
+// key/value head) take the small-k kernel (D 64 or 128); beyond 64 columns the
+// many-candidate engine measured faster.
+constexpr int kSmallKMax = 64;
 
-bool use_small_k(int D, int max_k) { return (D == 64 || D == 128) && max_k >= 1 && max_k <= kSmallKMax; }
+bool use_small_k(int D, int max_k, int G)
+{
+    return (D == 64 || D == 128) && max_k >= 1 && (long long)max_k * G <= kSmallKMax && kSmallKMax % G == 0;
+}
 
 int sk_ctas_per_sm(int D, int N)
 {
@@ -279,15 +286,13 @@ int sk_ctas_per_sm(int D, int N)
         switch (N) {
         case 16: return SkCfg<64, 16>::kCtasPerSm;
         case 32: return SkCfg<64, 32>::kCtasPerSm;
-        case 64: return SkCfg<64, 64>::kCtasPerSm;
-        default: return SkCfg<64, 128>::kCtasPerSm;
+        default: return SkCfg<64, 64>::kCtasPerSm;
         }
     }
     switch (N) {
     case 16: return SkCfg<128, 16>::kCtasPerSm;
     case 32: return SkCfg<128, 32>::kCtasPerSm;
-    case 64: return SkCfg<128, 64>::kCtasPerSm;
-    default: return SkCfg<128, 128>::kCtasPerSm;
+    default: return SkCfg<128, 64>::kCtasPerSm;
     }
 }
 
@@ -310,13 +315,15 @@ struct SkPlan {
 // Key splits per (request, head): cut the pool sweep into runs of whole
 // 128-key tiles so that the grid gets about sk_items_per_block() items per
 // resident block, at most kSkMaxSplit runs.
-SkPlan sk_plan(int R, int H, int D, int max_k, int n_cap, int sms)
+// The candidate columns of an item are (candidate, query head of the group):
+// max_k * G of them; H_kv = H / G key/value heads make R * H_kv (request, head) pairs.
+SkPlan sk_plan(int R, int H_kv, int G, int D, int max_k, int n_cap, int sms)
 {
     SkPlan pl;
-    pl.N = sk_pad_n(max_k);
+    pl.N = sk_pad_n(max_k * G);
     pl.blocks_per_sm = sk_ctas_per_sm(D, pl.N);
     const long long tiles = (n_cap + kSkKeys - 1) / kSkKeys;
-    const long long pairs = (long long)R * H;
+    const long long pairs = (long long)R * H_kv;
     const long long target = (long long)sk_items_per_block() * sms * pl.blocks_per_sm;
     long long ns = (target + pairs - 1) / pairs;   // splits per (request, head) for the target item count
     if (ns > tiles) ns = tiles;
@@ -355,8 +362,7 @@ int launch_sk_d(int N, unsigned grid, const CUtensorMap& tq, const CUtensorMap& 
     switch (N) {
     case 16: return launch_sk_kernel<D, 16>(grid, tq, tk, tv, p, s);
     case 32: return launch_sk_kernel<D, 32>(grid, tq, tk, tv, p, s);
-    case 64: return launch_sk_kernel<D, 64>(grid, tq, tk, tv, p, s);
-    default: return launch_sk_kernel<D, 128>(grid, tq, tk, tv, p, s);
+    default: return launch_sk_kernel<D, 64>(grid, tq, tk, tv, p, s);
     }
 }
 
@@ -365,7 +371,8 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
                         int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer,
                         void* workspace, size_t workspace_bytes, int* dev_status, cudaStream_t s)
 {
-    SkPlan pl = sk_plan(R, H, D, max_k, pool->n_cap, current_sms());
+    const int G = H / pool->H;
+    SkPlan pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms());
     if (pl.nsplit > 1 && (!workspace || workspace_bytes < sk_workspace_bytes(pl, R, H, D, total_cand))) {
         pl.nsplit = 1;
         pl.tiles_per_split = (pool->n_cap + kSkKeys - 1) / kSkKeys;
@@ -378,7 +385,8 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
     }
     CUtensorMap tq, tk, tv;
     int rc;
-    if ((rc = make_token_map(&tq, q_c, total_cand, H, D, pl.N)) != UNIPIN_OK) return rc;
+    // the N candidate columns: N / G tokens x the G query heads of one key/value head
+    if ((rc = make_token_map(&tq, q_c, total_cand, H, D, pl.N / G, G)) != UNIPIN_OK) return rc;
     if ((rc = make_pool_map(&tk, pool->k, pool, kSkKeys)) != UNIPIN_OK) return rc;
     if ((rc = make_pool_map(&tv, pool->v, pool, kSkKeys)) != UNIPIN_OK) return rc;
 
@@ -392,6 +400,7 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
     p.slots = slot_ids;
     p.R = R;
     p.H = H;
+    p.G = G;
     p.total_rows = total_cand;
     p.out_fp32 = out_fp32 ? 1 : 0;
     p.layer = layer;
@@ -409,7 +418,7 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
         p.part_o = reinterpret_cast<float*>(ws + kSchedBytes + sk_counter_bytes(R, H));
         p.part_ml = p.part_o + (size_t)pl.nsplit * total_cand * H * D;
     }
-    const unsigned grid = persistent_blocks((long long)R * H * pl.nsplit, pl.blocks_per_sm);
+    const unsigned grid = persistent_blocks((long long)R * pool->H * pl.nsplit, pl.blocks_per_sm);
     return D == 64 ? launch_sk_d<64>(pl.N, grid, tq, tk, tv, p, s) : launch_sk_d<128>(pl.N, grid, tq, tk, tv, p, s);
 }
 
@@ -473,17 +482,19 @@ const char* unipin_status_string(int status)
 size_t unipin_masked_prefill_workspace_size(void) { return kSchedBytes; }
 
 int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void* out, int out_fp32, float* lse,
-                               const int* cu_seqlens, const int* past_lens, int B, int H, int D, int max_seqlen,
-                               int total_tokens, float scale, const unipin_kvpool* pool, const int* slot_ids,
-                               int layer, void* workspace, size_t workspace_bytes, int* dev_status, void* stream)
+                               const int* cu_seqlens, const int* past_lens, int B, int H, int H_kv, int D,
+                               int max_seqlen, int total_tokens, float scale, const unipin_kvpool* pool,
+                               const int* slot_ids, int layer, void* workspace, size_t workspace_bytes,
+                               int* dev_status, void* stream)
 {
-    if (B < 0 || H < 1 || max_seqlen < 0 || total_tokens < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (B < 0 || H < 1 || H_kv < 1 || H % H_kv != 0 || max_seqlen < 0 || total_tokens < 0)
+        return UNIPIN_ERR_INVALID_ARG;
     if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
     if (!(scale > 0.f) || !std::isfinite(scale)) return UNIPIN_ERR_INVALID_ARG;
     if (pool) {
         int rc = check_pool(pool, H, D, layer);
         if (rc != UNIPIN_OK) return rc;
-        if (!slot_ids) return UNIPIN_ERR_INVALID_ARG;
+        if (pool->H != H_kv || !slot_ids) return UNIPIN_ERR_INVALID_ARG;
     }
     if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
     if (!q || !k || !v || !out || !cu_seqlens || !past_lens) return UNIPIN_ERR_INVALID_ARG;
@@ -501,8 +512,8 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
 
     CUtensorMap tq, tk, tv, tpk, tpv;
     if ((rc = make_token_map(&tq, q, total_tokens, H, D, kBlockM)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tk, k, total_tokens, H, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tv, v, total_tokens, H, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tk, k, total_tokens, H_kv, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tv, v, total_tokens, H_kv, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
     if (pool) {
         // the past K/V tiles the kernel loads are also stored into the pool (no second pass)
         if ((rc = make_pool_map(&tpk, pool->k, pool, key_tile_width(D, false))) != UNIPIN_OK) return rc;
@@ -522,6 +533,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.slots = nullptr;
     p.nseg = B;
     p.H = H;
+    p.G = H / H_kv;
     p.max_rows = max_seqlen;
     p.total_rows = total_tokens;
     p.out_fp32 = out_fp32 ? 1 : 0;
@@ -565,12 +577,15 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
                              total_tokens, dev_status, static_cast<cudaStream_t>(stream));
 }
 
-size_t unipin_rank_decode_workspace_size(int R, int H, int D, int max_k, int total_cand, int n_cap)
+size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_k, int total_cand, int n_cap)
 {
-    if (R < 1 || H < 1 || !supported_d(D) || max_k < 1 || total_cand < 1 || n_cap < 1) return 0;
+    if (R < 1 || H < 1 || H_kv < 1 || H % H_kv != 0 || !supported_d(D) || max_k < 1 || total_cand < 1 || n_cap < 1)
+        return 0;
     // The split grows with the SM count: size for the larger of this device's and a B200's.
     const int sms = current_sms() > kNumSmsHint ? current_sms() : kNumSmsHint;
-    if (use_small_k(D, max_k)) return sk_workspace_bytes(sk_plan(R, H, D, max_k, n_cap, sms), R, H, D, total_cand);
+    const int G = H / H_kv;
+    if (use_small_k(D, max_k, G))
+        return sk_workspace_bytes(sk_plan(R, H_kv, G, D, max_k, n_cap, sms), R, H, D, total_cand);
     return decode_workspace_bytes(decode_nsplit(R, H, D, max_k, n_cap, sms), total_cand, H, D);
 }
 
@@ -591,7 +606,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (use_small_k(D, max_k))
+    if (use_small_k(D, max_k, H / pool->H))
         return rank_decode_small_k(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, slot_ids, past_lens, R, H, D, max_k,
                                    total_cand, scale, pool, layer, workspace, workspace_bytes, dev_status, s);
 
@@ -618,6 +633,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     p.slots = slot_ids;
     p.nseg = R;
     p.H = H;
+    p.G = H / pool->H;
     p.max_rows = max_k;
     p.total_rows = total_cand;
     p.out_fp32 = out_fp32 ? 1 : 0;
@@ -643,15 +659,15 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     switch (D) {
     case 32:
         decode_merge_kernel<32><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
-                                                       p.out_fp32, total_cand, H, nsplit, p.sl2);
+                                                       p.out_fp32, total_cand, H, p.G, nsplit, p.sl2);
         break;
     case 64:
         decode_merge_kernel<64><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
-                                                       p.out_fp32, total_cand, H, nsplit, p.sl2);
+                                                       p.out_fp32, total_cand, H, p.G, nsplit, p.sl2);
         break;
     default:
         decode_merge_kernel<128><<<blocks, 256, 0, s>>>(p.part_o, p.part_ml, p.q, p.k_self, p.v_self, out,
-                                                        p.out_fp32, total_cand, H, nsplit, p.sl2);
+                                                        p.out_fp32, total_cand, H, p.G, nsplit, p.sl2);
         break;
     }
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
@@ -666,7 +682,8 @@ int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void
     if (R < 0 || H < 1 || max_k < 0 || total_cand < 0) return UNIPIN_ERR_INVALID_ARG;
     if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
     if (R == 0 || total_cand == 0 || max_k == 0) return UNIPIN_OK;
-    const size_t need = unipin_rank_decode_workspace_size(R, H, D, max_k, total_cand, pool->n_cap);
+    if (pool->H < 1 || H % pool->H != 0) return UNIPIN_ERR_INVALID_ARG;
+    const size_t need = unipin_rank_decode_workspace_size(R, H, pool->H, D, max_k, total_cand, pool->n_cap);
     if (need > kNoAllocScratchBytes) return UNIPIN_ERR_OUT_OF_RANGE;
     void* scratch = nullptr;
     const int rc = noalloc_scratch_address(&scratch);
@@ -685,10 +702,12 @@ size_t unipin_masked_prefill_bwd_workspace_size(int total_tokens, int H)
 
 int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                               const float* lse, float* dq, float* dk, float* dv, const int* cu_seqlens,
-                              const int* past_lens, int B, int H, int D, int max_seqlen, int total_tokens,
-                              float scale, void* workspace, size_t workspace_bytes, int* dev_status, void* stream)
+                              const int* past_lens, int B, int H, int H_kv, int D, int max_seqlen,
+                              int total_tokens, float scale, void* workspace, size_t workspace_bytes,
+                              int* dev_status, void* stream)
 {
-    if (B < 0 || H < 1 || max_seqlen < 0 || total_tokens < 0) return UNIPIN_ERR_INVALID_ARG;
+    if (B < 0 || H < 1 || H_kv < 1 || H % H_kv != 0 || max_seqlen < 0 || total_tokens < 0)
+        return UNIPIN_ERR_INVALID_ARG;
     if (D != 32 && D != 64) return UNIPIN_ERR_UNSUPPORTED;
     if (!(scale > 0.f) || !std::isfinite(scale)) return UNIPIN_ERR_INVALID_ARG;
     if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
@@ -698,7 +717,7 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
     for (const void* ptr : {q, k, v, out, dout, (const void*)lse, (const void*)dq, (const void*)dk, (const void*)dv,
                             (const void*)workspace})
         if (!aligned16(ptr)) return UNIPIN_ERR_MISALIGNED;
-    const long long items = (long long)B * H * ((max_seqlen + kBwRows - 1) / kBwRows);
+    const long long items = (long long)B * H_kv * ((max_seqlen + kBwRows - 1) / kBwRows);
     if (items >= (1ll << 31)) return UNIPIN_ERR_INVALID_ARG;
     int rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
@@ -719,6 +738,7 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
     p.past = past_lens;
     p.B = B;
     p.H = H;
+    p.G = H / H_kv;
     p.total_rows = total_tokens;
     p.max_rows = max_seqlen;
     p.scale = scale;
@@ -726,7 +746,7 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
 
-    const long long rows = (long long)total_tokens * H;
+    const long long rows = (long long)total_tokens * H_kv;   // one warp per (token, key/value head)
     const unsigned prep_blocks = (unsigned)((rows + 7) / 8);
     if (D == 32)
         bwd_prep_kernel<32><<<prep_blocks, 256, 0, s>>>(p);
@@ -736,8 +756,8 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
 
     CUtensorMap tq, tk, tv, tdo;
     if ((rc = make_token_map(&tq, q, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tk, k, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
-    if ((rc = make_token_map(&tv, v, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tk, k, total_tokens, H_kv, D, kBwRows)) != UNIPIN_OK) return rc;
+    if ((rc = make_token_map(&tv, v, total_tokens, H_kv, D, kBwRows)) != UNIPIN_OK) return rc;
     if ((rc = make_token_map(&tdo, dout, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
     if (D == 32)
         bwd_kv_kernel<32><<<(unsigned)items, kBwThreads, BwCfg<32>::kSmemBytes, s>>>(tq, tk, tv, tdo, p);

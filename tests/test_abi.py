@@ -48,31 +48,34 @@ def test_host_validation_needs_no_device(lib):
     P, I = ctypes.c_void_p, ctypes.c_int
     f = lib.unipin_masked_prefill_attn
     SZ = ctypes.c_size_t
-    f.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, ctypes.c_float, P, P, I, P, SZ, P, P]
+    f.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, I, ctypes.c_float, P, P, I, P, SZ, P, P]
     f.restype = I
     args = [None, None, None, None, 1, None, None, None]
-    assert f(*args, 1, 1, 48, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -2
-    assert f(*args, -1, 1, 64, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -1
-    assert f(*args, 1, 1, 64, 16, 16, -1.0, None, None, 0, None, 0, None, None) == -1
+    assert f(*args, 1, 1, 1, 48, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -2
+    assert f(*args, -1, 1, 1, 64, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -1
+    assert f(*args, 1, 1, 1, 64, 16, 16, -1.0, None, None, 0, None, 0, None, None) == -1
+    assert f(*args, 1, 4, 3, 64, 16, 16, 0.1, None, None, 0, None, 0, None, None) == -1   # 4 heads over 3
     # nothing to do: B = 0 returns OK without touching the device
-    assert f(*args, 0, 1, 64, 16, 0, 0.1, None, None, 0, None, 0, None, None) == 0
+    assert f(*args, 0, 1, 1, 64, 16, 0, 0.1, None, None, 0, None, 0, None, None) == 0
     b = lib.unipin_masked_prefill_bwd
-    b.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, ctypes.c_float, P, SZ, P, P]
+    b.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_float, P, SZ, P, P]
     b.restype = I
     nul = [None] * 11
-    assert b(*nul, 1, 1, 128, 16, 16, 0.1, None, 0, None, None) == -2    # D = 128: not supported
-    assert b(*nul, 1, 1, 64, 16, 16, 0.0, None, 0, None, None) == -1     # scale must be positive
-    assert b(*nul, 1, 1, 64, 16, 16, 0.1, None, 0, None, None) == -1     # missing tensors
-    assert b(*nul, 0, 1, 64, 16, 0, 0.1, None, 0, None, None) == 0
+    assert b(*nul, 1, 1, 1, 128, 16, 16, 0.1, None, 0, None, None) == -2    # D = 128: not supported
+    assert b(*nul, 1, 1, 1, 64, 16, 16, 0.0, None, 0, None, None) == -1     # scale must be positive
+    assert b(*nul, 1, 1, 1, 64, 16, 16, 0.1, None, 0, None, None) == -1     # missing tensors
+    assert b(*nul, 0, 1, 1, 64, 16, 0, 0.1, None, 0, None, None) == 0
     wb = lib.unipin_masked_prefill_bwd_workspace_size
     wb.argtypes = [I, I]
     wb.restype = SZ
     assert wb(1000, 8) == 32000 and wb(3, 1) == 16
     g = lib.unipin_rank_decode_workspace_size
-    g.argtypes = [I, I, I, I, I, I]
+    g.argtypes = [I, I, I, I, I, I, I]
     g.restype = SZ
-    assert g(32, 8, 64, 16, 512, 2048) > 256       # small k: split-n partials on top of the work counter
-    assert g(32, 8, 64, 1000, 32000, 2048) == 256  # large k: the work counter only
+    assert g(32, 8, 8, 64, 16, 512, 2048) > 256       # small k: split-n partials on top of the work counter
+    assert g(32, 8, 8, 64, 1000, 32000, 2048) == 256  # large k: the work counter only
+    assert g(32, 8, 2, 64, 16, 512, 2048) > 256       # grouped heads: 4 query heads per pool head
+    assert g(32, 8, 3, 64, 16, 512, 2048) == 0        # 8 query heads over 3 key/value heads
     wp = lib.unipin_masked_prefill_workspace_size
     wp.restype = SZ
     assert wp() == 256
