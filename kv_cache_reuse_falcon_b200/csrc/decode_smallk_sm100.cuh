@@ -1,4 +1,4 @@
-// Rank decode for small candidate counts (k <= 128 per request), sm_100a.
+// Rank decode for small candidate counts (k <= 64 per request), sm_100a.
 //
 // The rank decode of [review] §2.4 / [notes] §6: the k candidates of request r
 // attend to pool rows 0..n_r-1 of slot s_r (layer l, head h) and to
@@ -8,7 +8,7 @@
 // dimension, so no tensor-core row and no softmax thread is spent on padding
 // candidates:
 //
-//   S^T = K Q^T   M = 128 keys, N = k padded to 16/32/64/128, K = D
+//   S^T = K Q^T   M = 128 keys, N = k padded to 16/32/64, K = D
 //   O  += P V     M = 128 candidate rows (rows past the padded count are
 //                 discarded), N = D, K = 128 keys; P (bf16) is staged through
 //                 shared memory in the 128-byte-swizzled K-major layout of a
@@ -31,15 +31,26 @@
 // candidate's own key (self term) and writes the output.  With one split the
 // item writes the output directly.
 //
-// Warp roles (192 threads, two blocks per SM where shared memory and TMEM
-// allow, so one block's per-item latencies hide behind the other's stream):
-//   warps 0-3  softmax and epilogue (thread t: key t of a tile; candidate t's
-//              output row in the epilogue)
-//   warp 4     TMA producer: claims items, loads Q (N candidate rows) and the
-//              V and K tiles of each key tile into a ring of stages
-//   warp 5     MMA issuer (one elected thread), owns TMEM
-// Every wait is bounded (see sm100_ptx.cuh); a block that gives up reports
-// UNIPIN_ERR_DEVICE_TIMEOUT and exits cleanly.
+// Warp roles (256 threads; two blocks per SM where shared memory and TMEM
+// allow):
+//   warps 0-1  epilogue: the own scores, the final O rows (TMEM lanes 0-63 =
+//              candidate rows), partials, arrival counter and merge
+//   warp 2     TMA producer: claims items, loads Q (N candidate rows), and
+//              drives two streams into the ring - K tiles (a slot refills as
+//              soon as its S MMA is done) and V tiles (once its P.V is done)
+//   warp 3     MMA issuer (one elected thread), owns TMEM: issues S^T as K
+//              lands (up to four S buffers ahead of the softmax) and P.V as P
+//              is written, each as its inputs arrive
+//   warps 4-7  softmax (thread t: key t of a tile, TMEM lane t); the four
+//              warps vote with one named-barrier reduction per tile
+// O has two TMEM buffers and the softmax hands each item's statistics (m, l)
+// to the epilogue through a two-entry buffer, so the key stream of the next
+// item runs while the epilogue of the last one waits on its stores and its
+// arrival counter: the ring does not stall at item boundaries.
+// Every mbarrier wait is bounded (see sm100_ptx.cuh); a block that gives up
+// reports UNIPIN_ERR_DEVICE_TIMEOUT and exits cleanly.  The softmax warps
+// leave their loop only together, on a named-barrier reduction, so none is
+// left waiting at such a barrier.
 #pragma once
 
 #include "sm100_ptx.cuh"
@@ -49,20 +60,25 @@
 namespace unipin {
 
 constexpr int kSkKeys = 128;        // keys per tile (the MMA's M)
-constexpr int kSkThreads = 192;
+constexpr int kSkThreads = 256;
+constexpr int kSkEpiWarps = 2;      // warps 0-1
+constexpr int kSkProducerWarp = 2;
+constexpr int kSkMmaWarp = 3;
+constexpr int kSkSoftmaxWarp0 = 4;  // warps 4-7
 constexpr int kSkItemSlots = 4;
-constexpr int kSkConsumers = 5;     // the MMA warp and the four softmax warps pop every item
+constexpr int kSkConsumers = 7;     // the MMA warp, the four softmax and the two epilogue warps pop every item
 constexpr int kSkMaxSplit = 16;     // key splits per (request, head) at most
 constexpr float kSkRescaleLog2 = 8.0f;
 
 // Candidate columns the kernel is compiled for, given the largest k.
-__host__ __device__ constexpr int sk_pad_n(int k) { return k <= 16 ? 16 : k <= 32 ? 32 : k <= 64 ? 64 : 128; }
+__host__ __device__ constexpr int sk_pad_n(int k) { return k <= 16 ? 16 : k <= 32 ? 32 : 64; }
 __host__ __device__ constexpr int sk_tmem_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
 
 template <int D, int N>
 struct SkCfg {
     static_assert(D == 64 || D == 128, "small-k decode: head dim 64 or 128");
-    static_assert(N == 16 || N == 32 || N == 64 || N == 128, "small-k decode: padded candidate count");
+    static_assert(N == 16 || N == 32 || N == 64, "small-k decode: padded candidate count");
+    static_assert(N <= kSkEpiWarps * 32, "small-k decode: one epilogue thread per candidate column");
     static constexpr int kChunks = D / 64;                 // 64-element boxes across D
     static constexpr int kAtom = kSkKeys * 128;            // 128 rows of 128 bytes (one swizzle block column)
     static constexpr int kTileKV = kChunks * kAtom;        // one K or V tile
@@ -74,26 +90,33 @@ struct SkCfg {
     // whatever follows in shared memory and give discarded output rows.
     static constexpr int kPBox = N * 128;
     static constexpr int kPBytes = 2 * kPBox;
-    // TMEM columns: S^T buffers at 0 and N, O (D columns) at 2N.
-    static constexpr int kColO = 2 * N;
-    static constexpr int kTmemCols = sk_tmem_cols(2 * N + D);
+    // TMEM columns: kSBufs S^T buffers of N columns from 0 (four where they fit
+    // beside two O buffers in the block's share, so that S runs well ahead of
+    // the softmax), then two O buffers of D columns.
+    static constexpr int kSBufs = (D == 64 ? sk_tmem_cols(4 * N + 2 * D) <= 256 : sk_tmem_cols(4 * N + 2 * D) <= 512) ? 4 : 2;
+    static constexpr int kColO = kSBufs * N;
+    static constexpr int kTmemCols = sk_tmem_cols(kSBufs * N + 2 * D);
+    static_assert(kTmemCols <= 512, "small-k decode: TMEM columns");
     static constexpr int kCtasPerSm = (D == 64 && kTmemCols <= 256) ? 2 : 1;
-    // Scratch floats: red[4][N], mref[N], corr[N], coef_b[N], flags[2][4],
-    // selfs[kSkItemSlots][N]; merge weights reuse a P buffer.
-    static constexpr int kScratchBytes = ((4 * N + 3 * N + 8 + kSkItemSlots * N) * 4 + 1023) / 1024 * 1024;
+    // Scratch floats: softmax red[4][N], mref[N], corr[N]; hand-off hand_m[2][N],
+    // hand_l[2][N]; epilogue coef_b[N], wts[kSkMaxSplit][N], last[4].
+    static constexpr int kScratchFloats = 4 * N + 2 * N + 4 * N + N + kSkMaxSplit * N + 4;
+    static constexpr int kScratchBytes = (kScratchFloats * 4 + 1023) / 1024 * 1024;
     static constexpr int kBarBytes = 1024;
-    static constexpr int kBudget = kCtasPerSm == 2 ? 112 * 1024 : 226 * 1024;
-    // Double-buffer Q (the next item's Q loads during this item) and P^T (the
-    // softmax writes P_{i+1} while P.V of tile i runs) where a two-stage ring
-    // still fits; single buffers otherwise.
+    // two blocks per SM: 2 x (113 KB + the 1 KB the runtime keeps per block) = 228 KB
+    static constexpr int kBudget = kCtasPerSm == 2 ? 113 * 1024 : 226 * 1024;
+    // Q is double-buffered (the next item's Q loads during this item); P is
+    // double-buffered (the softmax writes P_{i+1} while P.V of tile i runs)
+    // unless a single buffer buys one more ring stage, since the ring depth sets
+    // the bytes in flight.
     static constexpr int fixed_bytes(int qbufs, int pbufs)
     {
         return qbufs * kQBytes + pbufs * kPBytes + kScratchBytes + kBarBytes;
     }
-    static constexpr bool fits(int qbufs, int pbufs) { return kBudget - fixed_bytes(qbufs, pbufs) >= 2 * kStageBytes; }
-    static constexpr int kQBufs = fits(2, 1) ? 2 : 1;
-    static constexpr int kPBufs = fits(kQBufs, 2) ? 2 : 1;
-    static constexpr int kStagesFit = (kBudget - fixed_bytes(kQBufs, kPBufs)) / kStageBytes;
+    static constexpr int stages_with(int pbufs) { return (kBudget - fixed_bytes(2, pbufs)) / kStageBytes; }
+    static constexpr int kQBufs = 2;
+    static constexpr int kPBufs = stages_with(1) > stages_with(2) ? 1 : 2;
+    static constexpr int kStagesFit = stages_with(kPBufs);
     static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
     static_assert(kStages >= 2, "small-k decode: ring depth");
     static constexpr int kOffP = 0;                                  // first: the 128-row reads overhang
@@ -128,6 +151,8 @@ struct SkParams {
     int* status;
     unsigned long long wait_limit_ns;
     unsigned long long* sched;     // zeroed item counter or null (static striding)
+    int prefetch_tiles;            // key tiles the producer asks L2 for ahead of its ring loads
+    unsigned poll_ns;              // back-off of the polling producer and MMA warps when nothing is ready
 };
 
 // What every role derives identically from an item index.  An item is a
@@ -274,44 +299,59 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     uint8_t* ring = smem + C::kOffRing;
     uint8_t* sQ = smem + C::kOffQ;
     uint8_t* sP = smem + C::kOffP;
-    float* red = reinterpret_cast<float*>(smem + C::kOffScratch);   // [4][N]
+    float* red = reinterpret_cast<float*>(smem + C::kOffScratch);   // [4][N] softmax
     float* mref = red + 4 * N;                                      // [N] reference max (log2 units)
     float* corr = mref + N;                                         // [N]
-    float* coef_b = corr + N;                                       // [N] merge: weight of the own value
-    volatile int* flags = reinterpret_cast<volatile int*>(coef_b + N);   // [2][4]
-    float* selfs = coef_b + N + 8;                                  // [kSkItemSlots][N] own scores, per item slot
+    float* hand_m = corr + N;                                       // [2][N] item statistics, softmax -> epilogue
+    float* hand_l = hand_m + 2 * N;                                 // [2][N]
+    float* coef_b = hand_l + 2 * N;                                 // [N] epilogue: weight of the own value
+    float* wts = coef_b + N;                                        // [kSkMaxSplit][N] epilogue: split weights
+    volatile int* last_flag = reinterpret_cast<volatile int*>(wts + kSkMaxSplit * N);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* bar_q = bars + 0;            // [2] Q buffer landed
     uint64_t* q_empty = bars + 2;          // [2] the last S MMA of the item using Q buffer b finished
-    uint64_t* s_full = bars + 4;           // [2] S^T buffer computed
-    uint64_t* s_free = bars + 6;           // [2] S^T buffer read out (4 softmax warps)
-    uint64_t* p_full = bars + 8;           // [2] P^T buffer written (4 softmax warps)
-    uint64_t* pv_done = bars + 10;         // [2] O^T += V^T P^T of P buffer b finished
-    uint64_t* grp = bars + 12;             // softmax-group barrier (4 warps)
-    uint64_t* bar_drain = bars + 13;
-    uint64_t* kv_full = bars + 14;         // [NS]
-    uint64_t* kv_empty = kv_full + NS;     // [NS]
-    uint64_t* item_full = kv_empty + NS;   // [kSkItemSlots]
+    uint64_t* pv_done = bars + 4;          // [2] O += P V of P buffer b finished
+    uint64_t* p_full = bars + 6;           // [2] P buffer written (4 softmax warps)
+    uint64_t* o_full = bars + 8;           // [2] the last P.V of the item in O buffer b finished
+    uint64_t* o_free = bars + 10;          // [2] O buffer b read out (2 epilogue warps)
+    uint64_t* h_full = bars + 12;          // [2] hand-off entry written (4 softmax warps)
+    uint64_t* h_free = bars + 14;          // [2] hand-off entry read (2 epilogue warps)
+    uint64_t* egrp = bars + 16;            // epilogue-group barrier (2 warps)
+    uint64_t* bar_drain = bars + 17;
+    uint64_t* s_full = bars + 18;          // [kSBufs] S^T buffer computed
+    uint64_t* s_free = s_full + C::kSBufs; // [kSBufs] S^T buffer read out (4 softmax warps)
+    uint64_t* k_full = s_free + C::kSBufs; // [NS] K tile landed
+    uint64_t* k_empty = k_full + NS;       // [NS] its S MMA finished
+    uint64_t* v_full = k_empty + NS;       // [NS] V tile landed
+    uint64_t* v_empty = v_full + NS;       // [NS] its P.V finished
+    uint64_t* item_full = v_empty + NS;    // [kSkItemSlots]
     uint64_t* item_empty = item_full + kSkItemSlots;
     volatile long long* item_ring = reinterpret_cast<volatile long long*>(item_empty + kSkItemSlots);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 2 * kSkItemSlots);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    volatile int* last_flag = abort_flag + 1;
 
     if (threadIdx.x == 0) {
         for (int b = 0; b < 2; ++b) {
             mbar_init(bar_q + b, 1);
             mbar_init(q_empty + b, 1);
+            mbar_init(pv_done + b, 1);
+            mbar_init(p_full + b, 4);
+            mbar_init(o_full + b, 1);
+            mbar_init(o_free + b, kSkEpiWarps);
+            mbar_init(h_full + b, 4);
+            mbar_init(h_free + b, kSkEpiWarps);
+        }
+        for (int b = 0; b < C::kSBufs; ++b) {
             mbar_init(s_full + b, 1);
             mbar_init(s_free + b, 4);
-            mbar_init(p_full + b, 4);
-            mbar_init(pv_done + b, 1);
         }
-        mbar_init(grp, 4);
+        mbar_init(egrp, kSkEpiWarps);
         mbar_init(bar_drain, 1);
         for (int s = 0; s < NS; ++s) {
-            mbar_init(kv_full + s, 1);
-            mbar_init(kv_empty + s, 1);
+            mbar_init(k_full + s, 1);
+            mbar_init(k_empty + s, 1);
+            mbar_init(v_full + s, 1);
+            mbar_init(v_empty + s, 1);
         }
         for (int s = 0; s < kSkItemSlots; ++s) {
             mbar_init(item_full + s, 1);
@@ -321,7 +361,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         fence_mbarrier_init();
     }
     if (threadIdx.x < N) mref[threadIdx.x] = -INFINITY;
-    if (warp == 5) {
+    if (warp == kSkMmaWarp) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -333,14 +373,12 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
     const long long total_items = (long long)p.R * (p.H / p.G) * p.nsplit;
     int n_items = 0;
-    // Consumers: the next item (warp-uniform); `own` receives selfs[slot][own_col] read
-    // before the slot is released (the producer may refill it right after).
-    auto pop_item = [&](bool& ok, long long& g, int own_col, float& own) -> bool {
+    // Consumers: the next item (warp-uniform)
+    auto pop_item = [&](bool& ok, long long& g) -> bool {
         const int si = n_items % kSkItemSlots;
         ok = __all_sync(0xffffffffu, mbar_wait(item_full + si, (n_items / kSkItemSlots) & 1, ctl));
         if (!ok) return false;
         g = item_ring[si];
-        own = (own_col >= 0 && own_col < N) ? selfs[si * N + own_col] : -INFINITY;
         __syncwarp();
         if (lane == 0) mbar_arrive(item_empty + si);
         ++n_items;
@@ -348,84 +386,146 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     };
     const bool leader = lane == 0;
 
-    if (warp == 4) {
+    if (warp == kSkProducerWarp) {
         // ------------------------------------------------------------ producer
+        // Two streams into the ring: K tiles (freed when their S MMA finishes)
+        // and V tiles (freed when their P.V finishes).  A K slot thus refills
+        // while the softmax still works on that tile, and V, needed only after
+        // the softmax, is requested as soon as its slot frees.  One polling loop
+        // drives both (warp-uniform; the leader lane issues the copies).
         if (leader) {
             tma_prefetch_map(&tm_q);
             tma_prefetch_map(&tm_k);
             tma_prefetch_map(&tm_v);
         }
-        int u = 0, nq = 0;
-        bool ok = true;
-        long long g_static = blockIdx.x;
-        while (ok) {
-            const int si = n_items % kSkItemSlots;
-            if (n_items >= kSkItemSlots) {
-                ok = __all_sync(0xffffffffu, mbar_wait(item_empty + si, ((n_items / kSkItemSlots) - 1) & 1, ctl));
-                if (!ok) break;
+        struct PItem {
+            int plane, t_begin, nt, nt_all, npast;
+        };
+        PItem items[4];          // items with tiles whose V stream has not finished, by sequence % 4
+        int uk = 0, uv = 0;      // K / V tiles issued (global tile index)
+        int nk = 0, nv = 0;      // items with tiles started by the K stream / finished by the V stream
+        int ik = 0, iv = 0;      // tile within the current K / V item
+        int nq = 0;
+        bool k_has = false, q_done = false, claim_done = false, ok = true;
+        int q_h = 0, q_tok = 0;
+        // The first item of a block is its index; later ones come from the shared
+        // counter (offset by the grid), claimed one item ahead so that the
+        // atomic's latency overlaps this item's loads.
+        long long g_next = blockIdx.x;
+        uint64_t t_prog = global_timer_ns();
+        for (uint32_t spin = 1;; ++spin) {
+            bool prog = false;
+            // 1. publish the next item once the K stream has finished its current one
+            if (!k_has && !claim_done && nk - nv < 3) {
+                const int si = n_items % kSkItemSlots;
+                if (n_items < kSkItemSlots ||
+                    __all_sync(0xffffffffu, mbar_test_wait(item_empty + si, ((n_items / kSkItemSlots) - 1) & 1))) {
+                    const long long g = __shfl_sync(0xffffffffu, g_next, 0);
+                    const bool found = g < total_items;
+                    if (found) {
+                        if (p.sched) {
+                            if (leader) g_next = (long long)gridDim.x + (long long)atomicAdd(p.sched, 1ull);
+                        } else {
+                            g_next = g + gridDim.x;
+                        }
+                    }
+                    if (leader) {
+                        item_ring[si] = found ? g : -1;
+                        mbar_arrive(item_full + si);   // release: the consumers see the ring entry
+                    }
+                    ++n_items;
+                    prog = true;
+                    if (!found) {
+                        claim_done = true;
+                    } else {
+                        const SkWork w = sk_make_work<N>(p, g);
+                        if (w.nt > 0) {
+                            items[nk % 4] = PItem{(p.layer * p.S + w.slot) * (p.H / p.G) + w.h, w.t_begin, w.nt,
+                                                  w.nt_all, w.npast};
+                            q_h = w.h;
+                            q_tok = w.tok0;
+                            ++nk;
+                            k_has = true;
+                            ik = 0;
+                            q_done = false;
+                        }
+                    }
+                }
             }
-            long long g = 0;
-            if (p.sched) {
-                if (leader) g = (long long)atomicAdd(p.sched, 1ull);
-                g = __shfl_sync(0xffffffffu, g, 0);
+            // 2. K stream: the item's Q, then its K tiles
+            if (k_has) {
+                if (!q_done) {
+                    const int qb = nq % NQ;
+                    if (nq < NQ || __all_sync(0xffffffffu, mbar_test_wait(q_empty + qb, ((nq / NQ) - 1) & 1))) {
+                        if (leader) {
+                            mbar_arrive_expect_tx(bar_q + qb, C::kQBytes);
+                            for (int c = 0; c < C::kChunks; ++c)
+                                // N / G candidate tokens x the G query heads of key/value head q_h
+                                tma_load_3d(sQ + qb * C::kQBytes + c * C::kAtomQ, &tm_q, bar_q + qb, c * 64, q_h * p.G,
+                                            q_tok);
+                        }
+                        ++nq;
+                        q_done = true;
+                        prog = true;
+                    }
+                }
+                const int st = uk % NS;
+                if (q_done &&
+                    (uk < NS || __all_sync(0xffffffffu, mbar_test_wait(k_empty + st, ((uk / NS) - 1) & 1)))) {
+                    const PItem& it = items[(nk - 1) % 4];
+                    const int start = sk_tile_start(it.t_begin + ik, it.nt_all, it.npast);
+                    if (leader) {
+                        uint8_t* dst = ring + st * C::kStageBytes + C::kTileKV;
+                        mbar_arrive_expect_tx(k_full + st, C::kTileKV);
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_3d(dst + c * C::kAtom, &tm_k, k_full + st, c * 64, start, it.plane);
+                    }
+                    ++uk;
+                    prog = true;
+                    if (++ik == it.nt) k_has = false;
+                }
+            }
+            // 3. V stream: V_u once K_u has been issued
+            if (uv < uk) {
+                const int st = uv % NS;
+                if (uv < NS || __all_sync(0xffffffffu, mbar_test_wait(v_empty + st, ((uv / NS) - 1) & 1))) {
+                    const PItem& it = items[nv % 4];
+                    const int start = sk_tile_start(it.t_begin + iv, it.nt_all, it.npast);
+                    if (leader) {
+                        uint8_t* dst = ring + st * C::kStageBytes;
+                        mbar_arrive_expect_tx(v_full + st, C::kTileKV);
+                        for (int c = 0; c < C::kChunks; ++c)
+                            tma_load_3d(dst + c * C::kAtom, &tm_v, v_full + st, c * 64, start, it.plane);
+                    }
+                    ++uv;
+                    prog = true;
+                    if (++iv == it.nt) {
+                        iv = 0;
+                        ++nv;
+                    }
+                }
+            }
+            if (claim_done && !k_has && uv == uk) break;   // every copy issued
+            if (prog) {
+                t_prog = global_timer_ns();
             } else {
-                g = g_static;
-                g_static += gridDim.x;
-            }
-            const bool found = g < total_items;
-            SkWork w;
-            if (found) {
-                // the own score of every candidate column (log2 units), off the softmax warps' path
-                w = sk_make_work<N>(p, g);
-                if (w.valid) {
-                    const int hkv = p.H / p.G;
-                    for (int n = lane; n < w.ncol; n += 32) {
-                        const size_t qrow = (size_t)(w.tok0 + n / p.G) * p.H + w.h * p.G + n % p.G;
-                        const size_t kvrow = (size_t)(w.tok0 + n / p.G) * hkv + w.h;
-                        selfs[si * N + n] = p.sl2 * sk_dot_bf16<D>(p.q + qrow * D, p.k_self + kvrow * D);
+                __nanosleep(p.poll_ns);
+                if ((spin & 15) == 0) {
+                    // warp-uniform: give up when the block aborted or nothing moved for too long
+                    const bool aborted = *abort_flag != 0;
+                    const bool stop = __any_sync(0xffffffffu, aborted || global_timer_ns() - t_prog > p.wait_limit_ns);
+                    if (stop) {
+                        if (leader && !aborted) {
+                            *abort_flag = 1;
+                            report(p.status, (int)UNIPIN_ERR_DEVICE_TIMEOUT);
+                        }
+                        ok = false;
+                        break;
                     }
                 }
-                __syncwarp();
-            }
-            if (leader) {
-                item_ring[si] = found ? g : -1;
-                mbar_arrive(item_full + si);   // release: the consumers see selfs[si] with the item
-            }
-            ++n_items;
-            if (!found) break;
-            if (w.nt == 0) continue;
-            const int qb = nq % NQ;
-            if (nq >= NQ) {
-                ok = __all_sync(0xffffffffu, mbar_wait(q_empty + qb, ((nq / NQ) - 1) & 1, ctl));
-                if (!ok) break;
-            }
-            if (leader) {
-                mbar_arrive_expect_tx(bar_q + qb, C::kQBytes);
-                for (int c = 0; c < C::kChunks; ++c)
-                    // N / G candidate tokens x the G query heads of key/value head w.h
-                    tma_load_3d(sQ + qb * C::kQBytes + c * C::kAtomQ, &tm_q, bar_q + qb, c * 64, w.h * p.G, w.tok0);
-            }
-            ++nq;
-            const int plane = (p.layer * p.S + w.slot) * (p.H / p.G) + w.h;
-            for (int i = 0; ok && i < w.nt; ++i) {
-                const int start = sk_tile_start(w.t_begin + i, w.nt_all, w.npast);
-                const int st = u % NS;
-                if (u >= NS) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(kv_empty + st, ((u / NS) - 1) & 1, ctl));
-                    if (!ok) break;
-                }
-                if (leader) {
-                    uint8_t* dst = ring + st * C::kStageBytes;
-                    mbar_arrive_expect_tx(kv_full + st, C::kStageBytes);
-                    for (int c = 0; c < C::kChunks; ++c) {
-                        tma_load_3d(dst + c * C::kAtom, &tm_v, kv_full + st, c * 64, start, plane);
-                        tma_load_3d(dst + C::kTileKV + c * C::kAtom, &tm_k, kv_full + st, c * 64, start, plane);
-                    }
-                }
-                ++u;
             }
         }
-        if (!ok && leader) {
+        if (!ok && !claim_done && leader) {
             const int si = n_items % kSkItemSlots;
             if (n_items < kSkItemSlots ||
                 mbar_wait_drain(item_empty + si, ((n_items / kSkItemSlots) - 1) & 1, p.wait_limit_ns)) {
@@ -436,143 +536,171 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         }
         if (leader) {
             // Let every copy this warp started land before the block exits.
-            for (int v = (u > NS ? u - NS : 0); v < u; ++v)
-                mbar_wait_drain(kv_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
+            for (int v = (uk > NS ? uk - NS : 0); v < uk; ++v)
+                mbar_wait_drain(k_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
+            for (int v = (uv > NS ? uv - NS : 0); v < uv; ++v)
+                mbar_wait_drain(v_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
             for (int v = (nq > NQ ? nq - NQ : 0); v < nq; ++v)
                 mbar_wait_drain(bar_q + v % NQ, (v / NQ) & 1, p.wait_limit_ns);
             for (int v = (n_items > kSkItemSlots ? n_items - kSkItemSlots : 0); v < n_items; ++v)
                 mbar_wait_drain(item_empty + v % kSkItemSlots, (v / kSkItemSlots) & 1, p.wait_limit_ns);
         }
-    } else if (warp == 5) {
+    } else if (warp == kSkMmaWarp) {
         // --------------------------------------------------------- MMA issuer
-        // Per key tile i: S^T_i = K_i Q^T, then O^T += V_{i-1}^T P^T_{i-1} once
-        // the softmax has written P_{i-1}; so S_{i+1} is computed while the
-        // softmax works on S_i.
+        // Two streams, issued as their inputs arrive (one polling loop):
+        //   S^T_i = K_i Q^T  once K_i has landed and an S buffer is free; up to
+        //                    kSBufs tiles ahead of the softmax, across items;
+        //   O += P_i V_i     once the softmax has written P_i and V_i has landed
+        //                    (the first of an item also needs its O buffer back
+        //                    from the epilogue).  Item j accumulates in O buffer j % 2.
+        constexpr int NSB = C::kSBufs;
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kSkKeys, N, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true, false);
         const uint32_t ring_a = smem_u32(ring);
         // K (A of S^T): K-major, 128-byte rows, 8-row groups 1024 bytes apart.
         const uint64_t dk0 = smem_desc(ring_a + C::kTileKV, 16, 1024, kLayoutSw128);
-        // V (B of O += P V, MN-major): 64-element head-dim blocks 16 KB apart,
-        // 8-key groups 1024 bytes apart.
-        const uint64_t dv0 = smem_desc(ring_a, C::kAtom, 1024, kLayoutSw128);
         const uint64_t dq0 = smem_desc(smem_u32(sQ), 16, 1024, kLayoutSw128);
+        // V (B of O += P V, MN-major): 64-element head-dim blocks 16 KB apart, 8-key groups 1024 bytes apart.
+        const uint64_t dv0 = smem_desc(ring_a, C::kAtom, 1024, kLayoutSw128);
         // P (A of O += P V): K-major rows of 64 keys per box, 8-row groups 1024 bytes apart.
         const uint64_t dp0 = smem_desc(smem_u32(sP), 16, 1024, kLayoutSw128);
-        const uint32_t tO = tmem + C::kColO;
-        int u = 0, nq = 0;
-        int gs = 0;            // S tiles issued
-        int gp = 0;            // P.V products issued
-        int pfull_seen[2] = {0, 0};
-        bool ok = true;
-        long long g;
-        auto issue_pv = [&](int st, int pb, bool acc) {
-            // K-steps of 16 keys: 32 bytes within a P row (then the second box), 16 V rows
-#pragma unroll
-            for (int kk = 0; kk < kSkKeys / 16; ++kk) {
-                const uint64_t a = dp0 + (uint64_t)((pb * C::kPBytes + (kk / 4) * C::kPBox + (kk % 4) * 32) >> 4);
-                const uint64_t b = dv0 + (uint64_t)((st * C::kStageBytes + kk * 2048) >> 4);
-                umma_bf16_ss(tO, a, b, idesc_pv, (acc || kk > 0) ? 1u : 0u);
-            }
-            umma_commit(pv_done + pb);
-            umma_commit(kv_empty + st);
-        };
-        auto wait_p = [&](int gidx) {
-            const int pb = gidx % NP;
-            const int n = gidx / NP;
-            bool r = true;
-            while (r && pfull_seen[pb] <= n) {
-                r = __all_sync(0xffffffffu, mbar_wait(p_full + pb, pfull_seen[pb] & 1, ctl));
-                ++pfull_seen[pb];
-            }
-            tc_fence_after_sync();
-            return r;
-        };
-        float unused_own;
-        while (pop_item(ok, g, -1, unused_own)) {
-            const SkWork w = sk_make_work<N>(p, g);
-            if (w.nt == 0) continue;
-            const int qb = nq % NQ;
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_q + qb, (nq / NQ) & 1, ctl));
-            if (!ok) break;
-            ++nq;
-            for (int i = 0; ok && i < w.nt; ++i) {
-                // S_i needs K_i landed and an S buffer the softmax has read out; P.V of
-                // tile i-1 needs P_{i-1}.  Issue each as soon as its inputs are there: a
-                // P.V queued behind the next tile's data would hold its ring stage, and
-                // the ring would then have a single load in flight.
-                const int st = (u + i) % NS;
-                const int sb = gs & 1;
-                bool need_qk = true;
-                bool need_pv = i >= 1;
-                const uint64_t t0 = global_timer_ns();
-                for (uint32_t spin = 1; need_qk || need_pv; ++spin) {
-                    if (need_pv) {
-                        const int pb = gp % NP;
-                        if (__all_sync(0xffffffffu, mbar_test_wait(p_full + pb, pfull_seen[pb] & 1))) {
-                            ++pfull_seen[pb];
-                            tc_fence_after_sync();
-                            if (leader) issue_pv((u + i - 1) % NS, pb, i - 1 > 0);
-                            ++gp;
-                            need_pv = false;
-                        }
-                    }
-                    if (need_qk && __all_sync(0xffffffffu, mbar_test_wait(kv_full + st, ((u + i) / NS) & 1) &&
-                                                              (gs < 2 || mbar_test_wait(s_free + sb, ((gs >> 1) - 1) & 1)))) {
-                        tc_fence_after_sync();
-                        if (leader) {
-#pragma unroll
-                            for (int kk = 0; kk < D / 16; ++kk) {
-                                const int box = kk / 4;
-                                const int in_row = (kk % 4) * 32;
-                                const uint64_t a =
-                                    dk0 + (uint64_t)((st * C::kStageBytes + box * C::kAtom + in_row) >> 4);
-                                const uint64_t b = dq0 + (uint64_t)((qb * C::kQBytes + box * C::kAtomQ + in_row) >> 4);
-                                umma_bf16_ss(tmem + sb * N, a, b, idesc_qk, kk > 0 ? 1u : 0u);
-                            }
-                            umma_commit(s_full + sb);
-                            if (i == w.nt - 1) umma_commit(q_empty + qb);
-                        }
-                        ++gs;
-                        need_qk = false;
-                    }
-                    if ((spin & 31) == 0) {
-                        // warp-uniform: every lane leaves the loop together
-                        const bool aborted = *abort_flag != 0;
-                        const bool stop = __any_sync(0xffffffffu, aborted || global_timer_ns() - t0 > p.wait_limit_ns);
-                        if (stop) {
-                            if (leader && !aborted) {
-                                *abort_flag = 1;
-                                report(p.status, (int)UNIPIN_ERR_DEVICE_TIMEOUT);
-                            }
-                            ok = false;
-                            break;
+        int pv_nt[8];                 // tile counts of the items with tiles whose P.V are not all issued
+        int nqueued = 0, npv_item = 0;
+        int gs = 0;                   // S tiles issued (= global tile index of the next S)
+        int gp = 0;                   // P.V products issued
+        int is = 0, s_nt = 0, nq = 0, ip = 0;
+        bool s_has = false, s_done = false, q_ok = false, ok = true;
+        uint64_t t_prog = global_timer_ns();
+        for (uint32_t spin = 1;; ++spin) {
+            bool prog = false;
+            // ---- S stream: take the next item with tiles
+            if (!s_has && !s_done && nqueued - npv_item < 7) {
+                const int si = n_items % kSkItemSlots;
+                if (__all_sync(0xffffffffu, mbar_test_wait(item_full + si, (n_items / kSkItemSlots) & 1))) {
+                    const long long g = item_ring[si];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(item_empty + si);
+                    ++n_items;
+                    prog = true;
+                    if (g < 0) {
+                        s_done = true;
+                    } else {
+                        const SkWork w = sk_make_work<N>(p, g);
+                        if (w.nt > 0) {
+                            pv_nt[nqueued % 8] = w.nt;
+                            ++nqueued;
+                            s_has = true;
+                            s_nt = w.nt;
+                            is = 0;
+                            q_ok = false;
                         }
                     }
                 }
             }
-            if (!ok) break;
-            if (!(ok = wait_p(gp))) break;
-            if (leader) issue_pv((u + w.nt - 1) % NS, gp % NP, w.nt > 1);
-            ++gp;
-            u += w.nt;
+            if (s_has) {
+                const int qb = nq % NQ;
+                if (!q_ok && __all_sync(0xffffffffu, mbar_test_wait(bar_q + qb, (nq / NQ) & 1))) q_ok = true;
+                const int st = gs % NS;
+                const int sb = gs % NSB;
+                if (q_ok && __all_sync(0xffffffffu, mbar_test_wait(k_full + st, (gs / NS) & 1) &&
+                                                        (gs < NSB || mbar_test_wait(s_free + sb, ((gs / NSB) - 1) & 1)))) {
+                    tc_fence_after_sync();
+                    if (leader) {
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const int box = kk / 4;
+                            const int in_row = (kk % 4) * 32;
+                            const uint64_t a = dk0 + (uint64_t)((st * C::kStageBytes + box * C::kAtom + in_row) >> 4);
+                            const uint64_t b = dq0 + (uint64_t)((qb * C::kQBytes + box * C::kAtomQ + in_row) >> 4);
+                            umma_bf16_ss(tmem + sb * N, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                        }
+                        umma_commit(s_full + sb);
+                        umma_commit(k_empty + st);
+                        if (is == s_nt - 1) umma_commit(q_empty + qb);
+                    }
+                    ++gs;
+                    prog = true;
+                    if (++is == s_nt) {
+                        s_has = false;
+                        ++nq;
+                    }
+                }
+            }
+            // ---- P.V stream: tiles whose S was issued
+            if (gp < gs) {
+                const int nt = pv_nt[npv_item % 8];
+                const int ob = npv_item & 1;
+                const int pb = gp % NP;
+                const int st = gp % NS;
+                if (__all_sync(0xffffffffu, mbar_test_wait(p_full + pb, (gp / NP) & 1) &&
+                                                mbar_test_wait(v_full + st, (gp / NS) & 1) &&
+                                                (ip > 0 || npv_item < 2 ||
+                                                 mbar_test_wait(o_free + ob, ((npv_item >> 1) - 1) & 1)))) {
+                    tc_fence_after_sync();
+                    if (leader) {
+                        // K-steps of 16 keys: 32 bytes within a P row (then the second box), 16 V rows
+#pragma unroll
+                        for (int kk = 0; kk < kSkKeys / 16; ++kk) {
+                            const uint64_t a =
+                                dp0 + (uint64_t)((pb * C::kPBytes + (kk / 4) * C::kPBox + (kk % 4) * 32) >> 4);
+                            const uint64_t b = dv0 + (uint64_t)((st * C::kStageBytes + kk * 2048) >> 4);
+                            umma_bf16_ss(tmem + C::kColO + ob * D, a, b, idesc_pv, (ip > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(pv_done + pb);
+                        umma_commit(v_empty + st);
+                        if (ip == nt - 1) umma_commit(o_full + ob);
+                    }
+                    ++gp;
+                    prog = true;
+                    if (++ip == nt) {
+                        ip = 0;
+                        ++npv_item;
+                    }
+                }
+            }
+            if (s_done && !s_has && gp == gs) break;
+            if (prog) {
+                t_prog = global_timer_ns();
+            } else {
+                __nanosleep(p.poll_ns);
+                if ((spin & 15) == 0) {
+                    // warp-uniform: give up when the block aborted or nothing moved for too long
+                    const bool aborted = *abort_flag != 0;
+                    const bool stop = __any_sync(0xffffffffu, aborted || global_timer_ns() - t_prog > p.wait_limit_ns);
+                    if (stop) {
+                        if (leader && !aborted) {
+                            *abort_flag = 1;
+                            report(p.status, (int)UNIPIN_ERR_DEVICE_TIMEOUT);
+                        }
+                        ok = false;
+                        break;
+                    }
+                }
+            }
         }
+        (void)ok;
         if (leader) {
             umma_commit(bar_drain);
             mbar_wait_drain(bar_drain, 0, p.wait_limit_ns);
         }
-    } else {
-        // ------------------------------------------------- softmax + epilogue
-        const int t = threadIdx.x;                               // key of a tile / candidate row of O
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    } else if (warp >= kSkSoftmaxWarp0) {
+        // ------------------------------------------------------------ softmax
+        // The four warps move in step: each named-barrier reduction below is
+        // reached by all 128 threads, and they leave the item loop only
+        // together, on such a reduction (bounded waits only flag a failure).
+        const int wq = warp - kSkSoftmaxWarp0;                   // TMEM lane quarter
+        const int t = wq * 32 + lane;                            // key of a tile; O row t (candidate t)
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        constexpr int kBar = 1;                                  // named barrier of the group
+        constexpr int kGroup = 128;
+        constexpr int NSB = C::kSBufs;
         const float sl2 = p.sl2;
-        int gs = 0, gp = 0;
+        int gs = 0, gp = 0, nb = 0, nh = 0;
+        bool pending_fail = false;                               // a wait after the last reduction failed
         int pv_seen[2] = {0, 0};
-        uint32_t ngrp = 0;
-        bool ok = true;
         long long g;
         // Wait until the P.V product with global index gidx has finished
-        // (completions of each P buffer are consumed in order).
+        // (completions of each P buffer are consumed in order); warp-uniform.
         auto wait_pv = [&](int gidx) {
             if (gidx < 0) return true;
             const int pb = gidx % NP;
@@ -585,70 +713,74 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             tc_fence_after_sync();
             return r;
         };
-        float own_popped;
-        while (pop_item(ok, g, threadIdx.x, own_popped)) {
+        for (;;) {
+            bool okp;
+            const bool got = pop_item(okp, g);
+            if (bar_red_or(kBar, kGroup, !okp || pending_fail || *abort_flag != 0)) break;
+            if (!got) break;   // the end marker: the same ring entry for every warp
             const SkWork w = sk_make_work<N>(p, g);
-            if (!w.rows_ok) {
-                if (t == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
-                continue;
-            }
-            if (!w.valid && t == 0 && w.split == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
-            // Column t = (candidate t / G, query head w.h * G + t % G): its output row, its own
-            // key/value row, and its own score (log2 units), taken while the first tile is in flight.
-            const int hkv = p.H / p.G;
-            const size_t qrow = (size_t)(w.tok0 + t / p.G) * p.H + w.h * p.G + t % p.G;
-            const size_t kvrow = (size_t)(w.tok0 + t / p.G) * hkv + w.h;
-            const float ss_own = (t < w.ncol && w.valid) ? own_popped : -INFINITY;
+            if (!w.rows_ok && t == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
+            if (w.rows_ok && !w.valid && t == 0 && w.split == 0) report(p.status, (int)UNIPIN_ERR_OUT_OF_RANGE);
+            const int ob = nb & 1;
+            const uint32_t tO = lane_base + C::kColO + ob * D;
             // per-thread partial column sums of P (owned columns), relative to mref
             constexpr int kOwn = N >= 32 ? N / 32 : 1;
             float lown[kOwn];
 #pragma unroll
             for (int e = 0; e < kOwn; ++e) lown[e] = 0.f;
+            bool quit = false;
             for (int i = 0; i < w.nt; ++i) {
                 const int tile = w.t_begin + i;
                 const int lo = tile * kSkKeys;
                 const int start = sk_tile_start(tile, w.nt_all, w.npast);
                 const int key = start + t;
                 const bool key_ok = key >= lo && key < w.npast;
-                const int sb = gs & 1;
-                ok = __all_sync(0xffffffffu, mbar_wait(s_full + sb, (gs >> 1) & 1, ctl));
-                if (!ok) break;
-                tc_fence_after_sync();
-                uint32_t sraw[N];
-                tmem_ld_n<N>(lane_base + sb * N, sraw);
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(s_free + sb);
-                ++gs;
+                const int sb = gs % NSB;
+                const bool ok_s = __all_sync(0xffffffffu, mbar_wait(s_full + sb, (gs / NSB) & 1, ctl));
                 float x[N];
-#pragma unroll
-                for (int c = 0; c < N; ++c)
-                    x[c] = (key_ok && c < w.ncol) ? __uint_as_float(sraw[c]) * sl2 : -INFINITY;
-                // vote: does any score exceed its candidate's reference max by > 2^8?
                 bool need = false;
+                if (ok_s) {
+                    tc_fence_after_sync();
+                    uint32_t sraw[N];
+                    tmem_ld_n<N>(lane_base + sb * N, sraw);
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(s_free + sb);
 #pragma unroll
-                for (int c = 0; c < N; c += 4) {
-                    const float4 m4 = *reinterpret_cast<const float4*>(mref + c);
-                    need |= x[c] > m4.x + kSkRescaleLog2;
-                    need |= x[c + 1] > m4.y + kSkRescaleLog2;
-                    need |= x[c + 2] > m4.z + kSkRescaleLog2;
-                    need |= x[c + 3] > m4.w + kSkRescaleLog2;
+                    for (int c = 0; c < N; ++c)
+                        x[c] = (key_ok && c < w.ncol) ? __uint_as_float(sraw[c]) * sl2 : -INFINITY;
+                    // vote: does any score exceed its candidate's reference max by > 2^8?
+#pragma unroll
+                    for (int c = 0; c < N; c += 4) {
+                        const float4 m4 = *reinterpret_cast<const float4*>(mref + c);
+                        need |= x[c] > m4.x + kSkRescaleLog2;
+                        need |= x[c + 1] > m4.y + kSkRescaleLog2;
+                        need |= x[c + 2] > m4.z + kSkRescaleLog2;
+                        need |= x[c + 3] > m4.w + kSkRescaleLog2;
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < N; ++c) x[c] = -INFINITY;
                 }
-                const int fb = ngrp & 1;
-                const int warp_need = __any_sync(0xffffffffu, need) ? 1 : 0;
-                if (lane == 0) flags[fb * 4 + warp] = warp_need;
-                if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
-                const bool any_need = (flags[fb * 4 + 0] | flags[fb * 4 + 1] | flags[fb * 4 + 2] | flags[fb * 4 + 3]) != 0;
-                if (any_need) {
-                    // exact column maxima of this tile; move every reference max to it
-                    float cm[N];
+                ++gs;
+                const bool fail_s = !ok_s || pending_fail || *abort_flag != 0;
+                bool ok_w = true;
+                if (bar_red_or(kBar, kGroup, need || fail_s)) {
+                    if (bar_red_or(kBar, kGroup, fail_s)) {
+                        quit = true;
+                        break;
+                    }
+                    // exact column maxima of this tile (16 columns at a time: lane pair l/2
+                    // owns column c0 + l/2); move every reference max to it
 #pragma unroll
-                    for (int c = 0; c < N; ++c) cm[c] = x[c];
-                    sk_rs_step<N, 16, true>(cm, lane);
+                    for (int c0 = 0; c0 < N; c0 += 16) {
+                        float cm[16];
 #pragma unroll
-                    for (int e = 0; e < kOwn; ++e)
-                        if (N >= 32 || (lane & 1) == 0) red[warp * N + sk_owned_col<N>(lane, e)] = cm[e];
-                    if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
+                        for (int c = 0; c < 16; ++c) cm[c] = x[c0 + c];
+                        sk_rs_step<16, 16, true>(cm, lane);
+                        if ((lane & 1) == 0) red[wq * N + c0 + (lane >> 1)] = cm[0];
+                    }
+                    bar_group_sync(kBar, kGroup);
                     if (t < N) {
                         const float mt = fmaxf(fmaxf(red[t], red[N + t]), fmaxf(red[2 * N + t], red[3 * N + t]));
                         const float mo = mref[t];
@@ -656,27 +788,26 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                         corr[t] = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mn);
                         mref[t] = mn;
                     }
-                    if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
+                    bar_group_sync(kBar, kGroup);
 #pragma unroll
                     for (int e = 0; e < kOwn; ++e) lown[e] *= corr[sk_owned_col<N>(lane, e)];
                     if (i > 0) {
                         // rescale the O rows accumulated so far (after the last P.V): row c is candidate c
-                        if (!(ok = wait_pv(gp - 1))) break;
-                        if (warp * 32 < N) {
+                        ok_w = wait_pv(gp - 1);
+                        if (ok_w && wq * 32 < N) {
                             const float cf = corr[t < N ? t : 0];
 #pragma unroll
                             for (int c0 = 0; c0 < D; c0 += 16) {
                                 uint32_t o[16];
-                                tmem_ld16(lane_base + C::kColO + c0, o);
+                                tmem_ld16(tO + c0, o);
 #pragma unroll
                                 for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * cf);
-                                tmem_st16(lane_base + C::kColO + c0, o);
+                                tmem_st16(tO + c0, o);
                             }
                         }
                     }
                 }
                 // P = 2^(x - m)
-                float ps[N];
 #pragma unroll
                 for (int c = 0; c < N; c += 4) {
                     const float4 m4 = *reinterpret_cast<const float4*>(mref + c);
@@ -684,205 +815,242 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float mu = mm[e] == -INFINITY ? 0.f : mm[e];
-                        ps[c + e] = ex2_approx(x[c + e] - mu);
+                        x[c + e] = ex2_approx(x[c + e] - mu);
                     }
                 }
                 // the P buffer is free once the P.V that last read it has finished
                 const int pb = gp % NP;
-                if (!(ok = wait_pv(gp - NP))) break;
-                // column t of P: key t of the tile is element t % 64 of a 128-byte row of box t / 64
-                {
+                const bool ok_p = ok_w && wait_pv(gp - NP);
+                if (ok_p) {
+                    // column t of P: key t of the tile is element t % 64 of a 128-byte row of box t / 64
                     uint8_t* pbox = sP + pb * C::kPBytes + (t / 64) * C::kPBox;
                     const int kx = t % 64;
 #pragma unroll
                     for (int c = 0; c < N; ++c)
                         *reinterpret_cast<__nv_bfloat16*>(pbox + c * 128 + ((((kx >> 3) ^ (c & 7))) << 4) +
-                                                          (kx & 7) * 2) = __float2bfloat16_rn(ps[c]);
-                }
-                fence_proxy_async_smem();
-                tc_fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(p_full + pb);
-                ++gp;
-                sk_rs_step<N, 16, false>(ps, lane);
-#pragma unroll
-                for (int e = 0; e < kOwn; ++e) lown[e] += ps[e];
-            }
-            if (!ok) break;
-            // ------------------------------------------------------ epilogue
-            // the own value row is fetched before the last wait, so its latency overlaps it
-            // (where registers allow: the widest variant keeps it in the store loop)
-            constexpr bool kPrefetchV = N <= 32;
-            uint4 vrow[kPrefetchV ? D / 8 : 1];
-            if (kPrefetchV && p.nsplit == 1 && t < w.ncol) {
-                const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + kvrow * D);
-#pragma unroll
-                for (int d8 = 0; d8 < D / 8; ++d8) vrow[d8] = __ldg(v4 + d8);
-            }
-            if (w.nt > 0 && !(ok = wait_pv(gp - 1))) break;
-#pragma unroll
-            for (int e = 0; e < kOwn; ++e)
-                if (N >= 32 || (lane & 1) == 0) red[warp * N + sk_owned_col<N>(lane, e)] = lown[e];
-            if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
-            // thread t < N: candidate t's sum, max and output coefficients
-            float m_c = -INFINITY, l_c = 0.f, ca = 0.f, cb = 0.f;
-            if (t < N) {
-                l_c = red[t] + red[N + t] + red[2 * N + t] + red[3 * N + t];
-                m_c = w.nt > 0 ? mref[t] : -INFINITY;
-                mref[t] = -INFINITY;   // ready for the next item
-                if (p.nsplit == 1 && t < w.ncol && w.valid) {
-                    // final: (a O + b v_self) / (a l + b)
-                    const float mf = fmaxf(m_c, ss_own);
-                    const float a = (m_c == -INFINITY) ? 0.f : ex2_approx(m_c - mf);
-                    const float b = ex2_approx(ss_own - mf);
-                    const float inv = 1.f / (l_c * a + b);
-                    ca = a * inv;
-                    cb = b * inv;
-                }
-            }
-            // O row t = candidate t (warp-collective load where the warp holds candidate rows)
-            uint32_t o[D];
-            if (w.nt > 0 && warp * 32 < N) {
-                if constexpr (D == 64) tmem_ld64(lane_base + C::kColO, o);
-                else tmem_ld128(lane_base + C::kColO, o);
-            } else {
-#pragma unroll
-                for (int d = 0; d < D; ++d) o[d] = 0u;
-            }
-            tc_fence_before_sync();
-            if (t < w.ncol) {
-                const size_t row = qrow;
-                if (p.nsplit == 1) {
-#pragma unroll
-                    for (int d8 = 0; d8 < D / 8; ++d8) {
-                        uint4 vb;
-                        if constexpr (kPrefetchV) vb = vrow[d8];
-                        else vb = __ldg(reinterpret_cast<const uint4*>(p.v_self + kvrow * D) + d8);
-                        const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vb);
-                        float r[8];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 vf = __bfloat1622float2(vh[e]);
-                            r[2 * e] = __uint_as_float(o[d8 * 8 + 2 * e]) * ca + cb * vf.x;
-                            r[2 * e + 1] = __uint_as_float(o[d8 * 8 + 2 * e + 1]) * ca + cb * vf.y;
-                        }
-                        sk_store4(p.out, p.out_fp32, row * D + d8 * 8, make_float4(r[0], r[1], r[2], r[3]));
-                        sk_store4(p.out, p.out_fp32, row * D + d8 * 8 + 4, make_float4(r[4], r[5], r[6], r[7]));
-                    }
+                                                          (kx & 7) * 2) = __float2bfloat16_rn(x[c]);
+                    fence_proxy_async_smem();
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(p_full + pb);
                 } else {
-                    float* po = p.part_o + ((size_t)w.split * p.total_rows * p.H + row) * D;
+                    pending_fail = true;   // decided together at the next reduction
+                }
+                ++gp;
+                sk_rs_step<N, 16, false>(x, lane);
 #pragma unroll
-                    for (int d = 0; d < D; d += 4)
-                        *reinterpret_cast<float4*>(po + d) =
+                for (int e = 0; e < kOwn; ++e) lown[e] += x[e];
+            }
+            if (quit) break;
+            // hand the item's statistics to the epilogue (every item, so both sides count alike)
+            const int hb = nh & 1;
+            if (w.nt > 0) {
+#pragma unroll
+                for (int e = 0; e < kOwn; ++e)
+                    if (N >= 32 || (lane & 1) == 0) red[wq * N + sk_owned_col<N>(lane, e)] = lown[e];
+            }
+            const bool ok_h = nh < 2 || __all_sync(0xffffffffu, mbar_wait(h_free + hb, ((nh >> 1) - 1) & 1, ctl));
+            if (bar_red_or(kBar, kGroup, !ok_h || pending_fail || *abort_flag != 0)) break;
+            if (t < N) {
+                hand_l[hb * N + t] = w.nt > 0 ? red[t] + red[N + t] + red[2 * N + t] + red[3 * N + t] : 0.f;
+                hand_m[hb * N + t] = w.nt > 0 ? mref[t] : -INFINITY;
+                mref[t] = -INFINITY;   // ready for the next item
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(h_full + hb);
+            ++nh;
+            if (w.nt > 0) ++nb;
+            // red and mref are reused by the next item
+            bar_group_sync(kBar, kGroup);
+        }
+    } else {
+        // ----------------------------------------------------------- epilogue
+        const int t = threadIdx.x;                               // candidate column t; O row t = TMEM lane t
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        const int hkv = p.H / p.G;
+        int nb = 0, nh = 0;
+        uint32_t negrp = 0;
+        bool ok = true;
+        long long g;
+        while (pop_item(ok, g)) {
+            const SkWork w = sk_make_work<N>(p, g);
+            // Column t = (candidate t / G, query head w.h * G + t % G): its output row, its own
+            // key/value row, and its own score (log2 units), taken while the item's keys stream.
+            const size_t qrow = (size_t)(w.tok0 + t / p.G) * p.H + w.h * p.G + t % p.G;
+            const size_t kvrow = (size_t)(w.tok0 + t / p.G) * hkv + w.h;
+            const bool mine = w.valid && t < w.ncol;
+            const float ss_own = mine ? p.sl2 * sk_dot_bf16<D>(p.q + qrow * D, p.k_self + kvrow * D) : -INFINITY;
+            // the item's statistics
+            const int hb = nh & 1;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(h_full + hb, (nh >> 1) & 1, ctl)))) break;
+            const float l_c = t < N ? hand_l[hb * N + t] : 0.f;
+            const float m_c = t < N ? hand_m[hb * N + t] : -INFINITY;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(h_free + hb);
+            ++nh;
+            if (!w.rows_ok) continue;
+            // O row t, 32 columns at a time (warp-collective loads where the warp holds candidate rows)
+            const int ob = nb & 1;
+            const bool have_o = w.nt > 0 && warp * 32 < N;
+            if (w.nt > 0) {
+                if (!(ok = __all_sync(0xffffffffu, mbar_wait(o_full + ob, (nb >> 1) & 1, ctl)))) break;
+                tc_fence_after_sync();
+            }
+            // final coefficients (one split): out = (a O + b v_self) / (a l + b)
+            float ca = 0.f, cb = 0.f;
+            if (p.nsplit == 1 && mine) {
+                const float mf = fmaxf(m_c, ss_own);
+                const float a = (m_c == -INFINITY) ? 0.f : ex2_approx(m_c - mf);
+                const float b = ex2_approx(ss_own - mf);
+                const float inv = 1.f / (l_c * a + b);
+                ca = a * inv;
+                cb = b * inv;
+            }
+            float* po = p.part_o + ((size_t)w.split * p.total_rows * p.H + qrow) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                if (have_o) {
+                    tmem_ld32(lane_base + C::kColO + ob * D + c0, o);
+                } else {
+#pragma unroll
+                    for (int d = 0; d < 32; ++d) o[d] = 0u;
+                }
+                if (p.nsplit == 1) {
+                    // a rejected request (ca = cb = 0) gets zero rows
+                    if (t < w.ncol) {
+                        const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + kvrow * D + c0);
+#pragma unroll
+                        for (int d8 = 0; d8 < 4; ++d8) {
+                            const uint4 vb = mine ? __ldg(v4 + d8) : make_uint4(0u, 0u, 0u, 0u);
+                            const __nv_bfloat162* vh = reinterpret_cast<const __nv_bfloat162*>(&vb);
+                            float r[8];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 vf = __bfloat1622float2(vh[e]);
+                                r[2 * e] = __uint_as_float(o[d8 * 8 + 2 * e]) * ca + cb * vf.x;
+                                r[2 * e + 1] = __uint_as_float(o[d8 * 8 + 2 * e + 1]) * ca + cb * vf.y;
+                            }
+                            sk_store4(p.out, p.out_fp32, qrow * D + c0 + d8 * 8, make_float4(r[0], r[1], r[2], r[3]));
+                            sk_store4(p.out, p.out_fp32, qrow * D + c0 + d8 * 8 + 4, make_float4(r[4], r[5], r[6], r[7]));
+                        }
+                    }
+                } else if (t < w.ncol) {
+#pragma unroll
+                    for (int d = 0; d < 32; d += 4)
+                        *reinterpret_cast<float4*>(po + c0 + d) =
                             make_float4(__uint_as_float(o[d]), __uint_as_float(o[d + 1]), __uint_as_float(o[d + 2]),
                                         __uint_as_float(o[d + 3]));
-                    float* ml = p.part_ml + ((size_t)w.split * p.total_rows * p.H + row) * 2;
-                    ml[0] = w.valid ? m_c : -INFINITY;
-                    ml[1] = w.valid ? l_c : 0.f;
                 }
             }
-            if (p.nsplit > 1) {
-                // publish the partial; the last split of this (request, head) to arrive merges
+            if (w.nt > 0) {
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(o_free + ob);
+                ++nb;
+            }
+            if (p.nsplit == 1) continue;
+            // publish the partial; the last split of this (request, head) to arrive merges
+            if (t < w.ncol) {
+                float* ml = p.part_ml + ((size_t)w.split * p.total_rows * p.H + qrow) * 2;
+                ml[0] = w.valid ? m_c : -INFINITY;
+                ml[1] = w.valid ? l_c : 0.f;
+            }
+            __threadfence();
+            if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
+            if (t == 0) {
+                const unsigned prev = atomicAdd(p.pair_cnt + w.pair, 1u);
+                *last_flag = prev == (unsigned)(p.nsplit - 1);
+            }
+            if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
+            if (*last_flag) {
                 __threadfence();
-                if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
-                if (t == 0) {
-                    const unsigned prev = atomicAdd(p.pair_cnt + w.pair, 1u);
-                    *last_flag = prev == (unsigned)(p.nsplit - 1);
-                }
-                if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
-                if (*last_flag) {
-                    __threadfence();
-                    float* wts = reinterpret_cast<float*>(sP + (gp % NP) * C::kPBytes);   // [kSkMaxSplit][N]
-                    if (t < w.ncol) {
-                        // weights of the splits and of the own key: LSE merge in log2 units
-                        const size_t row = qrow;
-                        float ms[kSkMaxSplit], ls[kSkMaxSplit];
+                if (t < w.ncol) {
+                    // weights of the splits and of the own key: LSE merge in log2 units
+                    float ms[kSkMaxSplit], ls[kSkMaxSplit];
 #pragma unroll
-                        for (int s = 0; s < kSkMaxSplit; ++s) {
-                            float2 ml = make_float2(-INFINITY, 0.f);
-                            if (s < p.nsplit)
-                                ml = __ldcg(reinterpret_cast<const float2*>(
-                                    p.part_ml + ((size_t)s * p.total_rows * p.H + row) * 2));
-                            ms[s] = ml.x;
-                            ls[s] = ml.y;
-                        }
-                        float mf = ss_own;
-#pragma unroll
-                        for (int s = 0; s < kSkMaxSplit; ++s) mf = fmaxf(mf, ms[s]);
-                        const float b = ex2_approx(ss_own - mf);
-                        float den = b;
-                        float a[kSkMaxSplit];
-#pragma unroll
-                        for (int s = 0; s < kSkMaxSplit; ++s) {
-                            a[s] = (ms[s] == -INFINITY || !(ls[s] > 0.f)) ? 0.f : ex2_approx(ms[s] - mf);
-                            den = fmaf(a[s], ls[s], den);
-                        }
-                        // a rejected request (no own score: every term -inf) gets zero weights
-                        const float inv = w.valid ? 1.f / den : 0.f;
-#pragma unroll
-                        for (int s = 0; s < kSkMaxSplit; ++s)
-                            if (s < p.nsplit) wts[s * N + t] = w.valid ? a[s] * inv : 0.f;
-                        coef_b[t] = w.valid ? b * inv : 0.f;
+                    for (int s = 0; s < kSkMaxSplit; ++s) {
+                        float2 ml = make_float2(-INFINITY, 0.f);
+                        if (s < p.nsplit)
+                            ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s * p.total_rows * p.H + qrow) * 2));
+                        ms[s] = ml.x;
+                        ls[s] = ml.y;
                     }
-                    if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
-                    // out = b v_self + sum_s w_s O_s, four head-dim elements per thread and step;
-                    // four steps' loads are issued before their sums
-                    constexpr int kQ = D / 4;
-                    const int total = w.ncol * kQ;
-                    const size_t split_stride = (size_t)p.total_rows * p.H * D;
-                    for (int base = 0; base < total; base += 4 * 128) {
-                        float4 acc[4];
-                        size_t idx[4];
-                        int cc[4];
+                    float mf = ss_own;
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int q = base + u * 128 + t;
-                            const bool act = q < total;
-                            cc[u] = act ? q / kQ : -1;
-                            const int c = act ? cc[u] : 0;
-                            // column c: candidate c / G, query head w.h * G + c % G
-                            idx[u] = ((size_t)(w.tok0 + c / p.G) * p.H + w.h * p.G + c % p.G) * D + (q % kQ) * 4;
-                            const size_t vidx = ((size_t)(w.tok0 + c / p.G) * hkv + w.h) * D + (q % kQ) * 4;
-                            acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            if (act) {
-                                const uint2 vb = __ldg(reinterpret_cast<const uint2*>(p.v_self + vidx));
-                                const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.x));
-                                const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.y));
-                                const float cbv = coef_b[c];
-                                acc[u] = make_float4(cbv * v01.x, cbv * v01.y, cbv * v23.x, cbv * v23.y);
-                            }
+                    for (int s = 0; s < kSkMaxSplit; ++s) mf = fmaxf(mf, ms[s]);
+                    const float b = ex2_approx(ss_own - mf);
+                    float den = b;
+#pragma unroll
+                    for (int s = 0; s < kSkMaxSplit; ++s) {
+                        const float a = (ms[s] == -INFINITY || !(ls[s] > 0.f)) ? 0.f : ex2_approx(ms[s] - mf);
+                        den = fmaf(a, ls[s], den);
+                        if (s < p.nsplit) wts[s * N + t] = a;
+                    }
+                    // a rejected request (no own score: every term -inf) gets zero weights
+                    const float inv = w.valid ? 1.f / den : 0.f;
+                    for (int s = 0; s < p.nsplit; ++s) wts[s * N + t] *= inv;
+                    coef_b[t] = w.valid ? b * inv : 0.f;
+                }
+                if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
+                // out = b v_self + sum_s w_s O_s, four head-dim elements per thread and step;
+                // four steps' loads are issued before their sums
+                constexpr int kQ = D / 4;
+                constexpr int kEt = kSkEpiWarps * 32;
+                const int total = w.ncol * kQ;
+                const size_t split_stride = (size_t)p.total_rows * p.H * D;
+                for (int base = 0; base < total; base += 4 * kEt) {
+                    float4 acc[4];
+                    size_t idx[4];
+                    int cc[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int q = base + u * kEt + t;
+                        const bool act = q < total;
+                        cc[u] = act ? q / kQ : -1;
+                        const int c = act ? cc[u] : 0;
+                        // column c: candidate c / G, query head w.h * G + c % G
+                        idx[u] = ((size_t)(w.tok0 + c / p.G) * p.H + w.h * p.G + c % p.G) * D + (q % kQ) * 4;
+                        const size_t vidx = ((size_t)(w.tok0 + c / p.G) * hkv + w.h) * D + (q % kQ) * 4;
+                        acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (act) {
+                            const uint2 vb = __ldg(reinterpret_cast<const uint2*>(p.v_self + vidx));
+                            const float2 v01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.x));
+                            const float2 v23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&vb.y));
+                            const float cbv = coef_b[c];
+                            acc[u] = make_float4(cbv * v01.x, cbv * v01.y, cbv * v23.x, cbv * v23.y);
                         }
+                    }
 #pragma unroll
-                        for (int s = 0; s < kSkMaxSplit; ++s) {
-                            if (s < p.nsplit) {
+                    for (int s = 0; s < kSkMaxSplit; ++s) {
+                        if (s < p.nsplit) {
 #pragma unroll
-                                for (int u = 0; u < 4; ++u) {
-                                    if (cc[u] >= 0) {
-                                        const float4 pv =
-                                            __ldcg(reinterpret_cast<const float4*>(p.part_o + s * split_stride + idx[u]));
-                                        const float wv = wts[s * N + cc[u]];
-                                        acc[u].x = fmaf(wv, pv.x, acc[u].x);
-                                        acc[u].y = fmaf(wv, pv.y, acc[u].y);
-                                        acc[u].z = fmaf(wv, pv.z, acc[u].z);
-                                        acc[u].w = fmaf(wv, pv.w, acc[u].w);
-                                    }
+                            for (int u = 0; u < 4; ++u) {
+                                if (cc[u] >= 0) {
+                                    const float4 pv =
+                                        __ldcg(reinterpret_cast<const float4*>(p.part_o + s * split_stride + idx[u]));
+                                    const float wv = wts[s * N + cc[u]];
+                                    acc[u].x = fmaf(wv, pv.x, acc[u].x);
+                                    acc[u].y = fmaf(wv, pv.y, acc[u].y);
+                                    acc[u].z = fmaf(wv, pv.z, acc[u].z);
+                                    acc[u].w = fmaf(wv, pv.w, acc[u].w);
                                 }
                             }
                         }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u)
-                            if (cc[u] >= 0) sk_store4(p.out, p.out_fp32, idx[u], acc[u]);
                     }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (cc[u] >= 0) sk_store4(p.out, p.out_fp32, idx[u], acc[u]);
                 }
             }
-            // scratch (red, weights) is reused by the next item
-            if (!(ok = warp_group_sync(grp, ngrp, ctl, lane))) break;
+            // last_flag, coef_b and wts are reused by the next item
+            if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
         }
     }
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == kSkMmaWarp) {
         __syncwarp();
         tc_fence_after_sync();
         tmem_dealloc(tmem, C::kTmemCols);

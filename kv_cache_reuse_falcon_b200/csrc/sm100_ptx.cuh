@@ -205,6 +205,31 @@ __device__ __forceinline__ bool warp_group_sync(uint64_t* bar, uint32_t& n, cons
     return ok;
 }
 
+// Named-barrier reduction over `nthreads` threads (a multiple of 32) of this
+// CTA: returns whether `pred` holds for any of them.  It has no time limit, so
+// a group that uses it must reach every such barrier the same number of times:
+// its threads never leave a loop one by one, only together on a result of
+// this reduction (every wait before it is bounded).
+__device__ __forceinline__ bool bar_red_or(int id, int nthreads, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "barrier.cta.red.or.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+        : "memory");
+    return r != 0;
+}
+
+// Named barrier among `nthreads` threads (same rules as bar_red_or).
+__device__ __forceinline__ void bar_group_sync(int id, int nthreads)
+{
+    asm volatile("barrier.cta.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Time-limited wait that ignores the abort flag: used on the exit path to
 // let copies and MMAs that are already in flight land before the CTA's
 // shared memory and TMEM are released.
@@ -234,6 +259,16 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// 3-D tiled prefetch global -> L2 of one box (no shared memory, no completion
+// signal): a later tma_load_3d of the same box reads it from L2.
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
 }
 
 // 3-D tiled store shared -> global (box as the map's), tracked by this thread's bulk group.

@@ -303,7 +303,30 @@ int sk_items_per_block()
     static int v = [] {
         const char* s = std::getenv("UNIPIN_DECODE_ITEMS_PER_BLOCK");
         int n = s ? std::atoi(s) : 0;
-        return n > 0 ? n : 4;
+        return n > 0 ? n : 1;
+    }();
+    return v;
+}
+
+// Key tiles the small-k producer prefetches into L2 ahead of its ring loads
+// (off by default: it measured slower); UNIPIN_DECODE_PREFETCH_TILES sets it.
+int sk_prefetch_tiles()
+{
+    static int v = [] {
+        const char* s = std::getenv("UNIPIN_DECODE_PREFETCH_TILES");
+        int n = s ? std::atoi(s) : 0;
+        return n > 0 ? (n > 64 ? 64 : n) : 0;
+    }();
+    return v;
+}
+
+// Back-off (ns) of the small-k kernel's polling warps; UNIPIN_DECODE_POLL_NS overrides it.
+unsigned sk_poll_ns()
+{
+    static unsigned v = [] {
+        const char* s = std::getenv("UNIPIN_DECODE_POLL_NS");
+        int n = s ? std::atoi(s) : -1;
+        return (unsigned)(n >= 0 ? (n > 10000 ? 10000 : n) : 64);
     }();
     return v;
 }
@@ -412,6 +435,8 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
     p.sched = sched;
+    p.prefetch_tiles = sk_prefetch_tiles();
+    p.poll_ns = sk_poll_ns();
     if (pl.nsplit > 1) {
         char* ws = static_cast<char*>(workspace);
         p.pair_cnt = reinterpret_cast<unsigned*>(ws + kSchedBytes);
