@@ -57,6 +57,13 @@ def _load():
         lib.oracle_prefill_bwd_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, ctypes.c_double, I, P, P, P]
         lib.oracle_prefill_bwd_f64.restype = I
         lib.oracle_pool_write.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, I]
+        lib.oracle_pool_write_e4m3.argtypes = [P, P, I, I, I, I, I, I, P, P, P, P, P, I, ctypes.c_float,
+                                               ctypes.c_float]
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_dequant_bf16.argtypes = [P, I64, ctypes.c_float, P]
         lib.oracle_pool_write.restype = I
         lib.oracle_num_threads.restype = I
         lib.oracle_set_num_threads.argtypes = [I]
@@ -164,6 +171,61 @@ def pool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids
                                    _ptr(k), _ptr(v), _ptr(cu), _ptr(past), _ptr(slots), past.shape[0])
     if rc != 0:
         raise ValueError("oracle_pool_write rejected its arguments")
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """E4M3 codes (uint8) of float32 values: nearest value, ties to even, saturating at +-448."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    lib = _load()
+    out = np.empty(x.shape, np.uint8)
+    flat, of = x.reshape(-1), out.reshape(-1)
+    for i in range(flat.shape[0]):
+        of[i] = lib.oracle_e4m3_encode(float(flat[i]))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """The real value (float64) of each E4M3 code."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    lib = _load()
+    return np.array([lib.oracle_e4m3_decode(int(b)) for b in c.reshape(-1)], np.float64).reshape(c.shape)
+
+
+def e4m3_dequant_bf16(codes, scale: float) -> np.ndarray:
+    """bfloat16 bit patterns of decode(code) * scale (float32 product, nearest even)."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.uint16)
+    _load().oracle_e4m3_dequant_bf16(_ptr(c), c.size, float(scale), _ptr(out))
+    return out
+
+
+def pool_write_e4m3(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids, k_scale: float,
+                    v_scale: float) -> None:
+    """In-place CPU mirror of the pool write into an E4M3 pool (codes of k / k_scale, v / v_scale).
+
+    The division is taken as a float32 multiply by 1 / scale, the reciprocal itself rounded to
+    float32 once, as the library does."""
+    for name, t in (("pool_k", pool_k), ("pool_v", pool_v)):
+        if t.dtype != np.uint8 or not t.flags.c_contiguous:
+            raise TypeError("%s must be a C-contiguous uint8 array" % name)
+    L, S, H, n_cap, D = pool_k.shape
+    k, v = _u16(k), _u16(v)
+    cu, past, slots = _i32(cu_seqlens), _i32(past_lens), _i32(slot_ids)
+    inv_k = float(np.float32(1.0) / np.float32(k_scale))
+    inv_v = float(np.float32(1.0) / np.float32(v_scale))
+    rc = _load().oracle_pool_write_e4m3(_ptr(pool_k), _ptr(pool_v), L, S, H, n_cap, D, int(layer), _ptr(k), _ptr(v),
+                                        _ptr(cu), _ptr(past), _ptr(slots), past.shape[0], inv_k, inv_v)
+    if rc != 0:
+        raise ValueError("oracle_pool_write_e4m3 rejected its arguments")
+
+
+def decode_e4m3(qc, kc, vc, cu_c, slot_ids, past_lens, pool_k8, pool_v8, layer: int, k_scale: float,
+                v_scale: float, scale: Optional[float] = None):
+    """Rank decode over an E4M3 pool: the pool rows read as bfloat16(decode(code) * scale), then the
+    same decode as over a bfloat16 pool."""
+    pk = e4m3_dequant_bf16(pool_k8, k_scale)
+    pv = e4m3_dequant_bf16(pool_v8, v_scale)
+    return decode(qc, kc, vc, cu_c, slot_ids, past_lens, pk, pv, layer, scale=scale)
 
 
 def _bwd(fn, q, k, v, dout, cu_seqlens, past_lens, scale, cand_self):

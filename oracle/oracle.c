@@ -417,3 +417,107 @@ int oracle_pool_write(uint16_t *pool_k, uint16_t *pool_v, int L, int S, int H, i
     }
     return 0;
 }
+
+/*
+ * E4M3 pool variant (an extrapolation: the pages apply FP8 E4M3 to linear
+ * layers, [notes]/[review] FP8 sections; here the pool stores K and V in it).
+ *
+ * E4M3 ("fn" form): 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits.
+ *   exponent field 0       subnormal  (-1)^s * m/8 * 2^-6    (m = 1..7)
+ *   exponent field 1..15   normal     (-1)^s * (1 + m/8) * 2^(e-7)
+ *   field 15 with m = 7 is NaN; there is no infinity; the largest finite
+ *   magnitude is 1.75 * 2^8 = 448.
+ *
+ * Encoding (the reading used for the pool): round the real value to the
+ * nearest E4M3 value, ties to the even mantissa, and clamp magnitudes that
+ * round beyond 448 to 448 ("saturate to finite").  NaN encodes as 0x7F.
+ */
+uint8_t oracle_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a == 0.0) return sign;
+    /* grid spacing of the binade holding a: 2^-9 below the smallest normal 2^-6 */
+    int e;
+    frexp(a, &e);                     /* a = f * 2^e, f in [0.5, 1): binade exponent e - 1 */
+    int be = e - 1;
+    if (be < -6) be = -6;             /* subnormal range shares the spacing of the first binade */
+    double spacing = ldexp(1.0, be - 3);
+    double q = nearbyint(a / spacing);   /* exact division by a power of two; ties to even */
+    double val = q * spacing;
+    if (val > 448.0) val = 448.0;
+    /* re-derive the fields from the rounded value (rounding may carry into the next binade) */
+    if (val < ldexp(1.0, -6)) {
+        int m = (int)(val / ldexp(1.0, -9));
+        return sign | (uint8_t)m;
+    }
+    frexp(val, &e);
+    int ex = e - 1;
+    int m = (int)(val / ldexp(1.0, ex - 3)) - 8;
+    return sign | (uint8_t)(((ex + 7) << 3) | m);
+}
+
+double oracle_e4m3_decode(uint8_t c)
+{
+    int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return (uint16_t)((u >> 16) | 0x40);   /* quiet NaN */
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+/*
+ * Pool write into an E4M3 pool: the same rows as oracle_pool_write, each
+ * element stored as E4M3(k * inv_scale) with the product taken in float32
+ * (the bfloat16 input widened exactly, one rounding of the product).
+ */
+int oracle_pool_write_e4m3(uint8_t *pool_k, uint8_t *pool_v, int L, int S, int H, int n_cap, int D,
+                           int layer, const uint16_t *k, const uint16_t *v, const int32_t *cu_seqlens,
+                           const int32_t *past_lens, const int32_t *slot_ids, int B, float inv_k, float inv_v)
+{
+    if (layer < 0 || layer >= L || B < 0) return -1;
+    for (int b = 0; b < B; ++b) {
+        if (slot_ids[b] < 0 || slot_ids[b] >= S) return -1;
+        if (past_lens[b] < 0 || past_lens[b] > n_cap) return -1;
+        if (past_lens[b] > cu_seqlens[b + 1] - cu_seqlens[b]) return -1;
+    }
+    for (int b = 0; b < B; ++b) {
+        for (int h = 0; h < H; ++h) {
+            int64_t row0 = (((int64_t)layer * S + slot_ids[b]) * H + h) * (int64_t)n_cap;
+            for (int64_t j = 0; j < past_lens[b]; ++j) {
+                int64_t src = (((int64_t)cu_seqlens[b] + j) * H + h) * (int64_t)D;
+                for (int d = 0; d < D; ++d) {
+                    float kf = (float)bf16_to_f64(k[src + d]) * inv_k;
+                    float vf = (float)bf16_to_f64(v[src + d]) * inv_v;
+                    pool_k[(row0 + j) * D + d] = oracle_e4m3_encode(kf);
+                    pool_v[(row0 + j) * D + d] = oracle_e4m3_encode(vf);
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * What an attention kernel reads from an E4M3 pool: bfloat16(decode(c) * scale),
+ * the product in float32, rounded to nearest even.  Elementwise over n codes.
+ */
+void oracle_e4m3_dequant_bf16(const uint8_t *codes, int64_t n, float scale, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        float f = (float)oracle_e4m3_decode(codes[i]) * scale;
+        out[i] = f32_to_bf16_rne(f);
+    }
+}
