@@ -50,11 +50,11 @@ def decode_flops(past, cand, H, D):
     return float(4.0 * D * H * (k * (p + 1)).sum())
 
 
-def decode_bytes(past, cand, H, D, out_bytes):
+def decode_bytes(past, cand, H, D, out_bytes, pool_elem_bytes=2):
     """Algorithmic bytes: pool K/V rows read once + candidate q/k/v read + output written."""
     p = np.asarray(past, dtype=np.float64).sum()
     k = np.asarray(cand, dtype=np.float64).sum()
-    return float(2 * p * H * D * 2 + 3 * k * H * D * 2 + k * H * D * out_bytes)
+    return float(2 * p * H * D * pool_elem_bytes + 3 * k * H * D * 2 + k * H * D * out_bytes)
 
 
 def prefill_bytes(T, H, D, out_bytes):
@@ -590,10 +590,40 @@ def run_sweep(device, peaks, iters=10, warm=3):
         e["ms_per_12_layers"] = ms * w.L
         out["decode_R32_n2048_D64_k%d" % kk] = e
         del qkv, outs, ws
+    del pk, pv
+    torch.cuda.empty_cache()
+
+    # the same decode from an E4M3 pool (codes of N(0, 1) / 0.0625 keys and values)
+    scales = (0.0625, 0.0625)
+    pk8 = (randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed).float() / scales[0]).to(torch.float8_e4m3fn)
+    pv8 = (randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed + 1).float() / scales[1]).to(torch.float8_e4m3fn)
+    for kk in (16,):
+        cand = np.full(w.B, kk, np.int32)
+        Tc = int(cand.sum())
+        cu = torch.from_numpy(synth.cu_from_lens(cand)).to(device)
+        qkv = [[randn((Tc, w.H, w.D), w.seed + 10 * l + j) for j in range(3)] for l in range(w.L)]
+        outs = [torch.empty((Tc, w.H, w.D), dtype=torch.bfloat16, device=device) for _ in range(w.L)]
+        nws = ub.rank_decode_pool_workspace_size(pk8, pv8, w.B, w.H, kk, Tc, pool_scales=scales)
+        ws = torch.empty(nws // 4 + 4, dtype=torch.float32, device=device)
+
+        def fn8():
+            for l in range(w.L):
+                ub.rank_decode_attn(qkv[l][0], qkv[l][1], qkv[l][2], cu, slots, pl, pk8, pv8, l, kk, out=outs[l],
+                                    out_fp32=False, workspace=ws, dev_status=status, stream=stream,
+                                    pool_scales=scales)
+
+        ms = timed(fn8) / w.L
+        e = roof_entry(ms, decode_flops(past, cand, w.H, w.D), decode_bytes(past, cand, w.H, w.D, 2, 1), peaks,
+                       "kvpool_dequant_kernel + decode_smallk_kernel<%d,16>" % w.D)
+        e["path"] = "E4M3 rows dequantized into the workspace, then the bfloat16 kernel"
+        e["candidates_per_s"] = float(Tc) / (ms * 1e-3)
+        out["decode_R32_n2048_D64_k%d_e4m3" % kk] = e
+        del qkv, outs, ws
+    del pk8, pv8
     torch.cuda.synchronize(device)
     if int(status.item()) != 0:
         raise RuntimeError("device status %s in the sweep" % ub.status_string(int(status.item())))
-    del pk, pv, flush
+    del flush
     torch.cuda.empty_cache()
     return out
 

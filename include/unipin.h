@@ -60,17 +60,37 @@ typedef enum {
     UNIPIN_ERR_DEVICE_TIMEOUT = -6  /* a bounded device wait expired (reported via dev_status) */
 } unipin_status;
 
+/* Element type of a pool's K and V. */
+typedef enum {
+    UNIPIN_POOL_BF16 = 0,   /* bfloat16 */
+    UNIPIN_POOL_E4M3 = 1    /* FP8 E4M3 codes with one scale for K and one for V */
+} unipin_pool_dtype;
+
 /*
  * The KV cache pool ([review] §2.4, [notes] §6): one preallocated tensor of
  * shape [L, S, H, n_cap, D] for K and one for V (layer, slot, KV head,
- * history position, head dim), bfloat16, row-major, caller-owned device
- * memory.  Row (l, s, h, j) starts at element (((l * S + s) * H + h) * n_cap + j) * D.
+ * history position, head dim), row-major, caller-owned device memory.  Row
+ * (l, s, h, j) starts at element (((l * S + s) * H + h) * n_cap + j) * D.
  * A slot holds one user's past K/V; rows j >= that user's n are never read.
+ *
+ * dtype UNIPIN_POOL_BF16: elements are bfloat16; k_scale and v_scale are ignored.
+ * dtype UNIPIN_POOL_E4M3: elements are FP8 E4M3 codes (1 byte; the format's
+ *   fn form: bias 7, no infinity, largest finite 448).  The pages apply E4M3 to
+ *   their linear layers ([notes]/[review] FP8 sections); storing the pool in it
+ *   is this library's extension, halving its size.  Writing x stores
+ *   E4M3(x * (1 / k_scale)) (the reciprocal and the product in float32, nearest
+ *   value with ties to even, magnitudes saturated at 448); attention reads code c
+ *   as bfloat16(value(c) * k_scale) (float32 product, nearest even), and alike
+ *   for V.  Scales must be finite and positive; with powers of two the read is
+ *   exact.
  */
 typedef struct {
     void* k;
     void* v;
     int L, S, H, n_cap, D;
+    int dtype;            /* unipin_pool_dtype */
+    float k_scale;        /* UNIPIN_POOL_E4M3 only */
+    float v_scale;
 } unipin_kvpool;
 
 /*
@@ -96,8 +116,9 @@ typedef struct {
  *   scale          softmax scale, normally 1/sqrt(D)
  *   pool, slot_ids optional (pool == NULL: no pool write).  When given (pool->H ==
  *                  H_kv), the past K/V of segment b is also written to pool rows
- *                  [layer, slot_ids[b], h, 0:n_b) exactly as unipin_kvpool_write does,
- *                  by the same kernel from the K/V tiles it loads anyway.
+ *                  [layer, slot_ids[b], h, 0:n_b) exactly as unipin_kvpool_write does:
+ *                  into a bfloat16 pool by the same kernel from the K/V tiles it loads
+ *                  anyway, into an E4M3 pool by a second kernel of the same call.
  *   workspace      optional device scratch, 16-byte aligned (NULL allowed).  With at
  *                  least unipin_masked_prefill_workspace_size() bytes, the persistent
  *                  thread blocks take (segment, head, query-tile pair) work items from
@@ -156,8 +177,9 @@ size_t unipin_masked_prefill_bwd_workspace_size(int total_tokens, int H);
  * Pool write ([review] §2.4: retrieval writes the past K/V of every layer
  * into the shared pool; [notes] §6: pool [L, S, H, n, D], slot reuse):
  *   pool.k[layer, slot_ids[b], h, j, :] = k[cu_seqlens[b] + j, h, :]   for j < past_lens[b]
- * and the same for v.  A byte copy (bit-exact); nothing else in the pool is
- * touched.  Slot ids within one call must be distinct (a repeated id leaves
+ * and the same for v.  Into a bfloat16 pool a byte copy (bit-exact); into an
+ * E4M3 pool each element quantized as the pool's description says.  Nothing
+ * else in the pool is touched.  Slot ids within one call must be distinct (a repeated id leaves
  * that slot holding one of the writers' rows, unspecified which).
  *   k, v           [T, H, D] bf16 with T = cu_seqlens[B]
  *   max_past       host int >= every past_lens[b] (sizes the grid)
@@ -204,11 +226,19 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
                             void* workspace, size_t workspace_bytes, int* dev_status, void* stream);
 
 /* Bytes of workspace unipin_rank_decode_attn uses at most for these sizes
- * (n_cap = the pool's rows per slot): 256 for the work counter, plus the
- * split-n partial results (and, for max_k <= 128, one arrival counter per
- * request and head) when it would split.  The split grows with the device's
- * SM count; the size returned covers the current device and a 148-SM B200. */
+ * (n_cap = the pool's rows per slot) over a bfloat16 pool: 256 for the work
+ * counter, plus the split-n partial results (and, for max_k <= 64 candidate
+ * columns, one arrival counter per request and head) when it would split.  The
+ * split grows with the device's SM count; the size returned covers the
+ * current device and a 148-SM B200. */
 size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_k, int total_cand, int n_cap);
+
+/* The same for a given pool of either dtype.  Over an UNIPIN_POOL_E4M3 pool the
+ * call first dequantizes rows 0..n_r-1 of each request's slot (layer `layer`)
+ * into bfloat16 in the workspace and then decodes from there, so it needs a
+ * workspace: this size plus R * pool->H * pool->n_cap * pool->D * 4 bytes and a
+ * little more; with less, it returns UNIPIN_ERR_INVALID_ARG. */
+size_t unipin_rank_decode_pool_workspace_size(const unipin_kvpool* pool, int R, int H, int max_k, int total_cand);
 
 /*
  * Rank decode that allocates nothing and takes no workspace.  There is no
@@ -224,6 +254,8 @@ size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_
  *   - If unipin_rank_decode_workspace_size(R, H, pool->H, D, max_k,
  *     total_cand, pool->n_cap) exceeds that size, nothing is launched and
  *     UNIPIN_ERR_OUT_OF_RANGE is returned.
+ *   - An UNIPIN_POOL_E4M3 pool is not taken (UNIPIN_ERR_UNSUPPORTED): its
+ *     dequantized rows do not fit a fixed array.
  *   - The first call on a device looks up the array's device address; make
  *     that first call before any stream capture.
  *   - Every call shares the one array and it keeps the last call's contents
@@ -256,6 +288,8 @@ typedef struct {
     unsigned long long k_offset;      /* byte offset of pool.k inside its allocation */
     unsigned long long v_offset;
     int L, S, H, n_cap, D;
+    int dtype;                        /* pool.dtype, pool.k_scale, pool.v_scale */
+    float k_scale, v_scale;
 } unipin_kvpool_share;
 
 /* Exporter side: fill *out for `pool`.  The pool's tensors must lie in memory

@@ -35,6 +35,7 @@ EXPORTS = (
     "unipin_kvpool_write",
     "unipin_rank_decode_attn",
     "unipin_rank_decode_workspace_size",
+    "unipin_rank_decode_pool_workspace_size",
     "unipin_masked_prefill_workspace_size",
     "unipin_status_string",
     "unipin_selftest_bounded_wait",
@@ -58,9 +59,13 @@ class UnipinError(RuntimeError):
         super().__init__("%s failed: %s (%d)" % (where, STATUS_NAMES.get(code, "?"), code))
 
 
+POOL_BF16, POOL_E4M3 = 0, 1    # unipin_pool_dtype
+
+
 class KVPool(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("L", ctypes.c_int), ("S", ctypes.c_int),
-                ("H", ctypes.c_int), ("n_cap", ctypes.c_int), ("D", ctypes.c_int)]
+                ("H", ctypes.c_int), ("n_cap", ctypes.c_int), ("D", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 class KVPoolShare(ctypes.Structure):
@@ -68,7 +73,7 @@ class KVPoolShare(ctypes.Structure):
     _fields_ = [("k_handle", ctypes.c_ubyte * 64), ("v_handle", ctypes.c_ubyte * 64),
                 ("k_offset", ctypes.c_ulonglong), ("v_offset", ctypes.c_ulonglong),
                 ("L", ctypes.c_int), ("S", ctypes.c_int), ("H", ctypes.c_int), ("n_cap", ctypes.c_int),
-                ("D", ctypes.c_int)]
+                ("D", ctypes.c_int), ("dtype", ctypes.c_int), ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
 
 
 def _load(path: str = _LIB_PATH):
@@ -91,6 +96,8 @@ def _load(path: str = _LIB_PATH):
     lib.unipin_rank_decode_attn.restype = I
     lib.unipin_rank_decode_workspace_size.argtypes = [I, I, I, I, I, I, I]
     lib.unipin_rank_decode_workspace_size.restype = SZ
+    lib.unipin_rank_decode_pool_workspace_size.argtypes = [P, I, I, I, I]
+    lib.unipin_rank_decode_pool_workspace_size.restype = SZ
     lib.unipin_status_string.argtypes = [I]
     lib.unipin_status_string.restype = ctypes.c_char_p
     lib.unipin_selftest_bounded_wait.argtypes = [P, ctypes.c_uint, P]
@@ -159,14 +166,24 @@ def _index(t: torch.Tensor, name: str, n: int):
         raise ValueError("%s must be a contiguous CUDA int32 tensor of length %d" % (name, n))
 
 
-def _pool(pool_k: torch.Tensor, pool_v: torch.Tensor) -> KVPool:
+_E4M3_TYPES = (torch.float8_e4m3fn, torch.uint8)
+
+
+def _pool(pool_k: torch.Tensor, pool_v: torch.Tensor, pool_scales=None) -> KVPool:
+    """A pool descriptor: bfloat16 tensors, or E4M3 codes (float8_e4m3fn or uint8) with
+    pool_scales = (k_scale, v_scale) (default (1, 1))."""
     for name, t in (("pool_k", pool_k), ("pool_v", pool_v)):
-        if t.dtype != torch.bfloat16 or t.dim() != 5 or not t.is_contiguous() or not t.is_cuda:
-            raise ValueError("%s must be a contiguous CUDA bfloat16 tensor [L, S, H, n_cap, D]" % name)
-    if pool_k.shape != pool_v.shape:
-        raise ValueError("pool_k and pool_v differ in shape")
+        if (t.dtype != torch.bfloat16 and t.dtype not in _E4M3_TYPES) or t.dim() != 5 or not t.is_contiguous() \
+                or not t.is_cuda:
+            raise ValueError("%s must be a contiguous CUDA tensor [L, S, H, n_cap, D] of bfloat16 or E4M3 codes "
+                             "(float8_e4m3fn or uint8)" % name)
+    if pool_k.shape != pool_v.shape or (pool_k.dtype == torch.bfloat16) != (pool_v.dtype == torch.bfloat16):
+        raise ValueError("pool_k and pool_v differ in shape or element type")
     L, S, H, n_cap, D = pool_k.shape
-    return KVPool(pool_k.data_ptr(), pool_v.data_ptr(), L, S, H, n_cap, D)
+    if pool_k.dtype == torch.bfloat16:
+        return KVPool(pool_k.data_ptr(), pool_v.data_ptr(), L, S, H, n_cap, D, POOL_BF16, 1.0, 1.0)
+    ks, vs = (1.0, 1.0) if pool_scales is None else (float(pool_scales[0]), float(pool_scales[1]))
+    return KVPool(pool_k.data_ptr(), pool_v.data_ptr(), L, S, H, n_cap, D, POOL_E4M3, ks, vs)
 
 
 def _workspace(workspace, nbytes: int, device):
@@ -190,9 +207,9 @@ def masked_prefill_workspace_size() -> int:
 
 def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=None, out_fp32: bool = True,
                         scale: Optional[float] = None, pool_k=None, pool_v=None, slot_ids=None, layer: int = 0,
-                        workspace="auto", dev_status=None, stream=None, lse=None):
-    """M-FALCON masked prefill; optionally also writes the past K/V into pool slots and the per-row
-    log-sum-exp (base 2, fp32 [T, H]) into `lse`."""
+                        workspace="auto", dev_status=None, stream=None, lse=None, pool_scales=None):
+    """M-FALCON masked prefill; optionally also writes the past K/V into pool slots (an E4M3 pool
+    takes pool_scales = (k_scale, v_scale)) and the per-row log-sum-exp (base 2, fp32 [T, H]) into `lse`."""
     _tokens(q, "q")
     T, H, D = q.shape
     _tokens(k, "k", D)
@@ -207,7 +224,7 @@ def masked_prefill_attn(q, k, v, cu_seqlens, past_lens, max_seqlen: int, out=Non
         raise ValueError("out has the wrong dtype or shape")
     pool = None
     if pool_k is not None:
-        pool = _pool(pool_k, pool_v)
+        pool = _pool(pool_k, pool_v, pool_scales)
         _index(slot_ids, "slot_ids", B)
     if lse is not None and (lse.dtype != torch.float32 or lse.shape != (T, H) or not lse.is_contiguous()):
         raise ValueError("lse must be a contiguous float32 tensor [T, H]")
@@ -259,9 +276,10 @@ def masked_prefill_bwd(q, k, v, out, dout, lse, cu_seqlens, past_lens, max_seqle
 
 
 def kvpool_write(pool_k, pool_v, layer: int, k, v, cu_seqlens, past_lens, slot_ids, max_past: int,
-                 dev_status=None, stream=None):
-    """Byte copy of each segment's past K/V rows into its pool slot at `layer`."""
-    pool = _pool(pool_k, pool_v)
+                 dev_status=None, stream=None, pool_scales=None):
+    """Each segment's past K/V rows into its pool slot at `layer`: a byte copy into a bfloat16 pool,
+    E4M3 codes of k / k_scale and v / v_scale into an E4M3 pool."""
+    pool = _pool(pool_k, pool_v, pool_scales)
     _tokens(k, "k", pool.D)
     _tokens(v, "v", pool.D)
     B = past_lens.shape[0]
@@ -281,15 +299,25 @@ def rank_decode_workspace_size(R: int, H: int, D: int, max_k: int, total_cand: i
                                                       n_cap))
 
 
+def rank_decode_pool_workspace_size(pool_k, pool_v, R: int, H: int, max_k: int, total_cand: int,
+                                    pool_scales=None) -> int:
+    """Workspace bytes of rank_decode_attn over this pool (an E4M3 pool also needs room for its
+    dequantized rows)."""
+    pool = _pool(pool_k, pool_v, pool_scales)
+    return int(LIB.unipin_rank_decode_pool_workspace_size(ctypes.byref(pool), int(R), int(H), int(max_k),
+                                                          int(total_cand)))
+
+
 def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, pool_v, layer: int, max_k: int,
                      out=None, out_fp32: bool = True, scale: Optional[float] = None, workspace="auto",
-                     dev_status=None, stream=None):
-    """Candidates attend to their slot's cached past rows plus themselves."""
+                     dev_status=None, stream=None, pool_scales=None):
+    """Candidates attend to their slot's cached past rows plus themselves (a bfloat16 pool, or an
+    E4M3 pool with pool_scales = (k_scale, v_scale))."""
     _tokens(q_c, "q_c")
     T, H, D = q_c.shape
     _tokens(k_c, "k_c", D)
     _tokens(v_c, "v_c", D)
-    pool = _pool(pool_k, pool_v)
+    pool = _pool(pool_k, pool_v, pool_scales)
     if _kv_heads(q_c, k_c, v_c) != pool.H:
         raise ValueError("k_c and v_c must have the pool's %d key/value heads" % pool.H)
     R = past_lens.shape[0]
@@ -300,8 +328,8 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
         out = torch.empty((T, H, D), dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q_c.device)
     elif out.dtype != (torch.float32 if out_fp32 else torch.bfloat16) or out.shape != q_c.shape or not out.is_contiguous():
         raise ValueError("out has the wrong dtype or shape")
-    ws, ws_bytes = _workspace(workspace, rank_decode_workspace_size(R, H, D, int(max_k), T, pool.n_cap, pool.H)
-                              if isinstance(workspace, str) else 0, q_c.device)
+    ws, ws_bytes = _workspace(workspace, int(LIB.unipin_rank_decode_pool_workspace_size(
+        ctypes.byref(pool), R, H, int(max_k), T)) if isinstance(workspace, str) else 0, q_c.device)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     rc = LIB.unipin_rank_decode_attn(_ptr(q_c), _ptr(k_c), _ptr(v_c), _ptr(out), int(bool(out_fp32)),
                                      _ptr(cu_seqlens_c), _ptr(slot_ids), _ptr(past_lens), R, H, D, int(max_k), T,
@@ -313,7 +341,7 @@ def rank_decode_attn(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, p
 
 def rank_decode_attn_noalloc(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, pool_k, pool_v, layer: int,
                              max_k: int, out, out_fp32: bool = True, scale: Optional[float] = None,
-                             dev_status=None, stream=None):
+                             dev_status=None, stream=None, pool_scales=None):
     """Rank decode through the entry point that allocates nothing (the caller passes `out`).
 
     For callers that cannot allocate device memory while serving: the scratch
@@ -324,7 +352,7 @@ def rank_decode_attn_noalloc(q_c, k_c, v_c, cu_seqlens_c, slot_ids, past_lens, p
     T, H, D = q_c.shape
     _tokens(k_c, "k_c", D)
     _tokens(v_c, "v_c", D)
-    pool = _pool(pool_k, pool_v)
+    pool = _pool(pool_k, pool_v, pool_scales)
     if _kv_heads(q_c, k_c, v_c) != pool.H:
         raise ValueError("k_c and v_c must have the pool's %d key/value heads" % pool.H)
     R = past_lens.shape[0]
@@ -366,9 +394,9 @@ def status_string(code: int) -> str:
 
 # ------------------------------------------------- pool sharing and slot ring
 
-def kvpool_share_export(pool_k: torch.Tensor, pool_v: torch.Tensor) -> bytes:
+def kvpool_share_export(pool_k: torch.Tensor, pool_v: torch.Tensor, pool_scales=None) -> bytes:
     """IPC description of a pool (bytes to hand to another process, e.g. through a file)."""
-    pool = _pool(pool_k, pool_v)
+    pool = _pool(pool_k, pool_v, pool_scales)
     desc = KVPoolShare()
     _check(LIB.unipin_kvpool_share_export(ctypes.byref(pool), ctypes.byref(desc)), "unipin_kvpool_share_export")
     return bytes(desc)
@@ -377,16 +405,17 @@ def kvpool_share_export(pool_k: torch.Tensor, pool_v: torch.Tensor) -> bytes:
 class _DeviceArray:
     """A zero-copy view of device memory owned elsewhere, for torch.as_tensor."""
 
-    def __init__(self, ptr: int, shape):
-        self.__cuda_array_interface__ = {"shape": tuple(int(x) for x in shape), "typestr": "<i2",
+    def __init__(self, ptr: int, shape, typestr: str = "<i2"):
+        self.__cuda_array_interface__ = {"shape": tuple(int(x) for x in shape), "typestr": typestr,
                                          "data": (int(ptr), False), "version": 3, "strides": None}
 
 
 class SharedPool:
     """A pool exported by another process, mapped into this one.
 
-    ``k`` and ``v`` are bf16 tensors [L, S, H, n_cap, D] over the exporter's
-    memory, usable with every call of this module; ``close()`` unmaps them.
+    ``k`` and ``v`` are tensors [L, S, H, n_cap, D] over the exporter's memory
+    (bfloat16, or float8_e4m3fn codes with ``scales`` = (k_scale, v_scale)),
+    usable with every call of this module; ``close()`` unmaps them.
     """
 
     def __init__(self, desc: bytes, device=None):
@@ -399,8 +428,13 @@ class SharedPool:
         d = self._desc
         shape = (d.L, d.S, d.H, d.n_cap, d.D)
         dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
-        self.k = torch.as_tensor(_DeviceArray(self._pool.k, shape), device=dev).view(torch.bfloat16)
-        self.v = torch.as_tensor(_DeviceArray(self._pool.v, shape), device=dev).view(torch.bfloat16)
+        if d.dtype == POOL_E4M3:
+            self.k = torch.as_tensor(_DeviceArray(self._pool.k, shape, "|u1"), device=dev).view(torch.float8_e4m3fn)
+            self.v = torch.as_tensor(_DeviceArray(self._pool.v, shape, "|u1"), device=dev).view(torch.float8_e4m3fn)
+        else:
+            self.k = torch.as_tensor(_DeviceArray(self._pool.k, shape), device=dev).view(torch.bfloat16)
+            self.v = torch.as_tensor(_DeviceArray(self._pool.v, shape), device=dev).view(torch.bfloat16)
+        self.scales = (d.k_scale, d.v_scale)
 
     def close(self):
         if self._pool.k:

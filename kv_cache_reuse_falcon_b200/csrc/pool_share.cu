@@ -34,14 +34,15 @@ PFN_getAddressRange address_range_fn()
     return fn;
 }
 
-bool pool_shape_ok(int L, int S, int H, int n_cap, int D)
+bool pool_shape_ok(int L, int S, int H, int n_cap, int D, int dtype)
 {
-    return L >= 1 && S >= 1 && H >= 1 && n_cap >= 1 && (D == 32 || D == 64 || D == 128);
+    return L >= 1 && S >= 1 && H >= 1 && n_cap >= 1 && (D == 32 || D == 64 || D == 128) &&
+           (dtype == UNIPIN_POOL_BF16 || dtype == UNIPIN_POOL_E4M3);
 }
 
-size_t pool_bytes(int L, int S, int H, int n_cap, int D)
+size_t pool_bytes(int L, int S, int H, int n_cap, int D, int dtype)
 {
-    return (size_t)L * S * H * n_cap * D * 2;
+    return (size_t)L * S * H * n_cap * D * (dtype == UNIPIN_POOL_E4M3 ? 1 : 2);
 }
 
 // Handle and byte offset of the allocation that holds [ptr, ptr + bytes).
@@ -79,10 +80,10 @@ extern "C" {
 int unipin_kvpool_share_export(const unipin_kvpool* pool, unipin_kvpool_share* out)
 {
     if (!pool || !out || !pool->k || !pool->v) return UNIPIN_ERR_INVALID_ARG;
-    if (!pool_shape_ok(pool->L, pool->S, pool->H, pool->n_cap, pool->D)) return UNIPIN_ERR_INVALID_ARG;
+    if (!pool_shape_ok(pool->L, pool->S, pool->H, pool->n_cap, pool->D, pool->dtype)) return UNIPIN_ERR_INVALID_ARG;
     unipin_kvpool_share s;
     std::memset(&s, 0, sizeof(s));
-    const size_t bytes = pool_bytes(pool->L, pool->S, pool->H, pool->n_cap, pool->D);
+    const size_t bytes = pool_bytes(pool->L, pool->S, pool->H, pool->n_cap, pool->D, pool->dtype);
     int rc = export_one(pool->k, bytes, s.k_handle, s.k_offset);
     if (rc == UNIPIN_OK) rc = export_one(pool->v, bytes, s.v_handle, s.v_offset);
     if (rc != UNIPIN_OK) return rc;
@@ -91,6 +92,9 @@ int unipin_kvpool_share_export(const unipin_kvpool* pool, unipin_kvpool_share* o
     s.H = pool->H;
     s.n_cap = pool->n_cap;
     s.D = pool->D;
+    s.dtype = pool->dtype;
+    s.k_scale = pool->k_scale;
+    s.v_scale = pool->v_scale;
     *out = s;
     return UNIPIN_OK;
 }
@@ -98,7 +102,7 @@ int unipin_kvpool_share_export(const unipin_kvpool* pool, unipin_kvpool_share* o
 int unipin_kvpool_share_open(const unipin_kvpool_share* in, unipin_kvpool* out)
 {
     if (!in || !out) return UNIPIN_ERR_INVALID_ARG;
-    if (!pool_shape_ok(in->L, in->S, in->H, in->n_cap, in->D)) return UNIPIN_ERR_INVALID_ARG;
+    if (!pool_shape_ok(in->L, in->S, in->H, in->n_cap, in->D, in->dtype)) return UNIPIN_ERR_INVALID_ARG;
     cudaIpcMemHandle_t hk, hv;
     std::memcpy(&hk, in->k_handle, sizeof(hk));
     std::memcpy(&hv, in->v_handle, sizeof(hv));
@@ -120,6 +124,9 @@ int unipin_kvpool_share_open(const unipin_kvpool_share* in, unipin_kvpool* out)
     out->H = in->H;
     out->n_cap = in->n_cap;
     out->D = in->D;
+    out->dtype = in->dtype;
+    out->k_scale = in->k_scale;
+    out->v_scale = in->v_scale;
     return UNIPIN_OK;
 }
 

@@ -187,6 +187,11 @@ int check_pool(const unipin_kvpool* pool, int H, int D, int layer)
     if (!pool || !pool->k || !pool->v) return UNIPIN_ERR_INVALID_ARG;
     if (pool->L < 1 || pool->S < 1 || pool->n_cap < 1 || pool->H < 1 || H % pool->H != 0 || pool->D != D)
         return UNIPIN_ERR_INVALID_ARG;
+    if (pool->dtype != UNIPIN_POOL_BF16 && pool->dtype != UNIPIN_POOL_E4M3) return UNIPIN_ERR_INVALID_ARG;
+    if (pool->dtype == UNIPIN_POOL_E4M3 &&
+        (!(pool->k_scale > 0.f) || !std::isfinite(pool->k_scale) || !(pool->v_scale > 0.f) ||
+         !std::isfinite(pool->v_scale) || !std::isfinite(1.f / pool->k_scale) || !std::isfinite(1.f / pool->v_scale)))
+        return UNIPIN_ERR_INVALID_ARG;
     if (!aligned16(pool->k) || !aligned16(pool->v)) return UNIPIN_ERR_MISALIGNED;
     if (layer < 0 || layer >= pool->L) return UNIPIN_ERR_OUT_OF_RANGE;
     if ((uint64_t)pool->L * pool->S * pool->H >= (1ull << 31)) return UNIPIN_ERR_INVALID_ARG;
@@ -222,6 +227,30 @@ int launch_pool_write(const unipin_kvpool* pool, int layer, const void* k, const
                       int* status, cudaStream_t s)
 {
     if (B == 0 || max_past == 0) return UNIPIN_OK;
+    const long long vecs = (long long)max_past * (D / 8);
+    const long long blocks = (vecs + 255) / 256;
+    dim3 grid((unsigned)(blocks < 65535 ? blocks : 65535), (unsigned)H, (unsigned)B);
+    if (pool->dtype == UNIPIN_POOL_E4M3) {
+        PoolWriteE4M3Params q;
+        q.k = static_cast<const uint4*>(k);
+        q.v = static_cast<const uint4*>(v);
+        q.pool_k = static_cast<uint2*>(pool->k);
+        q.pool_v = static_cast<uint2*>(pool->v);
+        q.cu = cu;
+        q.past = past;
+        q.slots = slots;
+        q.H = H;
+        q.D = D;
+        q.S = pool->S;
+        q.n_cap = pool->n_cap;
+        q.layer = layer;
+        q.total_tokens = total_tokens;
+        q.inv_k = 1.f / pool->k_scale;
+        q.inv_v = 1.f / pool->v_scale;
+        q.status = status;
+        kvpool_write_e4m3_kernel<<<grid, 256, 0, s>>>(q);
+        return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
+    }
     PoolWriteParams p;
     p.k = static_cast<const uint4*>(k);
     p.v = static_cast<const uint4*>(v);
@@ -237,9 +266,6 @@ int launch_pool_write(const unipin_kvpool* pool, int layer, const void* k, const
     p.layer = layer;
     p.total_tokens = total_tokens;
     p.status = status;
-    const long long vecs = (long long)max_past * (D / 8);
-    const long long blocks = (vecs + 255) / 256;
-    dim3 grid((unsigned)(blocks < 65535 ? blocks : 65535), (unsigned)H, (unsigned)B);
     kvpool_write_kernel<<<grid, 256, 0, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
@@ -486,6 +512,55 @@ int noalloc_scratch_address(void** addr)
     return UNIPIN_OK;
 }
 
+// An E4M3 pool is decoded from bfloat16 rows expanded into the workspace: the
+// remapped slot ids [R] (256-byte block), then K and V of a pool [1, R, H, n_cap, D].
+size_t dequant_slab_bytes(const unipin_kvpool* pool, int R)
+{
+    const size_t rows = (size_t)R * pool->H * pool->n_cap * pool->D;
+    return ((size_t)R * sizeof(int) + 255) / 256 * 256 + 2 * ((rows * 2 + 255) / 256 * 256);
+}
+
+int rank_decode_e4m3(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
+                     const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H, int D,
+                     int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer, void* workspace,
+                     size_t workspace_bytes, int* dev_status, cudaStream_t s)
+{
+    const size_t slab = dequant_slab_bytes(pool, R);
+    if (!workspace || workspace_bytes < slab) return UNIPIN_ERR_INVALID_ARG;
+    if (R > 65535 || pool->H > 65535) return UNIPIN_ERR_INVALID_ARG;
+    char* ws = static_cast<char*>(workspace);
+    const size_t slots_bytes = ((size_t)R * sizeof(int) + 255) / 256 * 256;
+    const size_t plane = (((size_t)R * pool->H * pool->n_cap * pool->D) * 2 + 255) / 256 * 256;
+    unipin_kvpool bf = *pool;
+    bf.k = ws + slots_bytes;
+    bf.v = ws + slots_bytes + plane;
+    bf.L = 1;
+    bf.S = R;
+    bf.dtype = UNIPIN_POOL_BF16;
+    PoolDequantParams p;
+    p.pool_k = static_cast<const uint2*>(pool->k);
+    p.pool_v = static_cast<const uint2*>(pool->v);
+    p.out_k = static_cast<uint4*>(bf.k);
+    p.out_v = static_cast<uint4*>(bf.v);
+    p.out_slots = reinterpret_cast<int*>(ws);
+    p.past = past_lens;
+    p.slots = slot_ids;
+    p.H = pool->H;
+    p.D = D;
+    p.S = pool->S;
+    p.n_cap = pool->n_cap;
+    p.layer = layer;
+    p.k_scale = pool->k_scale;
+    p.v_scale = pool->v_scale;
+    const long long vecs = (long long)pool->n_cap * (D / 8);
+    const long long blocks = (vecs + 255) / 256;
+    dim3 grid((unsigned)(blocks < 65535 ? blocks : 65535), (unsigned)pool->H, (unsigned)R);
+    kvpool_dequant_kernel<<<grid, 256, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return UNIPIN_ERR_CUDA;
+    return unipin_rank_decode_attn(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, p.out_slots, past_lens, R, H, D, max_k,
+                                   total_cand, scale, &bf, 0, ws + slab, workspace_bytes - slab, dev_status, s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -539,8 +614,10 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     if ((rc = make_token_map(&tq, q, total_tokens, H, D, kBlockM)) != UNIPIN_OK) return rc;
     if ((rc = make_token_map(&tk, k, total_tokens, H_kv, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
     if ((rc = make_token_map(&tv, v, total_tokens, H_kv, D, key_tile_width(D, false))) != UNIPIN_OK) return rc;
-    if (pool) {
-        // the past K/V tiles the kernel loads are also stored into the pool (no second pass)
+    // A bfloat16 pool takes the past K/V tiles the kernel loads anyway (no second
+    // pass); an E4M3 pool is written by the quantizing pool-write kernel after it.
+    const bool fuse_pool = pool && pool->dtype == UNIPIN_POOL_BF16;
+    if (fuse_pool) {
         if ((rc = make_pool_map(&tpk, pool->k, pool, key_tile_width(D, false))) != UNIPIN_OK) return rc;
         if ((rc = make_pool_map(&tpv, pool->v, pool, key_tile_width(D, false))) != UNIPIN_OK) return rc;
     } else {
@@ -568,7 +645,7 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     p.wait_limit_ns = wait_limit_ns();
     p.sched = sched;
     p.lse = lse;
-    if (pool) {
+    if (fuse_pool) {
         p.store_pool = 1;
         p.pool_k = pool->k;
         p.pool_v = pool->v;
@@ -579,7 +656,11 @@ int unipin_masked_prefill_attn(const void* q, const void* k, const void* v, void
     }
     const long long bound = (long long)B * H * ((max_seqlen + kPairRows - 1) / kPairRows);
     dim3 grid(persistent_blocks(bound), 1, 1);
-    return launch_attn<false>(D, grid, tq, tk, tv, tpk, tpv, p, s);
+    rc = launch_attn<false>(D, grid, tq, tk, tv, tpk, tpv, p, s);
+    if (rc != UNIPIN_OK || !pool || fuse_pool) return rc;
+    if (B > 65535 || pool->H > 65535) return UNIPIN_ERR_INVALID_ARG;
+    return launch_pool_write(pool, layer, k, v, cu_seqlens, past_lens, slot_ids, B, pool->H, D, max_seqlen,
+                             total_tokens, dev_status, s);
 }
 
 int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, const void* v, const int* cu_seqlens,
@@ -614,6 +695,14 @@ size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_
     return decode_workspace_bytes(decode_nsplit(R, H, D, max_k, n_cap, sms), total_cand, H, D);
 }
 
+size_t unipin_rank_decode_pool_workspace_size(const unipin_kvpool* pool, int R, int H, int max_k, int total_cand)
+{
+    if (!pool || pool->H < 1 || H < 1 || H % pool->H != 0) return 0;
+    const size_t base = unipin_rank_decode_workspace_size(R, H, pool->H, pool->D, max_k, total_cand, pool->n_cap);
+    if (base == 0 || pool->dtype != UNIPIN_POOL_E4M3) return base;
+    return dequant_slab_bytes(pool, R) + base;
+}
+
 int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, void* out, int out_fp32,
                             const int* cu_seqlens_c, const int* slot_ids, const int* past_lens, int R, int H, int D,
                             int max_k, int total_cand, float scale, const unipin_kvpool* pool, int layer,
@@ -631,6 +720,9 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pool->dtype == UNIPIN_POOL_E4M3)
+        return rank_decode_e4m3(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, slot_ids, past_lens, R, H, D, max_k,
+                                total_cand, scale, pool, layer, workspace, workspace_bytes, dev_status, s);
     if (use_small_k(D, max_k, H / pool->H))
         return rank_decode_small_k(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, slot_ids, past_lens, R, H, D, max_k,
                                    total_cand, scale, pool, layer, workspace, workspace_bytes, dev_status, s);
@@ -708,6 +800,7 @@ int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void
     if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
     if (R == 0 || total_cand == 0 || max_k == 0) return UNIPIN_OK;
     if (pool->H < 1 || H % pool->H != 0) return UNIPIN_ERR_INVALID_ARG;
+    if (pool->dtype == UNIPIN_POOL_E4M3) return UNIPIN_ERR_UNSUPPORTED;
     const size_t need = unipin_rank_decode_workspace_size(R, H, pool->H, D, max_k, total_cand, pool->n_cap);
     if (need > kNoAllocScratchBytes) return UNIPIN_ERR_OUT_OF_RANGE;
     void* scratch = nullptr;

@@ -81,6 +81,43 @@ def test_host_validation_needs_no_device(lib):
     assert wp() == 256
 
 
+class Pool(ctypes.Structure):
+    """unipin_kvpool as include/unipin.h declares it."""
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("L", ctypes.c_int), ("S", ctypes.c_int),
+                ("H", ctypes.c_int), ("n_cap", ctypes.c_int), ("D", ctypes.c_int), ("dtype", ctypes.c_int),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float)]
+
+
+def test_e4m3_pool_host_rules_need_no_device(lib):
+    """The E4M3 pool's workspace size and the calls that refuse it are host-side decisions."""
+    P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    ws = lib.unipin_rank_decode_pool_workspace_size
+    ws.argtypes = [P, I, I, I, I]
+    ws.restype = SZ
+    g = lib.unipin_rank_decode_workspace_size
+    g.argtypes = [I, I, I, I, I, I, I]
+    g.restype = SZ
+    bf = Pool(16, 16, 1, 4, 2, 512, 64, 0, 1.0, 1.0)
+    f8 = Pool(16, 16, 1, 4, 2, 512, 64, 1, 0.5, 0.25)
+    base = g(3, 4, 2, 64, 16, 48, 512)
+    assert ws(ctypes.byref(bf), 3, 4, 16, 48) == base
+    # the dequantized rows: 3 requests x 2 heads x 512 rows x 64 bf16, for K and V, and the slot ids
+    assert ws(ctypes.byref(f8), 3, 4, 16, 48) >= base + 2 * 3 * 2 * 512 * 64 * 2 + 3 * 4
+    assert ws(ctypes.byref(f8), 3, 3, 16, 48) == 0          # query heads not a multiple of the pool's
+    na = lib.unipin_rank_decode_attn_noalloc
+    na.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, ctypes.c_float, P, I, P, P]
+    na.restype = I
+    assert na(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), 3, 4, 64, 16, 48, 0.1, ctypes.byref(f8), 0,
+              None, None) == -2                              # E4M3 pools are not taken by the no-alloc call
+    dec = lib.unipin_rank_decode_attn
+    dec.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, ctypes.c_float, P, I, P, SZ, P, P]
+    dec.restype = I
+    for bad in (Pool(16, 16, 1, 4, 2, 512, 64, 2, 1.0, 1.0), Pool(16, 16, 1, 4, 2, 512, 64, 1, 0.0, 1.0),
+                Pool(16, 16, 1, 4, 2, 512, 64, 1, 1.0, float("inf"))):
+        assert dec(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), 3, 4, 64, 16, 48, 0.1, ctypes.byref(bad), 0,
+                   None, 0, None, None) == -1                # unknown dtype, scales not finite and positive
+
+
 def test_binding_refuses_to_load_without_library(tmp_path):
     from kv_cache_reuse_falcon_b200 import binding
     with pytest.raises(ImportError):

@@ -100,6 +100,6 @@ def test_share_calls_check_their_arguments_without_a_device():
     assert lib.unipin_kvpool_share_open(ctypes.byref(desc), None) == -1
     assert lib.unipin_kvpool_share_open(ctypes.byref(desc), ctypes.byref(pool)) == -1      # zero shape
     assert lib.unipin_kvpool_share_close(ctypes.byref(desc), ctypes.byref(pool)) == -1     # nothing open
-    assert ctypes.sizeof(ub.KVPoolShare) == 168
+    assert ctypes.sizeof(ub.KVPoolShare) == 176    # handles, offsets, shape, dtype and the two scales
     with pytest.raises(ValueError):
         ub.SharedPool(b"short")
