@@ -71,8 +71,9 @@ def pool_write_bytes(past, H, D):
 # by the kernel source it was taken on.  A changed kernel reports null until
 # it is captured again.
 _PREFILL_TRAFFIC_PER_TOKEN = {
-    # kernel_source_key() of csrc/attn_sm100.cuh, H, D: bytes per token
-    ("03012fff8e2df70c", 8, 128): (431.669760e6 + 123.166208e6) / 70236,
+    # kernel_source_key() of csrc/attn_sm100.cuh, H, D: bytes per token (reads + writes,
+    # the writes including the fused store of the past K/V into the pool)
+    ("aa4830eb8ccb19ef", 8, 128): (432.141056e6 + 292.076544e6) / 70236,
 }
 
 
@@ -725,8 +726,10 @@ def run_decode_only(args, rank, world, device, dist):
              "frac": gbs / peaks["hbm_gbs"]} if bound == "hbm" else
             {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
              "frac": tflops / peaks["bf16_tflops"]})
-    roof.update({"kernel": "attn_fwd_kernel<%d,decode>" % D, "traffic": None,
-                 "peak_source": "%s (burst for tensor)" % peaks["source"]})
+    # the library sends requests of at most 64 candidates (one query head per kv head) to the small-k kernel
+    kernel = ("decode_smallk_kernel<%d,%d>" % (D, 16 if kk <= 16 else 32 if kk <= 32 else 64)
+              if kk <= 64 and D in (64, 128) else "attn_fwd_kernel<%d,decode>" % D)
+    roof.update({"kernel": kernel, "traffic": None, "peak_source": "%s (burst for tensor)" % peaks["source"]})
     return {
         "metric": METRIC, "value": float(cand.sum()) * L / (ms_step * 1e-3), "unit": "candidate tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -741,6 +744,71 @@ def run_decode_only(args, rank, world, device, dist):
                    "roof_time_ms": 1e3 * max(t_hbm, t_tc)},
         "roofline": roof, "gpu_launches": args.steps * L * (2 if (ws_bytes > 256 and kk > 128) else 1),
         "clocks": clk,
+    }
+
+
+def run_backward_only(args, rank, world, device, dist):
+    """Gradients of the masked prefill: one forward for out and lse, then the timed backward calls."""
+    import torch
+    from kv_cache_reuse_falcon_b200 import binding as ub
+
+    w = synth.workload(args.workload)
+    rng = np.random.Generator(np.random.PCG64(rank_seed(w.seed, rank)))
+    past, cand = w.lengths(rng)
+    cu_h = synth.cu_from_lens(past + cand)
+    T = int(cu_h[-1])
+
+    def dev_bf16(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+    q, k, v, g = (dev_bf16(synth.normal_bf16(rng, (T, w.H, w.D))) for _ in range(4))
+    cu = torch.from_numpy(cu_h).to(device)
+    pl = torch.from_numpy(past).to(device)
+    max_len = int((past + cand).max())
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    stream = torch.cuda.current_stream(device)
+    lse = torch.empty((T, w.H), dtype=torch.float32, device=device)
+    o = ub.masked_prefill_attn(q, k, v, cu, pl, max_len, out_fp32=False, lse=lse, dev_status=status)
+    grads = [torch.empty((T, w.H, w.D), dtype=torch.float32, device=device) for _ in range(3)]
+    ws = torch.empty(ub.masked_prefill_bwd_workspace_size(T, w.H) // 4 + 4, dtype=torch.float32, device=device)
+
+    def step():
+        ub.masked_prefill_bwd(q, k, v, o, g, lse, cu, pl, max_len, dq=grads[0], dk=grads[1], dv=grads[2],
+                              workspace=ws, dev_status=status, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if clocks:
+        clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    for i in range(args.steps):
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop() if clocks else None
+    if int(status.item()) != 0:
+        raise RuntimeError("device status %s" % ub.status_string(int(status.item())))
+    ms_step = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    peaks = load_peaks()
+    flops = 2.5 * prefill_flops(past, cand, w.H, w.D)
+    e = roof_entry(ms_step, flops, 5 * T * w.H * w.D * 2 + 3 * T * w.H * w.D * 4 + 2 * T * w.H * 4, peaks,
+                   "bwd_prep_kernel<%d> + bwd_kv_kernel<%d>" % (w.D, w.D))
+    return {
+        "metric": METRIC, "value": float(T) / (ms_step * 1e-3), "unit": "tokens/s (backward)",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "n": w.n, "k": w.k, "H": w.H, "D": w.D, "tokens": T,
+                   "l2": "inputs larger than L2 (no flush)"},
+        "roofline": {"bound": e["bound"], "achieved": e["tflops"] if e["bound"] == "tensor" else e["gbs"],
+                     "peak": peaks["bf16_tflops"] if e["bound"] == "tensor" else peaks["hbm_gbs"],
+                     "unit": "TFLOP/s" if e["bound"] == "tensor" else "GB/s", "frac": e["frac_roof"],
+                     "kernel": e["kernel"], "traffic": None, "peak_source": peaks["source"]},
+        "gpu_launches": args.steps * 2, "clocks": clk,
     }
 
 
@@ -847,6 +915,8 @@ def main(argv=None):
     try:
         if synth.workload(args.workload).kind == "decode":
             res = run_decode_only(args, rank, world, device, dist)
+        elif synth.workload(args.workload).kind == "backward":
+            res = run_backward_only(args, rank, world, device, dist)
         else:
             res = run_ours(args, rank, world, device, dist)
     finally:

@@ -177,7 +177,7 @@ def ragged_lengths(rng: np.random.Generator, B: int, n_lo: int, n_hi: int, k_lo:
 @dataclasses.dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str          # "prefill", "prefill+pool", "decode", "ragged"
+    kind: str          # "prefill", "prefill+pool", "decode", "ragged", "backward"
     B: int
     H: int
     D: int
@@ -211,6 +211,8 @@ WORKLOADS: List[Workload] = [
     Workload("ragged_B256_H8_D128_n32-4096_k50-2000", "ragged", B=256, H=8, D=128,
              L=1, S=256, n_cap=4096, ragged=(32, 4096, 50, 2000)),
     Workload("table2_B8_H8_D64_n992_k656", "prefill", B=8, H=8, D=64, n=992, k=656),
+    # gradients of the masked prefill (joint training) at the prefill shape
+    Workload("backward_B64_H8_D64_n256_k128", "backward", B=64, H=8, D=64, n=256, k=128),
 ]
 
 
