@@ -534,31 +534,33 @@ def run_sweep(device, peaks, iters=10, warm=3):
         del q, k, v, o, kw
         torch.cuda.empty_cache()
 
-    # gradients of the prefill workload (B=64, n=256, k=128, D=64): forward with its row
-    # statistic once, then the backward call timed; FLOPs = 10*D per allowed pair (S, dP,
+    # gradients of the prefill workload (B=64, n=256, k=128) at D=64 and D=128: forward with its
+    # row statistic once, then the backward call timed; FLOPs = 10*D per allowed pair (S, dP,
     # dV, dK, dQ products)
     w = synth.workload("prefill_B64")
     past = np.full(w.B, w.n, np.int32)
     cand = np.full(w.B, w.k, np.int32)
     T = int((past + cand).sum())
-    q, k, v, g = (randn((T, w.H, w.D), w.seed + j) for j in range(4))
     cu = torch.from_numpy(synth.cu_from_lens(past + cand)).to(device)
     pl = torch.from_numpy(past).to(device)
-    lse = torch.empty((T, w.H), dtype=torch.float32, device=device)
-    o = ub.masked_prefill_attn(q, k, v, cu, pl, w.n + w.k, out_fp32=False, lse=lse, dev_status=status)
-    grads = [torch.empty((T, w.H, w.D), dtype=torch.float32, device=device) for _ in range(3)]
-    wsb = torch.empty(ub.masked_prefill_bwd_workspace_size(T, w.H) // 4 + 4, dtype=torch.float32, device=device)
+    for D in (64, 128):
+        q, k, v, g = (randn((T, w.H, D), w.seed + j) for j in range(4))
+        lse = torch.empty((T, w.H), dtype=torch.float32, device=device)
+        o = ub.masked_prefill_attn(q, k, v, cu, pl, w.n + w.k, out_fp32=False, lse=lse, dev_status=status)
+        grads = [torch.empty((T, w.H, D), dtype=torch.float32, device=device) for _ in range(3)]
+        wsb = torch.empty(ub.masked_prefill_bwd_workspace_size(T, w.H) // 4 + 4, dtype=torch.float32,
+                          device=device)
 
-    def fn_bwd():
-        ub.masked_prefill_bwd(q, k, v, o, g, lse, cu, pl, w.n + w.k, dq=grads[0], dk=grads[1], dv=grads[2],
-                              workspace=wsb, dev_status=status, stream=stream)
+        def fn_bwd():
+            ub.masked_prefill_bwd(q, k, v, o, g, lse, cu, pl, w.n + w.k, dq=grads[0], dk=grads[1], dv=grads[2],
+                                  workspace=wsb, dev_status=status, stream=stream)
 
-    ms = timed(fn_bwd)
-    flops = 2.5 * prefill_flops(past, cand, w.H, w.D)
-    nbytes = 5 * T * w.H * w.D * 2 + 3 * T * w.H * w.D * 4 + 2 * T * w.H * 4
-    e = roof_entry(ms, flops, nbytes, peaks, "bwd_prep_kernel<64> + bwd_kv_kernel<64>")
-    out["backward_B64_n256_k128_D64"] = e
-    del q, k, v, g, o, grads, lse
+        ms = timed(fn_bwd)
+        flops = 2.5 * prefill_flops(past, cand, w.H, D)
+        nbytes = 5 * T * w.H * D * 2 + 3 * T * w.H * D * 4 + 2 * T * w.H * 4
+        e = roof_entry(ms, flops, nbytes, peaks, "bwd_prep_kernel<%d> + bwd_kv_kernel<%d>" % (D, D))
+        out["backward_B64_n256_k128_D%d" % D] = e
+        del q, k, v, g, o, grads, lse
 
     # rank decode from the [12, 256, 8, 2048, 64] pool, 32 requests, every layer per step
     w = synth.workload("decode_R32")

@@ -157,7 +157,7 @@ size_t unipin_masked_prefill_workspace_size(void);
  *                  sums its query heads' gradients); written in full (dq is accumulated
  *                  across key tiles with atomic adds, so its low bits depend on
  *                  their order)
- *   D              32 or 64 (UNIPIN_ERR_UNSUPPORTED otherwise)
+ *   D              32, 64 or 128 (UNIPIN_ERR_UNSUPPORTED otherwise)
  *   workspace      device scratch of at least
  *                  unipin_masked_prefill_bwd_workspace_size(total_tokens, H) bytes
  *                  (the per-row dO . O), 16-byte aligned; not shared by overlapping calls

@@ -47,10 +47,13 @@ constexpr int kBwRows = 128;   // keys per key tile and queries per query tile
 
 template <int D>
 struct BwCfg {
-    static_assert(D == 32 || D == 64, "backward: head dim 32 or 64");
-    static constexpr int kRowBytes = D * 2;                        // one TMA box row covers D
-    static constexpr uint32_t kLayout = D == 64 ? kLayoutSw128 : kLayoutSw64;
-    static constexpr int kTile = kBwRows * kRowBytes;               // 128 rows of K, V, Q or dO
+    static_assert(D == 32 || D == 64 || D == 128, "backward: head dim 32, 64 or 128");
+    static constexpr int kBoxElems = D >= 64 ? 64 : D;              // elements of a row in one TMA box
+    static constexpr int kBoxes = D / kBoxElems;                    // boxes across D (2 at D = 128)
+    static constexpr int kRowBytes = kBoxElems * 2;
+    static constexpr uint32_t kLayout = D >= 64 ? kLayoutSw128 : kLayoutSw64;
+    static constexpr int kBox = kBwRows * kRowBytes;                // 128 rows of one box
+    static constexpr int kTile = kBoxes * kBox;                     // 128 rows of K, V, Q or dO
     static constexpr int kOffK = 0;
     static constexpr int kOffV = kTile;
     static constexpr int kOffQ = 2 * kTile;                         // [2] query-tile buffers
@@ -64,8 +67,13 @@ struct BwCfg {
     static constexpr int kColDP = 128;     // dP^T (128), then dS^T as bf16 pairs (64)
     static constexpr int kColDV = 256;
     static constexpr int kColDK = 256 + D;
-    static constexpr int kColDQ = 256 + 2 * D;
-    static_assert(kColDQ + D <= 512, "TMEM budget");
+    // dQ of a query tile: its own D columns where they fit; at D = 128 two halves of
+    // 64 columns in the score columns that P^T and dS^T leave free (64-127, 192-255),
+    // so the next tile's S^T and dP^T wait until the softmax has read them out.
+    static constexpr bool kSplitDQ = 256 + 3 * D > 512;
+    static constexpr int kDQHalf = kSplitDQ ? D / 2 : D;
+    static constexpr int dq_col(int half) { return kSplitDQ ? (half == 0 ? 64 : 192) : 256 + 2 * D; }
+    static_assert(kSplitDQ ? (kColDK + D <= 512 && kDQHalf <= 64) : (256 + 3 * D <= 512), "TMEM budget");
     static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
 
@@ -222,7 +230,8 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     uint64_t* mma2_done = bars + 7;
     uint64_t* grp = bars + 8;
     uint64_t* bar_drain = bars + 9;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 10);
+    uint64_t* dq_free = bars + 10;     // dQ read out of TMEM (4 softmax warps; split dQ only)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     if (threadIdx.x == 0) {
@@ -236,6 +245,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         mbar_init(mma2_done, 1);
         mbar_init(grp, 4);
         mbar_init(bar_drain, 1);
+        mbar_init(dq_free, 4);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -258,8 +268,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             tma_prefetch_map(&tm_v);
             tma_prefetch_map(&tm_do);
             mbar_arrive_expect_tx(bar_kv, 2 * C::kTile);
-            tma_load_3d(sK, &tm_k, bar_kv, 0, h, tok0 + j0);
-            tma_load_3d(sV, &tm_v, bar_kv, 0, h, tok0 + j0);
+            for (int c = 0; c < C::kBoxes; ++c) {
+                tma_load_3d(sK + c * C::kBox, &tm_k, bar_kv, c * C::kBoxElems, h, tok0 + j0);
+                tma_load_3d(sV + c * C::kBox, &tm_v, bar_kv, c * C::kBoxElems, h, tok0 + j0);
+            }
         }
         bool ok = true;
         for (int qi = 0; ok && qi < nq; ++qi) {
@@ -272,8 +284,10 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                 const int row0 = tok0 + j0 + (qi % nqt) * kBwRows;
                 const int hq = h * p.G + qi / nqt;
                 mbar_arrive_expect_tx(bar_qdo + qb, 2 * C::kTile);
-                tma_load_3d(sQ + qb * C::kTile, &tm_q, bar_qdo + qb, 0, hq, row0);
-                tma_load_3d(sDO + qb * C::kTile, &tm_do, bar_qdo + qb, 0, hq, row0);
+                for (int c = 0; c < C::kBoxes; ++c) {
+                    tma_load_3d(sQ + qb * C::kTile + c * C::kBox, &tm_q, bar_qdo + qb, c * C::kBoxElems, hq, row0);
+                    tma_load_3d(sDO + qb * C::kTile + c * C::kBox, &tm_do, bar_qdo + qb, c * C::kBoxElems, hq, row0);
+                }
             }
         }
         if (leader) {
@@ -286,32 +300,39 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         // --------------------------------------------------------- MMA issuer
         constexpr uint32_t idesc_s = idesc_bf16_f32(kBwRows, kBwRows, false, false);
         constexpr uint32_t idesc_g = idesc_bf16_f32(kBwRows, D, true, false);    // A from TMEM, B MN-major
-        constexpr uint32_t idesc_q = idesc_bf16_f32(kBwRows, D, true, true);     // A (dS) and B (K) MN-major
+        constexpr uint32_t idesc_q = idesc_bf16_f32(kBwRows, C::kDQHalf, true, true);   // A (dS) and B (K) MN-major
         const uint64_t dK_kmaj = smem_desc(smem_u32(sK), 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dV_kmaj = smem_desc(smem_u32(sV), 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dQ_kmaj = smem_desc(smem_u32(sQ), 16, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dDO_kmaj = smem_desc(smem_u32(sDO), 16, 8 * C::kRowBytes, C::kLayout);
-        const uint64_t dQ_mn = smem_desc(smem_u32(sQ), C::kTile, 8 * C::kRowBytes, C::kLayout);
-        const uint64_t dDO_mn = smem_desc(smem_u32(sDO), C::kTile, 8 * C::kRowBytes, C::kLayout);
-        const uint64_t dK_mn = smem_desc(smem_u32(sK), C::kTile, 8 * C::kRowBytes, C::kLayout);
+        // MN-major operands span D in boxes kBox bytes apart
+        const uint64_t dQ_mn = smem_desc(smem_u32(sQ), C::kBox, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dDO_mn = smem_desc(smem_u32(sDO), C::kBox, 8 * C::kRowBytes, C::kLayout);
+        const uint64_t dK_mn = smem_desc(smem_u32(sK), C::kBox, 8 * C::kRowBytes, C::kLayout);
         const uint64_t dDS_mn = smem_desc(smem_u32(sDS), 16384, 1024, kLayoutSw128);
         bool ok = __all_sync(0xffffffffu, mbar_wait(bar_kv, 0, ctl));
         for (int qi = 0; ok && qi < nq; ++qi) {
             const int qb = qi & 1;
             ok = __all_sync(0xffffffffu, mbar_wait(bar_qdo + qb, (qi >> 1) & 1, ctl));
             if (!ok) break;
+            // split dQ: the last tile's dQ halves sit in the score columns until read out
+            if (C::kSplitDQ && qi > 0) {
+                ok = __all_sync(0xffffffffu, mbar_wait(dq_free, (qi - 1) & 1, ctl));
+                if (!ok) break;
+            }
             tc_fence_after_sync();
             const uint64_t qoff = (uint64_t)((qb * C::kTile) >> 4);
             if (leader) {
-                // S^T = K Q^T and dP^T = V dO^T: K-steps of 16 elements (32 bytes of a row)
+                // S^T = K Q^T and dP^T = V dO^T: K-steps of 16 elements (32 bytes of a box row)
+                constexpr int kStepsPerBox = C::kBoxElems / 16;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = (uint64_t)((kk * 32) >> 4);
+                    const uint64_t off = (uint64_t)(((kk / kStepsPerBox) * C::kBox + (kk % kStepsPerBox) * 32) >> 4);
                     umma_bf16_ss(tmem + C::kColS, dK_kmaj + off, dQ_kmaj + qoff + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t off = (uint64_t)((kk * 32) >> 4);
+                    const uint64_t off = (uint64_t)(((kk / kStepsPerBox) * C::kBox + (kk % kStepsPerBox) * 32) >> 4);
                     umma_bf16_ss(tmem + C::kColDP, dV_kmaj + off, dDO_kmaj + qoff + off, idesc_s, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(s_ready);
@@ -328,11 +349,15 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                     umma_bf16_ts(tmem + C::kColDV, tmem + C::kColS + kk * 8, dDO_mn + off, idesc_g, acc);
                     umma_bf16_ts(tmem + C::kColDK, tmem + C::kColDP + kk * 8, dQ_mn + off, idesc_g, acc);
                 }
-                // dQ_tile = dS K: K-steps of 16 keys (2 KB of dS^T, 16 rows of K)
+                // dQ_tile = dS K: K-steps of 16 keys (2 KB of dS^T, 16 rows of K); at D = 128 in two
+                // halves of 64 head-dim columns (one K box each)
 #pragma unroll
-                for (int kk = 0; kk < kBwRows / 16; ++kk)
-                    umma_bf16_ss(tmem + C::kColDQ, dDS_mn + (uint64_t)((kk * 2048) >> 4),
-                                 dK_mn + (uint64_t)((kk * 16 * C::kRowBytes) >> 4), idesc_q, kk > 0 ? 1u : 0u);
+                for (int half = 0; half < D / C::kDQHalf; ++half)
+#pragma unroll
+                    for (int kk = 0; kk < kBwRows / 16; ++kk)
+                        umma_bf16_ss(tmem + C::dq_col(half), dDS_mn + (uint64_t)((kk * 2048) >> 4),
+                                     dK_mn + (uint64_t)((half * C::kBox + kk * 16 * C::kRowBytes) >> 4), idesc_q,
+                                     kk > 0 ? 1u : 0u);
                 umma_commit(mma2_done);
                 umma_commit(qdo_empty + qb);
             }
@@ -408,41 +433,53 @@ __global__ void __launch_bounds__(kBwThreads, 1)
             ok = __all_sync(0xffffffffu, mbar_wait(mma2_done, qi & 1, ctl));
             if (!ok) break;
             tc_fence_after_sync();
-            uint32_t dqr[D];
-            if constexpr (D == 64) tmem_ld64(lane_base + C::kColDQ, dqr);
-            else tmem_ld32(lane_base + C::kColDQ, dqr);
-            tc_fence_before_sync();
             const int row = qrow0 + t;
-            if (row < len) {
-                float* dst = p.dq + ((size_t)(tok0 + row) * p.H + hq) * D;
 #pragma unroll
-                for (int e = 0; e < D; e += 4)
-                    red_add_v4(dst + e, p.scale * __uint_as_float(dqr[e]), p.scale * __uint_as_float(dqr[e + 1]),
-                               p.scale * __uint_as_float(dqr[e + 2]), p.scale * __uint_as_float(dqr[e + 3]));
+            for (int half = 0; half < D / C::kDQHalf; ++half) {
+                uint32_t dqr[C::kDQHalf];
+                if constexpr (C::kDQHalf == 64) tmem_ld64(lane_base + C::dq_col(half), dqr);
+                else tmem_ld32(lane_base + C::dq_col(half), dqr);
+                if (row < len) {
+                    float* dst = p.dq + ((size_t)(tok0 + row) * p.H + hq) * D + half * C::kDQHalf;
+#pragma unroll
+                    for (int e = 0; e < C::kDQHalf; e += 4)
+                        red_add_v4(dst + e, p.scale * __uint_as_float(dqr[e]), p.scale * __uint_as_float(dqr[e + 1]),
+                                   p.scale * __uint_as_float(dqr[e + 2]), p.scale * __uint_as_float(dqr[e + 3]));
+                }
+            }
+            tc_fence_before_sync();
+            if (C::kSplitDQ) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(dq_free);
             }
         }
         if (ok) {
             // the tile's dK (scaled) and dV rows; all of this block's MMAs have finished.  The
             // TMEM loads are warp-collective: every lane loads, keys past the history store nothing.
-            uint32_t g[D];
-            if constexpr (D == 64) tmem_ld64(lane_base + C::kColDK, g);
-            else tmem_ld32(lane_base + C::kColDK, g);
-            if (key_ok) {
-                float* dkd = p.dk + ((size_t)(tok0 + key) * hkv + h) * D;
+            constexpr int kChunk = D >= 64 ? 64 : D;
 #pragma unroll
-                for (int e = 0; e < D; e += 4)
-                    *reinterpret_cast<float4*>(dkd + e) =
-                        make_float4(p.scale * __uint_as_float(g[e]), p.scale * __uint_as_float(g[e + 1]),
-                                    p.scale * __uint_as_float(g[e + 2]), p.scale * __uint_as_float(g[e + 3]));
-            }
-            if constexpr (D == 64) tmem_ld64(lane_base + C::kColDV, g);
-            else tmem_ld32(lane_base + C::kColDV, g);
-            if (key_ok) {
-                float* dvd = p.dv + ((size_t)(tok0 + key) * hkv + h) * D;
+            for (int c0 = 0; c0 < D; c0 += kChunk) {
+                uint32_t g[kChunk];
+                if constexpr (kChunk == 64) tmem_ld64(lane_base + C::kColDK + c0, g);
+                else tmem_ld32(lane_base + C::kColDK + c0, g);
+                if (key_ok) {
+                    float* dkd = p.dk + ((size_t)(tok0 + key) * hkv + h) * D + c0;
 #pragma unroll
-                for (int e = 0; e < D; e += 4)
-                    *reinterpret_cast<float4*>(dvd + e) = make_float4(__uint_as_float(g[e]), __uint_as_float(g[e + 1]),
-                                                                      __uint_as_float(g[e + 2]), __uint_as_float(g[e + 3]));
+                    for (int e = 0; e < kChunk; e += 4)
+                        *reinterpret_cast<float4*>(dkd + e) =
+                            make_float4(p.scale * __uint_as_float(g[e]), p.scale * __uint_as_float(g[e + 1]),
+                                        p.scale * __uint_as_float(g[e + 2]), p.scale * __uint_as_float(g[e + 3]));
+                }
+                if constexpr (kChunk == 64) tmem_ld64(lane_base + C::kColDV + c0, g);
+                else tmem_ld32(lane_base + C::kColDV + c0, g);
+                if (key_ok) {
+                    float* dvd = p.dv + ((size_t)(tok0 + key) * hkv + h) * D + c0;
+#pragma unroll
+                    for (int e = 0; e < kChunk; e += 4)
+                        *reinterpret_cast<float4*>(dvd + e) =
+                            make_float4(__uint_as_float(g[e]), __uint_as_float(g[e + 1]), __uint_as_float(g[e + 2]),
+                                        __uint_as_float(g[e + 3]));
+                }
             }
         }
     }

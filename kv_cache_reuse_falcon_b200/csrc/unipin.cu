@@ -139,7 +139,9 @@ int ensure_device()
         (cudaFuncSetAttribute(bwd_kv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               BwCfg<32>::kSmemBytes) != cudaSuccess ||
          cudaFuncSetAttribute(bwd_kv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              BwCfg<64>::kSmemBytes) != cudaSuccess))
+                              BwCfg<64>::kSmemBytes) != cudaSuccess ||
+         cudaFuncSetAttribute(bwd_kv_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              BwCfg<128>::kSmemBytes) != cudaSuccess))
         rc = UNIPIN_ERR_CUDA;
     if (rc != UNIPIN_OK) return rc;
     g_device_ready[dev] = true;
@@ -826,7 +828,7 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
 {
     if (B < 0 || H < 1 || H_kv < 1 || H % H_kv != 0 || max_seqlen < 0 || total_tokens < 0)
         return UNIPIN_ERR_INVALID_ARG;
-    if (D != 32 && D != 64) return UNIPIN_ERR_UNSUPPORTED;
+    if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
     if (!(scale > 0.f) || !std::isfinite(scale)) return UNIPIN_ERR_INVALID_ARG;
     if (B == 0 || total_tokens == 0 || max_seqlen == 0) return UNIPIN_OK;
     if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !cu_seqlens || !past_lens || !workspace)
@@ -868,8 +870,10 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
     const unsigned prep_blocks = (unsigned)((rows + 7) / 8);
     if (D == 32)
         bwd_prep_kernel<32><<<prep_blocks, 256, 0, s>>>(p);
-    else
+    else if (D == 64)
         bwd_prep_kernel<64><<<prep_blocks, 256, 0, s>>>(p);
+    else
+        bwd_prep_kernel<128><<<prep_blocks, 256, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return UNIPIN_ERR_CUDA;
 
     CUtensorMap tq, tk, tv, tdo;
@@ -879,8 +883,10 @@ int unipin_masked_prefill_bwd(const void* q, const void* k, const void* v, const
     if ((rc = make_token_map(&tdo, dout, total_tokens, H, D, kBwRows)) != UNIPIN_OK) return rc;
     if (D == 32)
         bwd_kv_kernel<32><<<(unsigned)items, kBwThreads, BwCfg<32>::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
-    else
+    else if (D == 64)
         bwd_kv_kernel<64><<<(unsigned)items, kBwThreads, BwCfg<64>::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
+    else
+        bwd_kv_kernel<128><<<(unsigned)items, kBwThreads, BwCfg<128>::kSmemBytes, s>>>(tq, tk, tv, tdo, p);
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 

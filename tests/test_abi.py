@@ -61,7 +61,7 @@ def test_host_validation_needs_no_device(lib):
     b.argtypes = [P, P, P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, ctypes.c_float, P, SZ, P, P]
     b.restype = I
     nul = [None] * 11
-    assert b(*nul, 1, 1, 1, 128, 16, 16, 0.1, None, 0, None, None) == -2    # D = 128: not supported
+    assert b(*nul, 1, 1, 1, 96, 16, 16, 0.1, None, 0, None, None) == -2     # D = 96: not supported
     assert b(*nul, 1, 1, 1, 64, 16, 16, 0.0, None, 0, None, None) == -1     # scale must be positive
     assert b(*nul, 1, 1, 1, 64, 16, 16, 0.1, None, 0, None, None) == -1     # missing tensors
     assert b(*nul, 0, 1, 1, 64, 16, 0, 0.1, None, 0, None, None) == 0

@@ -63,6 +63,8 @@ BWD_CASES = [
     ([1, 0, 129, 5], [0, 7, 3, 300], 1, 64),     # n=1, n=0, k=0
     ([128, 256], [128, 1], 2, 64),               # tile-aligned history
     ([90, 513], [40, 33], 3, 32),                # D = 32, several tiles
+    ([200, 37, 300], [77, 5, 260], 2, 128),      # D = 128: dQ in two halves over the score columns
+    ([1, 0, 129, 256], [0, 7, 3, 300], 1, 128),  # n=1, n=0, k=0, tile-aligned, D = 128
 ]
 
 

@@ -105,7 +105,7 @@ def test_gqa_rank_decode(ub, case, mode):
     parity(out.cpu().numpy(), ref, "gqa decode case %d %s" % (case, mode))
 
 
-@pytest.mark.parametrize("H,Hkv,D", [(4, 2, 64), (8, 1, 32)])
+@pytest.mark.parametrize("H,Hkv,D", [(4, 2, 64), (8, 1, 32), (4, 2, 128)])
 def test_gqa_backward(ub, H, Hkv, D):
     past, cand = [200, 37, 300], [77, 5, 130]
     cu, pl, q, k, v, rng = gqa_prefill(7200 + H, past, cand, H, Hkv, D)
