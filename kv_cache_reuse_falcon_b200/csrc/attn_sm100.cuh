@@ -94,6 +94,10 @@ struct AttnCfg {
     static constexpr int kTileKV = kN * D * 2;                  // one K or V tile
     static constexpr int kSlotBytes = 2 * kTileKV;              // a ring slot: K and V of one key tile
     static constexpr int kStages = (128 * 1024) / kSlotBytes;   // ring slots
+    // Pairs in every four of P's exponentials taken by the FMA-pipe polynomial (the rest
+    // by the MUFU ex2).  One in four at every D: two or three in four measured slower at
+    // D = 64 (the D = 64 prefill is not bound by the MUFU) and at D = 128.
+    static constexpr int kPolyOf4 = 1;
     static constexpr int kOffQ = 0;                             // Q_A, Q_B
     static constexpr int kOffRing = 2 * kTileQ;
     static constexpr int kOffBar = kOffRing + kStages * kSlotBytes;
@@ -804,8 +808,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m = m_new;
                 }
                 const float m_use = (m == -INFINITY) ? 0.f : m;
-                // P = 2^(s * scale * log2e - m): packed fp32 pairs; one pair in four
-                // takes the polynomial exp2 on the FMA pipe, the rest the MUFU ex2,
+                // P = 2^(s * scale * log2e - m): packed fp32 pairs; kPolyOf4 pairs in
+                // four take the polynomial exp2 on the FMA pipe, the rest the MUFU ex2,
                 // so the two pipes share the load.  P is written in pieces of 64 keys
                 // (32 columns of bf16 pairs).
                 const uint64_t sc2 = f2_pack(sl2, sl2);
@@ -819,7 +823,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int e = half * 64 + 2 * c;
                         const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[e]), __uint_as_float(s[e + 1])), sc2, nm2);
                         float p0, p1;
-                        if ((c & 3) == 3) {
+                        if ((c & 3) >= 4 - C::kPolyOf4) {
                             exp2_poly2(x2, p0, p1);
                         } else {
                             float x0, x1;
