@@ -23,13 +23,17 @@
 // reduce-scatter of the column sums.  O accumulates in TMEM with lane =
 // candidate, so the epilogue thread of candidate c reads its own row.
 //
-// Work item = (request, head, key split).  The key range of a request is cut
-// into `nsplit` runs of whole 128-key tiles so that every SM has several
-// items; each item leaves an unnormalised partial (O, m, l) per candidate in
-// the caller's workspace, and the last item of a (request, head) to finish -
-// found with a per-pair arrival counter - merges the partials with the
-// candidate's own key (self term) and writes the output.  With one split the
-// item writes the output directly.
+// Work: the 128-key tiles of all (request, key/value head) pairs, pair-major
+// (tpp tiles per pair, from the pool's capacity), are cut into one contiguous
+// range per block, so every block gets the same number of tiles (handing out
+// more, smaller ranges from a counter measured slower: each extra piece costs
+// an epilogue).  A block's range falls into one or more pieces (pair, tile
+// run); each piece is an item.
+// A pair covered by one piece writes its output directly; otherwise each piece
+// leaves an unnormalised partial (O, m, l) per candidate in the caller's
+// workspace, and the last piece of the pair to finish - found with a per-pair
+// arrival counter - merges the partials with the candidate's own key (self
+// term) and writes the output.
 //
 // Warp roles (256 threads; two blocks per SM where shared memory and TMEM
 // allow):
@@ -146,11 +150,13 @@ struct SkParams {
     int total_rows;                // T
     int out_fp32;
     int layer, S, n_cap;
-    int nsplit, tiles_per_split;
+    int nsplit;                    // partial slots per pair: the most pieces any pair has
+    int tpp;                       // key tiles per pair
+    long long total_tiles;         // pairs * tpp
+    int nranges;                   // contiguous tile ranges, one per block
     float sl2;                     // scale * log2(e)
     int* status;
     unsigned long long wait_limit_ns;
-    unsigned long long* sched;     // zeroed item counter or null (static striding)
     int prefetch_tiles;            // key tiles the producer asks L2 for ahead of its ring loads
     unsigned poll_ns;              // back-off of the polling producer and MMA warps when nothing is ready
 };
@@ -161,19 +167,46 @@ struct SkParams {
 struct SkWork {
     bool rows_ok;   // the request's candidate rows are addressable (cu in range, k * G <= N)
     bool valid;     // rows_ok and slot / history length in range
-    int r, h, split, pair;   // h: the key/value head
+    int r, h, split, pair;   // h: the key/value head; split: the piece's index among its pair's
+    int npieces;             // pieces that cover the pair
     int tok0, kc, npast, slot;
     int ncol;                // valid candidate columns, kc * G
     int nt_all;     // key tiles covering [0, npast)
     int t_begin, nt;
 };
 
+// Range b is tiles [b T / B, (b + 1) T / B) (B ranges); the range holding tile x.
+__device__ __forceinline__ long long sk_range_start(const SkParams& p, long long b)
+{
+    return b * p.total_tiles / p.nranges;
+}
+__device__ __forceinline__ long long sk_block_of(const SkParams& p, long long x)
+{
+    return ((x + 1) * p.nranges - 1) / p.total_tiles;
+}
+
+// Item g = (range g >> 20, its piece g & 0xFFFFF).  Whether the piece exists.
+__device__ __forceinline__ bool sk_piece_exists(const SkParams& p, long long g)
+{
+    const long long b = g >> 20;
+    const long long pair = sk_range_start(p, b) / p.tpp + (g & 0xFFFFF);
+    return pair * p.tpp < sk_range_start(p, b + 1);
+}
+
 template <int N>
 __device__ __forceinline__ SkWork sk_make_work(const SkParams& p, long long g)
 {
     SkWork w;
-    w.pair = (int)(g / p.nsplit);
-    w.split = (int)(g - (long long)w.pair * p.nsplit);
+    const long long b = g >> 20;
+    const long long s0 = sk_range_start(p, b), s1 = sk_range_start(p, b + 1);
+    const long long pair = s0 / p.tpp + (g & 0xFFFFF);
+    const long long p0 = pair * p.tpp;
+    const long long lo = s0 > p0 ? s0 : p0;
+    const long long hi = s1 < p0 + p.tpp ? s1 : p0 + p.tpp;
+    const long long first = sk_block_of(p, p0), last = sk_block_of(p, p0 + p.tpp - 1);
+    w.pair = (int)pair;
+    w.split = (int)(b - first);
+    w.npieces = (int)(last - first + 1);
     const int hkv = p.H / p.G;
     w.r = w.pair / hkv;
     w.h = w.pair - w.r * hkv;
@@ -185,9 +218,10 @@ __device__ __forceinline__ SkWork sk_make_work(const SkParams& p, long long g)
     w.rows_ok = w.tok0 >= 0 && w.kc >= 0 && w.ncol <= N && (long long)w.tok0 + w.kc <= (long long)p.total_rows;
     w.valid = w.rows_ok && w.slot >= 0 && w.slot < p.S && w.npast >= 0 && w.npast <= p.n_cap;
     w.nt_all = w.valid ? (w.npast + kSkKeys - 1) / kSkKeys : 0;
-    w.t_begin = min(w.split * p.tiles_per_split, w.nt_all);
-    const int t_end = min(w.t_begin + p.tiles_per_split, w.nt_all);
-    w.nt = (w.valid && w.kc > 0) ? t_end - w.t_begin : 0;
+    const int t0 = (int)(lo - p0), t1 = (int)(hi - p0);
+    w.t_begin = min(t0, w.nt_all);
+    const int t_end = min(t1, w.nt_all);
+    w.nt = (w.valid && w.kc > 0) ? max(t_end - w.t_begin, 0) : 0;
     return w;
 }
 
@@ -371,7 +405,6 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     const uint32_t tmem = *tmem_slot;
 
     WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
-    const long long total_items = (long long)p.R * (p.H / p.G) * p.nsplit;
     int n_items = 0;
     // Consumers: the next item (warp-uniform)
     auto pop_item = [&](bool& ok, long long& g) -> bool {
@@ -408,10 +441,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         int nq = 0;
         bool k_has = false, q_done = false, claim_done = false, ok = true;
         int q_h = 0, q_tok = 0;
-        // The first item of a block is its index; later ones come from the shared
-        // counter (offset by the grid), claimed one item ahead so that the
-        // atomic's latency overlaps this item's loads.
-        long long g_next = blockIdx.x;
+        long long g_next = (long long)blockIdx.x << 20;   // the block's pieces, in order
         uint64_t t_prog = global_timer_ns();
         for (uint32_t spin = 1;; ++spin) {
             bool prog = false;
@@ -420,15 +450,9 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 const int si = n_items % kSkItemSlots;
                 if (n_items < kSkItemSlots ||
                     __all_sync(0xffffffffu, mbar_test_wait(item_empty + si, ((n_items / kSkItemSlots) - 1) & 1))) {
-                    const long long g = __shfl_sync(0xffffffffu, g_next, 0);
-                    const bool found = g < total_items;
-                    if (found) {
-                        if (p.sched) {
-                            if (leader) g_next = (long long)gridDim.x + (long long)atomicAdd(p.sched, 1ull);
-                        } else {
-                            g_next = g + gridDim.x;
-                        }
-                    }
+                    const long long g = g_next;
+                    const bool found = sk_piece_exists(p, g);
+                    ++g_next;
                     if (leader) {
                         item_ring[si] = found ? g : -1;
                         mbar_arrive(item_full + si);   // release: the consumers see the ring entry
@@ -898,7 +922,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             }
             // final coefficients (one split): out = (a O + b v_self) / (a l + b)
             float ca = 0.f, cb = 0.f;
-            if (p.nsplit == 1 && mine) {
+            if (w.npieces == 1 && mine) {
                 const float mf = fmaxf(m_c, ss_own);
                 const float a = (m_c == -INFINITY) ? 0.f : ex2_approx(m_c - mf);
                 const float b = ex2_approx(ss_own - mf);
@@ -916,7 +940,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 #pragma unroll
                     for (int d = 0; d < 32; ++d) o[d] = 0u;
                 }
-                if (p.nsplit == 1) {
+                if (w.npieces == 1) {
                     // a rejected request (ca = cb = 0) gets zero rows
                     if (t < w.ncol) {
                         const uint4* v4 = reinterpret_cast<const uint4*>(p.v_self + kvrow * D + c0);
@@ -949,7 +973,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                 if (lane == 0) mbar_arrive(o_free + ob);
                 ++nb;
             }
-            if (p.nsplit == 1) continue;
+            if (w.npieces == 1) continue;
             // publish the partial; the last split of this (request, head) to arrive merges
             if (t < w.ncol) {
                 float* ml = p.part_ml + ((size_t)w.split * p.total_rows * p.H + qrow) * 2;
@@ -960,7 +984,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
             if (t == 0) {
                 const unsigned prev = atomicAdd(p.pair_cnt + w.pair, 1u);
-                *last_flag = prev == (unsigned)(p.nsplit - 1);
+                *last_flag = prev == (unsigned)(w.npieces - 1);
             }
             if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
             if (*last_flag) {
@@ -971,7 +995,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 #pragma unroll
                     for (int s = 0; s < kSkMaxSplit; ++s) {
                         float2 ml = make_float2(-INFINITY, 0.f);
-                        if (s < p.nsplit)
+                        if (s < w.npieces)
                             ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + ((size_t)s * p.total_rows * p.H + qrow) * 2));
                         ms[s] = ml.x;
                         ls[s] = ml.y;
@@ -985,11 +1009,11 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                     for (int s = 0; s < kSkMaxSplit; ++s) {
                         const float a = (ms[s] == -INFINITY || !(ls[s] > 0.f)) ? 0.f : ex2_approx(ms[s] - mf);
                         den = fmaf(a, ls[s], den);
-                        if (s < p.nsplit) wts[s * N + t] = a;
+                        if (s < w.npieces) wts[s * N + t] = a;
                     }
                     // a rejected request (no own score: every term -inf) gets zero weights
                     const float inv = w.valid ? 1.f / den : 0.f;
-                    for (int s = 0; s < p.nsplit; ++s) wts[s * N + t] *= inv;
+                    for (int s = 0; s < w.npieces; ++s) wts[s * N + t] *= inv;
                     coef_b[t] = w.valid ? b * inv : 0.f;
                 }
                 if (!(ok = warp_group_sync(egrp, negrp, ctl, lane))) break;
@@ -1023,7 +1047,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                     }
 #pragma unroll
                     for (int s = 0; s < kSkMaxSplit; ++s) {
-                        if (s < p.nsplit) {
+                        if (s < w.npieces) {
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 if (cc[u] >= 0) {

@@ -324,8 +324,8 @@ int sk_ctas_per_sm(int D, int N)
     }
 }
 
-// Work items a resident block should get on average (load balance against
-// per-item overhead); UNIPIN_DECODE_ITEMS_PER_BLOCK overrides it.
+// Tile ranges (blocks) per resident block slot (1: one wave of blocks);
+// UNIPIN_DECODE_ITEMS_PER_BLOCK overrides it.
 int sk_items_per_block()
 {
     static int v = [] {
@@ -360,30 +360,43 @@ unsigned sk_poll_ns()
 }
 
 struct SkPlan {
-    int N, nsplit, tiles_per_split, blocks_per_sm;
+    int N, blocks_per_sm;
+    int tpp;                // key tiles per (request, key/value head) pair
+    long long total_tiles;  // pairs * tpp
+    int nranges;            // contiguous tile ranges, one per block
+    int nsplit;             // the most pieces (ranges) any pair is cut into
 };
 
-// Key splits per (request, head): cut the pool sweep into runs of whole
-// 128-key tiles so that the grid gets about sk_items_per_block() items per
-// resident block, at most kSkMaxSplit runs.
-// The candidate columns of an item are (candidate, query head of the group):
-// max_k * G of them; H_kv = H / G key/value heads make R * H_kv (request, head) pairs.
-SkPlan sk_plan(int R, int H_kv, int G, int D, int max_k, int n_cap, int sms)
+// The tiles of all pairs, pair-major, cut into `nranges` equal contiguous
+// ranges: about sk_items_per_block() ranges per resident block, fewer when a
+// pair would be cut into more than kSkMaxSplit pieces (a range then spans at
+// least tpp / (kSkMaxSplit - 1) tiles).  With split = false one range per
+// pair (no partials).  The candidate columns of a pair are (candidate, query
+// head of the group): max_k * G of them.
+SkPlan sk_plan(int R, int H_kv, int G, int D, int max_k, int n_cap, int sms, bool split = true)
 {
     SkPlan pl;
     pl.N = sk_pad_n(max_k * G);
     pl.blocks_per_sm = sk_ctas_per_sm(D, pl.N);
-    const long long tiles = (n_cap + kSkKeys - 1) / kSkKeys;
+    pl.tpp = (n_cap + kSkKeys - 1) / kSkKeys;
     const long long pairs = (long long)R * H_kv;
-    const long long target = (long long)sk_items_per_block() * sms * pl.blocks_per_sm;
-    long long ns = (target + pairs - 1) / pairs;   // splits per (request, head) for the target item count
-    if (ns > tiles) ns = tiles;
-    if (ns > kSkMaxSplit) ns = kSkMaxSplit;
-    if (ns < 1) ns = 1;
-    long long per = (tiles + ns - 1) / ns;         // equal runs of tiles
-    ns = (tiles + per - 1) / per;
-    pl.nsplit = (int)(ns < 1 ? 1 : ns);
-    pl.tiles_per_split = (int)(pl.nsplit == 1 ? (tiles < 1 ? 1 : tiles) : per);
+    pl.total_tiles = pairs * pl.tpp;
+    long long B = pairs;
+    if (split) {
+        B = (long long)sk_items_per_block() * sms * pl.blocks_per_sm;
+        const long long min_tiles = (pl.tpp + kSkMaxSplit - 2) / (kSkMaxSplit - 1);
+        if (B > pl.total_tiles / min_tiles) B = pl.total_tiles / min_tiles;
+        if (B < 1) B = 1;
+    }
+    pl.nranges = (int)B;
+    // the most pieces of a pair: blocks holding its first and last tile
+    int most = 1;
+    for (long long q = 0; q < pairs; ++q) {
+        const long long x0 = q * pl.tpp, x1 = x0 + pl.tpp - 1;
+        const long long b0 = ((x0 + 1) * B - 1) / pl.total_tiles, b1 = ((x1 + 1) * B - 1) / pl.total_tiles;
+        if (b1 - b0 + 1 > most) most = (int)(b1 - b0 + 1);
+    }
+    pl.nsplit = most;
     return pl;
 }
 
@@ -424,16 +437,10 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
 {
     const int G = H / pool->H;
     SkPlan pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms());
-    if (pl.nsplit > 1 && (!workspace || workspace_bytes < sk_workspace_bytes(pl, R, H, D, total_cand))) {
-        pl.nsplit = 1;
-        pl.tiles_per_split = (pool->n_cap + kSkKeys - 1) / kSkKeys;
-    }
-    unsigned long long* sched = nullptr;
-    if (workspace && workspace_bytes >= kSchedBytes) {
-        sched = static_cast<unsigned long long*>(workspace);
-        const size_t zero = pl.nsplit > 1 ? kSchedBytes + sk_counter_bytes(R, H) : sizeof(unsigned long long);
-        if (cudaMemsetAsync(workspace, 0, zero, s) != cudaSuccess) return UNIPIN_ERR_CUDA;
-    }
+    if (pl.nsplit > 1 && (!workspace || workspace_bytes < sk_workspace_bytes(pl, R, H, D, total_cand)))
+        pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms(), false);
+    if (pl.nsplit > 1 && cudaMemsetAsync(workspace, 0, kSchedBytes + sk_counter_bytes(R, H), s) != cudaSuccess)
+        return UNIPIN_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     int rc;
     // the N candidate columns: N / G tokens x the G query heads of one key/value head
@@ -458,11 +465,12 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
     p.S = pool->S;
     p.n_cap = pool->n_cap;
     p.nsplit = pl.nsplit;
-    p.tiles_per_split = pl.tiles_per_split;
+    p.tpp = pl.tpp;
+    p.total_tiles = pl.total_tiles;
+    p.nranges = pl.nranges;
     p.sl2 = scale * kLog2e;
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
-    p.sched = sched;
     p.prefetch_tiles = sk_prefetch_tiles();
     p.poll_ns = sk_poll_ns();
     if (pl.nsplit > 1) {
@@ -471,7 +479,7 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
         p.part_o = reinterpret_cast<float*>(ws + kSchedBytes + sk_counter_bytes(R, H));
         p.part_ml = p.part_o + (size_t)pl.nsplit * total_cand * H * D;
     }
-    const unsigned grid = persistent_blocks((long long)R * pool->H * pl.nsplit, pl.blocks_per_sm);
+    const unsigned grid = (unsigned)pl.nranges;
     return D == 64 ? launch_sk_d<64>(pl.N, grid, tq, tk, tv, p, s) : launch_sk_d<128>(pl.N, grid, tq, tk, tv, p, s);
 }
 
