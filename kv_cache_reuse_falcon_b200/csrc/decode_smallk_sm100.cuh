@@ -157,7 +157,6 @@ struct SkParams {
     float sl2;                     // scale * log2(e)
     int* status;
     unsigned long long wait_limit_ns;
-    int prefetch_tiles;            // key tiles the producer asks L2 for ahead of its ring loads
     unsigned poll_ns;              // back-off of the polling producer and MMA warps when nothing is ready
 };
 

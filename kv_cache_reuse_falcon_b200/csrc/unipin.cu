@@ -336,18 +336,6 @@ int sk_items_per_block()
     return v;
 }
 
-// Key tiles the small-k producer prefetches into L2 ahead of its ring loads
-// (off by default: it measured slower); UNIPIN_DECODE_PREFETCH_TILES sets it.
-int sk_prefetch_tiles()
-{
-    static int v = [] {
-        const char* s = std::getenv("UNIPIN_DECODE_PREFETCH_TILES");
-        int n = s ? std::atoi(s) : 0;
-        return n > 0 ? (n > 64 ? 64 : n) : 0;
-    }();
-    return v;
-}
-
 // Back-off (ns) of the small-k kernel's polling warps; UNIPIN_DECODE_POLL_NS overrides it.
 unsigned sk_poll_ns()
 {
@@ -471,7 +459,6 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
     p.sl2 = scale * kLog2e;
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
-    p.prefetch_tiles = sk_prefetch_tiles();
     p.poll_ns = sk_poll_ns();
     if (pl.nsplit > 1) {
         char* ws = static_cast<char*>(workspace);
