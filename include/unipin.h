@@ -252,8 +252,9 @@ size_t unipin_rank_decode_pool_workspace_size(const unipin_kvpool* pool, int R, 
  * bytes (32 MiB) that the library reserves on every device it is loaded on
  * and keeps until the process exits.
  *   - If unipin_rank_decode_workspace_size(R, H, pool->H, D, max_k,
- *     total_cand, pool->n_cap) exceeds that size, nothing is launched and
- *     UNIPIN_ERR_OUT_OF_RANGE is returned.
+ *     total_cand, pool->n_cap) exceeds that size, the pool sweep is not split
+ *     (as unipin_rank_decode_attn does with a small workspace): the same
+ *     result, computed more slowly.
  *   - An UNIPIN_POOL_E4M3 pool is not taken (UNIPIN_ERR_UNSUPPORTED): its
  *     dequantized rows do not fit a fixed array.
  *   - The first call on a device looks up the array's device address; make

@@ -60,15 +60,31 @@ def test_noalloc_decode_matches_regular_decode_twice_in_a_row(ub, shape):
         parity(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "no-alloc decode")
 
 
-def test_noalloc_decode_rejects_requests_beyond_its_array(ub):
-    """A shape whose split-n scratch exceeds the fixed array returns OUT_OF_RANGE and launches nothing."""
+def test_noalloc_decode_runs_unsplit_beyond_its_array(ub):
+    """A shape whose split-n scratch exceeds the fixed array runs without the split: the regular
+    decode's result (which splits, with its own workspace) within fp32 rounding."""
     limit = ub.rank_decode_noalloc_scratch_bytes()
     H, D, n_cap = 4, 128, 4096
     R, k = 37, 256          # 148 (request, head) units: under two waves of blocks, so the sweep splits
-    need = ub.rank_decode_workspace_size(R, H, D, k, R * k, n_cap)
-    assert need > limit
-    P, I = ctypes.c_void_p, ctypes.c_int
-    pool = ub.KVPool(16, 16, 1, 1, H, n_cap, D)      # never dereferenced: the call returns first
-    rc = ub.LIB.unipin_rank_decode_attn_noalloc(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), R, H, D,
-                                                k, R * k, 0.1, ctypes.byref(pool), 0, None, None)
-    assert rc == -4
+    assert ub.rank_decode_workspace_size(R, H, D, k, R * k, n_cap) > limit
+    past, cand = [1000 + 61 * r for r in range(R)], [k] * R
+    layer, S = 0, 40
+    d, dd, pk, pv = _setup(7100, past, cand, H, D, S, n_cap, layer)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ref = ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, layer, dd.max_k,
+                              out_fp32=True, dev_status=status)
+    out = torch.full_like(ref, float("nan"))
+    ub.rank_decode_attn_noalloc(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, layer, dd.max_k,
+                                out, out_fp32=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    parity(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "no-alloc decode, unsplit")
+
+
+def test_noalloc_decode_refuses_an_e4m3_pool(ub):
+    """Its dequantized rows would not fit a fixed array: UNSUPPORTED before any launch."""
+    P = ctypes.c_void_p
+    pool = ub.KVPool(16, 16, 1, 1, 4, 512, 64, ub.POOL_E4M3, 1.0, 1.0)   # never dereferenced
+    rc = ub.LIB.unipin_rank_decode_attn_noalloc(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), 3, 4, 64,
+                                                16, 48, 0.1, ctypes.byref(pool), 0, None, None)
+    assert rc == -2
