@@ -131,6 +131,54 @@ def test_rank_decode_from_pool_workload(ub):
         parity(ok_.cpu().numpy(), refk, "decode R32 k%d" % kk)
 
 
+def test_rank_decode_from_e4m3_pool_workload(ub):
+    """The decode workload over an E4M3 pool [1, 256, 8, 2048, 64] written by the pool-write kernel
+    (scales 1/16): pool bytes bit-exact against the oracle's quantization, and the decode at k = 16
+    (the small-k kernel) and k = 1000 (the engine) against the oracle's E4M3 decode."""
+    w = synth.workload("decode_R32")
+    rng = np.random.Generator(np.random.PCG64(w.seed + 7))
+    past = np.full(w.B, w.n, np.int32)
+    scales = (0.0625, 0.0625)
+    # the history written by the pool-write call from packed K/V of each request's past rows
+    cu_p = synth.cu_from_lens(past)
+    kp = synth.normal_bf16(rng, (int(cu_p[-1]), w.H, w.D))
+    vp = synth.normal_bf16(rng, (int(cu_p[-1]), w.H, w.D))
+    slots = rng.permutation(w.S)[: w.B].astype(np.int32)
+    pk = torch.zeros((1, w.S, w.H, w.n_cap, w.D), dtype=torch.uint8, device="cuda")
+    pv = torch.zeros_like(pk)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    to16 = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).cuda()
+    to32 = lambda a: torch.from_numpy(np.ascontiguousarray(a, dtype=np.int32)).cuda()
+    ub.kvpool_write(pk, pv, 0, to16(kp), to16(vp), to32(cu_p), to32(past), to32(slots), w.n, dev_status=status,
+                    pool_scales=scales)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    hk = np.zeros((1, w.S, w.H, w.n_cap, w.D), np.uint8)
+    hv = hk.copy()
+    oracle.pool_write_e4m3(hk, hv, 0, kp, vp, cu_p, past, slots, *scales)
+    assert pk.cpu().numpy().tobytes() == hk.tobytes()
+    assert pv.cpu().numpy().tobytes() == hv.tobytes()
+    for kk in (16, 1000):
+        cand = np.full(w.B, kk, np.int32)
+        d = synth.make_decode(w.seed + 200 + kk, past, cand, w.H, w.D, n_slots=w.S)
+        d.slot_ids = slots
+        dd = DevDecode(d)
+        out = ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, 0, kk, out_fp32=True,
+                                  dev_status=status, pool_scales=scales)
+        torch.cuda.synchronize()
+        assert int(status.item()) == 0
+        rows = sample_rows(d.cu_seqlens, np.zeros_like(past), 600, 5) if kk > 16 else None
+        ref = oracle.decode_e4m3(d.q, d.k, d.v, d.cu_seqlens, d.slot_ids, d.past_lens, hk, hv, 0, *scales) \
+            if rows is None else None
+        if rows is None:
+            parity(out.cpu().numpy(), ref, "E4M3 decode R32 k%d" % kk)
+        else:
+            refs = oracle.decode(d.q, d.k, d.v, d.cu_seqlens, d.slot_ids, d.past_lens,
+                                 oracle.e4m3_dequant_bf16(hk, scales[0]), oracle.e4m3_dequant_bf16(hv, scales[1]),
+                                 0, tokens=rows)
+            parity(out[torch.from_numpy(rows).cuda()].cpu().numpy(), refs, "E4M3 decode R32 k%d" % kk)
+
+
 def test_ragged_mixed_batch_prefill_then_decode(ub):
     """256 users, n ~ U{32..4096}, k ~ U{50..2000}, H=8, D=128: prefill + pool write, then decode."""
     w, batch, _ = build("ragged_B256")
