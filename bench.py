@@ -600,7 +600,7 @@ def run_sweep(device, peaks, iters=10, warm=3):
     scales = (0.0625, 0.0625)
     pk8 = (randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed).float() / scales[0]).to(torch.float8_e4m3fn)
     pv8 = (randn((w.L, w.S, w.H, w.n_cap, w.D), w.seed + 1).float() / scales[1]).to(torch.float8_e4m3fn)
-    for kk in (16,):
+    for kk in (16, 64, 256):
         cand = np.full(w.B, kk, np.int32)
         Tc = int(cand.sum())
         cu = torch.from_numpy(synth.cu_from_lens(cand)).to(device)
@@ -616,9 +616,20 @@ def run_sweep(device, peaks, iters=10, warm=3):
                                     pool_scales=scales)
 
         ms = timed(fn8) / w.L
+        # the library's routing: the small-k kernel reads the codes in place up to 32 candidate
+        # columns at D=64 (64 at D=128); beyond, a dequantized copy feeds the bfloat16 kernels
+        if kk <= 32 or (w.D == 128 and kk <= 64):
+            kernel = "decode_smallk_kernel<%d,%d,e4m3>" % (w.D, 16 if kk <= 16 else 32 if kk <= 32 else 64)
+            path = "E4M3 codes expanded to bfloat16 in shared memory by the small-k kernel"
+        elif kk <= 64:
+            kernel = "kvpool_dequant_kernel + decode_smallk_kernel<%d,64>" % w.D
+            path = "E4M3 rows dequantized into the workspace, then the bfloat16 small-k kernel"
+        else:
+            kernel = "kvpool_dequant_kernel + attn_fwd_kernel<%d,decode>" % w.D
+            path = "E4M3 rows dequantized into the workspace, then the bfloat16 engine"
         e = roof_entry(ms, decode_flops(past, cand, w.H, w.D), decode_bytes(past, cand, w.H, w.D, 2, 1), peaks,
-                       "kvpool_dequant_kernel + decode_smallk_kernel<%d,16>" % w.D)
-        e["path"] = "E4M3 rows dequantized into the workspace, then the bfloat16 kernel"
+                       kernel)
+        e["path"] = path
         e["candidates_per_s"] = float(Tc) / (ms * 1e-3)
         out["decode_R32_n2048_D64_k%d_e4m3" % kk] = e
         del qkv, outs, ws

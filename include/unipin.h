@@ -203,7 +203,7 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
  *                  H must be a multiple of the pool's key/value heads)
  *   out            [T_c, H, D], fp32 if out_fp32 else bf16
  *   max_k          host int >= every k_r (sizes the grid and picks the kernel: with
- *                  max_k * G <= 128 (G = H / pool->H) and D in {64, 128} the pool keys
+ *                  max_k * G <= 64 (G = H / pool->H) and D in {64, 128} the pool keys
  *                  are the tensor-core M dimension, the G query heads of a key/value
  *                  head share one sweep of its history, and a request's key range is
  *                  swept by several thread blocks, the bandwidth-bound case;
@@ -214,7 +214,7 @@ int unipin_kvpool_write(const unipin_kvpool* pool, int layer, const void* k, con
  *                  unipin_rank_decode_workspace_size(...) bytes the pool sweep of
  *                  each request is also split over several thread blocks (split-n)
  *                  when that helps, and the splits are merged (in the kernel for
- *                  max_k <= 128, by a second kernel otherwise; the per-request
+ *                  max_k * G <= 64, by a second kernel otherwise; the per-request
  *                  arrival counters the in-kernel merge uses are zeroed by the call
  *                  on `stream`).  The result is the same either way up to fp32
  *                  rounding.  Two calls that overlap in time must not share a
@@ -233,11 +233,19 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
  * current device and a 148-SM B200. */
 size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_k, int total_cand, int n_cap);
 
-/* The same for a given pool of either dtype.  Over an UNIPIN_POOL_E4M3 pool the
- * call first dequantizes rows 0..n_r-1 of each request's slot (layer `layer`)
- * into bfloat16 in the workspace and then decodes from there, so it needs a
- * workspace: this size plus R * pool->H * pool->n_cap * pool->D * 4 bytes and a
- * little more; with less, it returns UNIPIN_ERR_INVALID_ARG. */
+/* The same for a given pool of either dtype.  Over an UNIPIN_POOL_E4M3 pool:
+ *   - with max_k * G <= 64 and D = 128, or max_k * G <= 32 and D = 64, and with
+ *     k_scale and v_scale both bfloat16 values in [2^-117, 2^118], the
+ *     small-candidate kernel reads the codes itself (each key tile lands in
+ *     shared memory as codes and is expanded there to the bfloat16 values the
+ *     tensor cores take), so the workspace is as for a bfloat16 pool: optional,
+ *     only for split-n;
+ *   - otherwise the call first dequantizes rows 0..n_r-1 of each request's slot
+ *     (layer `layer`) into bfloat16 in the workspace and then decodes from
+ *     there, so it needs a workspace: this size, which includes
+ *     R * pool->H * pool->n_cap * pool->D * 4 bytes for those rows; with less it
+ *     returns UNIPIN_ERR_INVALID_ARG.
+ * Either way code c stands for bfloat16(value(c) * scale). */
 size_t unipin_rank_decode_pool_workspace_size(const unipin_kvpool* pool, int R, int H, int max_k, int total_cand);
 
 /*
@@ -255,8 +263,10 @@ size_t unipin_rank_decode_pool_workspace_size(const unipin_kvpool* pool, int R, 
  *     total_cand, pool->n_cap) exceeds that size, the pool sweep is not split
  *     (as unipin_rank_decode_attn does with a small workspace): the same
  *     result, computed more slowly.
- *   - An UNIPIN_POOL_E4M3 pool is not taken (UNIPIN_ERR_UNSUPPORTED): its
- *     dequantized rows do not fit a fixed array.
+ *   - An UNIPIN_POOL_E4M3 pool is taken only where the small-candidate kernel
+ *     reads its codes (see unipin_rank_decode_pool_workspace_size); otherwise
+ *     the call returns UNIPIN_ERR_UNSUPPORTED: the dequantized rows it would
+ *     decode from do not fit a fixed array.
  *   - The first call on a device looks up the array's device address; make
  *     that first call before any stream capture.
  *   - Every call shares the one array and it keeps the last call's contents

@@ -57,6 +57,7 @@
 // left waiting at such a barrier.
 #pragma once
 
+#include "kvpool_sm100.cuh"
 #include "sm100_ptx.cuh"
 #include "tmem_wide.cuh"
 #include "unipin.h"
@@ -78,7 +79,10 @@ constexpr float kSkRescaleLog2 = 8.0f;
 __host__ __device__ constexpr int sk_pad_n(int k) { return k <= 16 ? 16 : k <= 32 ? 32 : 64; }
 __host__ __device__ constexpr int sk_tmem_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
 
-template <int D, int N>
+// kE4M3: the pool holds E4M3 codes; TMA brings each key tile's K and V codes
+// into a staging ring and the producer warp expands them into the bfloat16
+// ring stages the MMAs read (the same layout TMA writes for a bfloat16 pool).
+template <int D, int N, bool kE4M3 = false>
 struct SkCfg {
     static_assert(D == 64 || D == 128, "small-k decode: head dim 64 or 128");
     static_assert(N == 16 || N == 32 || N == 64, "small-k decode: padded candidate count");
@@ -101,37 +105,52 @@ struct SkCfg {
     static constexpr int kColO = kSBufs * N;
     static constexpr int kTmemCols = sk_tmem_cols(kSBufs * N + 2 * D);
     static_assert(kTmemCols <= 512, "small-k decode: TMEM columns");
-    static constexpr int kCtasPerSm = (D == 64 && kTmemCols <= 256) ? 2 : 1;
     // Scratch floats: softmax red[4][N], mref[N], corr[N]; hand-off hand_m[2][N],
     // hand_l[2][N]; epilogue coef_b[N], wts[kSkMaxSplit][N], last[4].
     static constexpr int kScratchFloats = 4 * N + 2 * N + 4 * N + N + kSkMaxSplit * N + 4;
     static constexpr int kScratchBytes = (kScratchFloats * 4 + 1023) / 1024 * 1024;
     static constexpr int kBarBytes = 1024;
+    static constexpr int kTile8 = kSkKeys * D;             // E4M3 codes of one K or V tile (rows of D bytes)
+    static constexpr int kStage8 = 2 * kTile8;             // K codes, then V codes
     // two blocks per SM: 2 x (113 KB + the 1 KB the runtime keeps per block) = 228 KB
-    static constexpr int kBudget = kCtasPerSm == 2 ? 113 * 1024 : 226 * 1024;
+    static constexpr int budget_for(int ctas) { return ctas == 2 ? 113 * 1024 : 226 * 1024; }
     // Q is double-buffered (the next item's Q loads during this item); P is
     // double-buffered (the softmax writes P_{i+1} while P.V of tile i runs)
     // unless a single buffer buys one more ring stage, since the ring depth sets
     // the bytes in flight.
-    static constexpr int fixed_bytes(int qbufs, int pbufs)
+    static constexpr int fixed_bytes(int pbufs, int stages8)
     {
-        return qbufs * kQBytes + pbufs * kPBytes + kScratchBytes + kBarBytes;
+        return 2 * kQBytes + pbufs * kPBytes + kScratchBytes + kBarBytes + stages8 * kStage8;
     }
-    static constexpr int stages_with(int pbufs) { return (kBudget - fixed_bytes(2, pbufs)) / kStageBytes; }
+    static constexpr int stages_for(int ctas, int pbufs, int stages8)
+    {
+        return (budget_for(ctas) - fixed_bytes(pbufs, stages8)) / kStageBytes;
+    }
+    // E4M3 staging: two stages where two bfloat16 stages still fit, else one
+    static constexpr int stages8_for(int ctas) { return !kE4M3 ? 0 : (stages_for(ctas, 1, 2) >= 2 ? 2 : 1); }
+    static constexpr int kCtasPerSm =
+        (D == 64 && kTmemCols <= 256 && stages_for(2, 1, stages8_for(2)) >= 2) ? 2 : 1;
+    static constexpr int kBudget = budget_for(kCtasPerSm);
+    static constexpr int kStages8 = stages8_for(kCtasPerSm);
     static constexpr int kQBufs = 2;
-    static constexpr int kPBufs = stages_with(1) > stages_with(2) ? 1 : 2;
-    static constexpr int kStagesFit = stages_with(kPBufs);
+    static constexpr int kPBufs = stages_for(kCtasPerSm, 1, kStages8) > stages_for(kCtasPerSm, 2, kStages8) ? 1 : 2;
+    static constexpr int kStagesFit = stages_for(kCtasPerSm, kPBufs, kStages8);
     static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
     static_assert(kStages >= 2, "small-k decode: ring depth");
     static constexpr int kOffP = 0;                                  // first: the 128-row reads overhang
     static constexpr int kOffRing = kPBufs * kPBytes;                // into the ring that follows
     static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
-    static constexpr int kOffScratch = kOffQ + kQBufs * kQBytes;
+    static constexpr int kOffStage8 = kOffQ + kQBufs * kQBytes;     // E4M3 staging ring
+    static constexpr int kOffScratch = kOffStage8 + kStages8 * kStage8;
     static constexpr int kOffBar = kOffScratch + kScratchBytes;
     static constexpr int kSmemBytes = kOffBar + kBarBytes;
     static_assert(kSmemBytes <= kBudget, "small-k decode: shared memory budget");
     static_assert(kSkMaxSplit * N * 4 <= kPBytes, "merge weights fit a P buffer");
     static_assert((kPBufs - 1) * kPBytes + kPBox + kSkKeys * 128 <= kSmemBytes, "P box reads stay in shared memory");
+};
+
+struct SkE4M3Mul {
+    uint32_t c1, c2;   // bfloat16x2 factors: the first product, then the second (c2 = 0: none)
 };
 
 struct SkParams {
@@ -158,6 +177,8 @@ struct SkParams {
     int* status;
     unsigned long long wait_limit_ns;
     unsigned poll_ns;              // back-off of the polling producer and MMA warps when nothing is ready
+    float k_scale, v_scale;        // E4M3 pool: code c stands for value(c) * scale
+    SkE4M3Mul k_mul, v_mul;        // the same scales as bfloat16 factors (see SkE4M3Mul)
 };
 
 // What every role derives identically from an item index.  An item is a
@@ -311,15 +332,146 @@ __device__ __forceinline__ void sk_store4(void* out, int out_fp32, size_t idx, f
             make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
 }
 
-template <int D, int N>
-__global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
+// Expanding E4M3 codes in shared memory.
+//
+// E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits) and bfloat16
+// (sign, 8 exponent bits with bias 127, 7 mantissa bits) differ, for the bits
+// they share, only in the exponent bias.  A code's sign moved to bit 15 and its
+// seven exponent/mantissa bits to bits 4..10 is therefore a bfloat16 of value
+// value(code) * 2^-120 - for subnormal codes too, which land on bfloat16
+// subnormals with the same factor - except the two NaN codes (0x7F, 0xFF).
+// One bfloat16 product by scale * 2^120 (or by 2^120, exact, then by scale)
+// rounds value(code) * scale once to nearest even.  Where scale is itself a
+// bfloat16 value and 2^-117 <= scale <= 2^118, that product is exact in
+// float32, so this equals bfloat16(value(code) * scale) computed with a float32
+// product, the pool's reading rule.  The host takes this kernel for an E4M3
+// pool only then.  NaN codes are detected per tile; a tile holding one is
+// expanded again by the conversion instructions, which give NaN.
+
+// Codes in bytes b_lo, b_hi of w -> bfloat16x2 of value * 2^-120 (lo half from b_lo)
+template <uint32_t kSel>
+__device__ __forceinline__ uint32_t sk_e4m3x2_raw(uint32_t w)
+{
+    const uint32_t x = __byte_perm(w, 0u, kSel);   // b_lo in byte 1, b_hi in byte 3, zero bytes between
+    return (x & 0x80008000u) | ((x >> 4) & 0x07F007F0u);
+}
+
+__device__ __forceinline__ uint32_t sk_bf16x2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Three warps (the producer and the two epilogue warps, on three different SM
+// sub-partitions: the expansion is bound by the integer pipes) expand each key
+// tile of E4M3 codes (128 rows of D bytes, as TMA lands them without swizzle)
+// into the bfloat16 tile the MMAs read: 64-element boxes of 128 rows x 128
+// bytes whose 16-byte units are swizzled by the row (unit j of row r at
+// j ^ (r & 7)), the layout a 128-byte-swizzled TMA load writes.  A lane step
+// turns 8 codes (one 8-byte read; 16 lanes read 128 contiguous bytes) into 8
+// values (one 16-byte write; 8 lanes fill one 128-byte row); expander e of the
+// three takes steps [kSteps e / 3, kSteps (e + 1) / 3) of every lane.
+constexpr int kSkExpanders = 3;
+
+template <int D>
+struct SkExpandSteps {
+    static constexpr int kSteps = kSkKeys * D / 8 / 32;   // 8-code steps per lane and tile
+    static constexpr int kPerRow = D / 8;
+    __device__ static int begin(int e) { return kSteps * e / kSkExpanders; }
+};
+
+// Step s of this lane: its codes' byte offset in the staged tile and its values'
+// byte offset in the bfloat16 tile.
+template <int D>
+__device__ __forceinline__ uint32_t sk_expand_dst(int lane, int s)
+{
+    const int u = lane + s * 32;
+    const int r = u / SkExpandSteps<D>::kPerRow;
+    const int j = u % SkExpandSteps<D>::kPerRow;   // elements 8j .. 8j+7 of row r
+    return (j >> 3) * (kSkKeys * 128) + r * 128 + (((j & 7) ^ (r & 7)) << 4);
+}
+
+// Steps [s0, s1): the codes of up to kBatch steps are read into registers
+// before any value is written (their reads are in flight together).  Returns
+// (warp-uniform) whether those codes hold a NaN code.
+template <int D, bool kTwo>
+__device__ __forceinline__ bool sk_expand_e4m3_fast(uint32_t dst, uint32_t src, SkE4M3Mul m, int lane, int s0,
+                                                    int s1)
+{
+    constexpr int kBatch = 4;
+    const uint32_t src_l = src + lane * 8;
+    uint32_t nan_bits = 0;
+#pragma unroll 1
+    for (int b = s0; b < s1; b += kBatch) {
+        uint32_t cx[kBatch], cy[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            cx[i] = 0u;
+            cy[i] = 0u;
+            if (b + i < s1)
+                asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(cx[i]), "=r"(cy[i]) : "r"(src_l + (b + i) * 256));
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+            if (b + i < s1) {
+                // bit 7 of a byte of (code & 0x7F) + 1 is set exactly for the NaN codes
+                nan_bits |= ((cx[i] & 0x7F7F7F7Fu) + 0x01010101u) | ((cy[i] & 0x7F7F7F7Fu) + 0x01010101u);
+                uint32_t o0 = sk_bf16x2_mul(sk_e4m3x2_raw<0x1404u>(cx[i]), m.c1);
+                uint32_t o1 = sk_bf16x2_mul(sk_e4m3x2_raw<0x3424u>(cx[i]), m.c1);
+                uint32_t o2 = sk_bf16x2_mul(sk_e4m3x2_raw<0x1404u>(cy[i]), m.c1);
+                uint32_t o3 = sk_bf16x2_mul(sk_e4m3x2_raw<0x3424u>(cy[i]), m.c1);
+                if constexpr (kTwo) {
+                    o0 = sk_bf16x2_mul(o0, m.c2);
+                    o1 = sk_bf16x2_mul(o1, m.c2);
+                    o2 = sk_bf16x2_mul(o2, m.c2);
+                    o3 = sk_bf16x2_mul(o3, m.c2);
+                }
+                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sk_expand_dst<D>(lane, b + i)),
+                             "r"(o0), "r"(o1), "r"(o2), "r"(o3)
+                             : "memory");
+            }
+        }
+    }
+    return __any_sync(0xffffffffu, (nan_bits & 0x80808080u) != 0);
+}
+
+// The same steps by the conversion instructions (exact for every code, NaN included).
+template <int D>
+__device__ __forceinline__ void sk_expand_e4m3_cvt(uint8_t* dst, const uint8_t* src, float scale, int lane, int s0,
+                                                   int s1)
+{
+    for (int s = s0; s < s1; ++s) {
+        const uint4 vals = bf16x8_from_e4m3(*reinterpret_cast<const uint2*>(src + (lane + s * 32) * 8), scale);
+        *reinterpret_cast<uint4*>(dst + sk_expand_dst<D>(lane, s)) = vals;
+    }
+}
+
+// Expander e's share of one tile.  Not inlined: the three expanding warps and
+// both tiles (K, V) run one copy of the code, which stays in the instruction cache.
+template <int D>
+__device__ __noinline__ void sk_expand_e4m3(uint8_t* dst, const uint8_t* src, SkE4M3Mul m, float scale, int lane,
+                                            int e)
+{
+    const int s0 = SkExpandSteps<D>::begin(e), s1 = SkExpandSteps<D>::begin(e + 1);
+    const bool has_nan = m.c2 != 0u ? sk_expand_e4m3_fast<D, true>(smem_u32(dst), smem_u32(src), m, lane, s0, s1)
+                                    : sk_expand_e4m3_fast<D, false>(smem_u32(dst), smem_u32(src), m, lane, s0, s1);
+    if (has_nan) {
+        __syncwarp();
+        sk_expand_e4m3_cvt<D>(dst, src, scale, lane, s0, s1);
+    }
+}
+
+template <int D, int N, bool kE4M3>
+__global__ void __launch_bounds__(kSkThreads, SkCfg<D, N, kE4M3>::kCtasPerSm)
     decode_smallk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const SkParams p)
 {
-    using C = SkCfg<D, N>;
+    using C = SkCfg<D, N, kE4M3>;
     constexpr int NS = C::kStages;
     constexpr int NP = C::kPBufs;
     constexpr int NQ = C::kQBufs;
+    constexpr int NS8 = C::kStages8;
     extern __shared__ __align__(1024) uint8_t smem[];
 
     const int warp = threadIdx.x / 32;
@@ -357,7 +509,11 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
     uint64_t* k_empty = k_full + NS;       // [NS] its S MMA finished
     uint64_t* v_full = k_empty + NS;       // [NS] V tile landed
     uint64_t* v_empty = v_full + NS;       // [NS] its P.V finished
-    uint64_t* item_full = v_empty + NS;    // [kSkItemSlots]
+    uint64_t* k8_full = v_empty + NS;      // [NS8] E4M3 pool: K codes landed in staging
+    uint64_t* v8_full = k8_full + NS8;     // [NS8] V codes landed
+    uint64_t* k8_empty = v8_full + NS8;    // [NS8] K codes read by the three expanders
+    uint64_t* v8_empty = k8_empty + NS8;   // [NS8] V codes read
+    uint64_t* item_full = v8_empty + NS8;  // [kSkItemSlots]
     uint64_t* item_empty = item_full + kSkItemSlots;
     volatile long long* item_ring = reinterpret_cast<volatile long long*>(item_empty + kSkItemSlots);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_empty + 2 * kSkItemSlots);
@@ -381,10 +537,17 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         mbar_init(egrp, kSkEpiWarps);
         mbar_init(bar_drain, 1);
         for (int s = 0; s < NS; ++s) {
-            mbar_init(k_full + s, 1);
+            // an E4M3 pool's tiles are written by the three expanders, a bfloat16 pool's by one TMA load
+            mbar_init(k_full + s, kE4M3 ? kSkExpanders : 1);
             mbar_init(k_empty + s, 1);
-            mbar_init(v_full + s, 1);
+            mbar_init(v_full + s, kE4M3 ? kSkExpanders : 1);
             mbar_init(v_empty + s, 1);
+        }
+        for (int s = 0; s < NS8; ++s) {
+            mbar_init(k8_full + s, 1);
+            mbar_init(v8_full + s, 1);
+            mbar_init(k8_empty + s, kSkExpanders);
+            mbar_init(v8_empty + s, kSkExpanders);
         }
         for (int s = 0; s < kSkItemSlots; ++s) {
             mbar_init(item_full + s, 1);
@@ -405,10 +568,10 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
 
     WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns, (int)UNIPIN_ERR_DEVICE_TIMEOUT};
     int n_items = 0;
-    // Consumers: the next item (warp-uniform)
-    auto pop_item = [&](bool& ok, long long& g) -> bool {
+    // Consumers: the next item (warp-uniform), waiting with `wait`
+    auto pop_item_w = [&](bool& ok, long long& g, auto&& wait) -> bool {
         const int si = n_items % kSkItemSlots;
-        ok = __all_sync(0xffffffffu, mbar_wait(item_full + si, (n_items / kSkItemSlots) & 1, ctl));
+        ok = wait(item_full + si, (uint32_t)((n_items / kSkItemSlots) & 1));
         if (!ok) return false;
         g = item_ring[si];
         __syncwarp();
@@ -416,7 +579,50 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         ++n_items;
         return g >= 0;
     };
+    auto pop_item = [&](bool& ok, long long& g) -> bool {
+        return pop_item_w(ok, g, [&](uint64_t* bar, uint32_t ph) {
+            return __all_sync(0xffffffffu, mbar_wait(bar, ph, ctl));
+        });
+    };
     const bool leader = lane == 0;
+    // E4M3 pool: expander e's share of the next K tile and of the next V tile
+    // whose codes have landed and whose bfloat16 ring slot is free (warp-uniform;
+    // kx / vx count the tiles this warp has expanded).  True if it did any.
+    auto expand_step = [&](int e, int& kx, int& vx) -> bool {
+        bool prog = false;
+        if constexpr (kE4M3) {
+            uint8_t* stage8 = smem + C::kOffStage8;
+            const int ks8 = kx % NS8, kst = kx % NS;
+            if (__all_sync(0xffffffffu, mbar_test_wait(k8_full + ks8, (kx / NS8) & 1) &&
+                                            (kx < NS || mbar_test_wait(k_empty + kst, ((kx / NS) - 1) & 1)))) {
+                sk_expand_e4m3<D>(ring + kst * C::kStageBytes + C::kTileKV, stage8 + ks8 * C::kStage8, p.k_mul,
+                                  p.k_scale, lane, e);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(k_full + kst);
+                    mbar_arrive(k8_empty + ks8);
+                }
+                ++kx;
+                prog = true;
+            }
+            const int vs8 = vx % NS8, vst = vx % NS;
+            if (__all_sync(0xffffffffu, mbar_test_wait(v8_full + vs8, (vx / NS8) & 1) &&
+                                            (vx < NS || mbar_test_wait(v_empty + vst, ((vx / NS) - 1) & 1)))) {
+                sk_expand_e4m3<D>(ring + vst * C::kStageBytes, stage8 + vs8 * C::kStage8 + C::kTile8, p.v_mul,
+                                  p.v_scale, lane, e);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(v_full + vst);
+                    mbar_arrive(v8_empty + vs8);
+                }
+                ++vx;
+                prog = true;
+            }
+        }
+        return prog;
+    };
 
     if (warp == kSkProducerWarp) {
         // ------------------------------------------------------------ producer
@@ -438,6 +644,8 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         int nk = 0, nv = 0;      // items with tiles started by the K stream / finished by the V stream
         int ik = 0, iv = 0;      // tile within the current K / V item
         int nq = 0;
+        int kc8 = 0, vc8 = 0;    // E4M3 pool: K / V tiles this warp has expanded its share of
+        uint8_t* stage8 = smem + C::kOffStage8;
         bool k_has = false, q_done = false, claim_done = false, ok = true;
         int q_h = 0, q_tok = 0;
         long long g_next = (long long)blockIdx.x << 20;   // the block's pieces, in order
@@ -493,15 +701,27 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                     }
                 }
                 const int st = uk % NS;
-                if (q_done &&
-                    (uk < NS || __all_sync(0xffffffffu, mbar_test_wait(k_empty + st, ((uk / NS) - 1) & 1)))) {
+                bool k_go;
+                if constexpr (kE4M3)   // the staging slot's last codes were read by all expanders
+                    k_go = q_done && (uk < NS8 || __all_sync(0xffffffffu, mbar_test_wait(k8_empty + uk % NS8,
+                                                                                         ((uk / NS8) - 1) & 1)));
+                else
+                    k_go = q_done &&
+                           (uk < NS || __all_sync(0xffffffffu, mbar_test_wait(k_empty + st, ((uk / NS) - 1) & 1)));
+                if (k_go) {
                     const PItem& it = items[(nk - 1) % 4];
                     const int start = sk_tile_start(it.t_begin + ik, it.nt_all, it.npast);
                     if (leader) {
-                        uint8_t* dst = ring + st * C::kStageBytes + C::kTileKV;
-                        mbar_arrive_expect_tx(k_full + st, C::kTileKV);
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_3d(dst + c * C::kAtom, &tm_k, k_full + st, c * 64, start, it.plane);
+                        if constexpr (kE4M3) {
+                            const int s8 = uk % NS8;
+                            mbar_arrive_expect_tx(k8_full + s8, C::kTile8);
+                            tma_load_3d(stage8 + s8 * C::kStage8, &tm_k, k8_full + s8, 0, start, it.plane);
+                        } else {
+                            uint8_t* dst = ring + st * C::kStageBytes + C::kTileKV;
+                            mbar_arrive_expect_tx(k_full + st, C::kTileKV);
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_3d(dst + c * C::kAtom, &tm_k, k_full + st, c * 64, start, it.plane);
+                        }
                     }
                     ++uk;
                     prog = true;
@@ -511,14 +731,27 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             // 3. V stream: V_u once K_u has been issued
             if (uv < uk) {
                 const int st = uv % NS;
-                if (uv < NS || __all_sync(0xffffffffu, mbar_test_wait(v_empty + st, ((uv / NS) - 1) & 1))) {
+                bool v_go;
+                if constexpr (kE4M3)
+                    v_go = uv < NS8 ||
+                           __all_sync(0xffffffffu, mbar_test_wait(v8_empty + uv % NS8, ((uv / NS8) - 1) & 1));
+                else
+                    v_go = uv < NS || __all_sync(0xffffffffu, mbar_test_wait(v_empty + st, ((uv / NS) - 1) & 1));
+                if (v_go) {
                     const PItem& it = items[nv % 4];
                     const int start = sk_tile_start(it.t_begin + iv, it.nt_all, it.npast);
                     if (leader) {
-                        uint8_t* dst = ring + st * C::kStageBytes;
-                        mbar_arrive_expect_tx(v_full + st, C::kTileKV);
-                        for (int c = 0; c < C::kChunks; ++c)
-                            tma_load_3d(dst + c * C::kAtom, &tm_v, v_full + st, c * 64, start, it.plane);
+                        if constexpr (kE4M3) {
+                            const int s8 = uv % NS8;
+                            mbar_arrive_expect_tx(v8_full + s8, C::kTile8);
+                            tma_load_3d(stage8 + s8 * C::kStage8 + C::kTile8, &tm_v, v8_full + s8, 0, start,
+                                        it.plane);
+                        } else {
+                            uint8_t* dst = ring + st * C::kStageBytes;
+                            mbar_arrive_expect_tx(v_full + st, C::kTileKV);
+                            for (int c = 0; c < C::kChunks; ++c)
+                                tma_load_3d(dst + c * C::kAtom, &tm_v, v_full + st, c * 64, start, it.plane);
+                        }
                     }
                     ++uv;
                     prog = true;
@@ -528,7 +761,11 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
                     }
                 }
             }
-            if (claim_done && !k_has && uv == uk) break;   // every copy issued
+            // 4. this warp's share of the code expansion (expander 0)
+            if constexpr (kE4M3)
+                if ((kc8 < uk || vc8 < uv) && expand_step(0, kc8, vc8)) prog = true;
+            // every copy issued (and, for codes, expanded)
+            if (claim_done && !k_has && uv == uk && (!kE4M3 || (kc8 == uk && vc8 == uv))) break;
             if (prog) {
                 t_prog = global_timer_ns();
             } else {
@@ -559,10 +796,17 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         }
         if (leader) {
             // Let every copy this warp started land before the block exits.
-            for (int v = (uk > NS ? uk - NS : 0); v < uk; ++v)
-                mbar_wait_drain(k_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
-            for (int v = (uv > NS ? uv - NS : 0); v < uv; ++v)
-                mbar_wait_drain(v_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
+            if constexpr (kE4M3) {
+                for (int v = (uk > NS8 ? uk - NS8 : 0); v < uk; ++v)
+                    mbar_wait_drain(k8_full + v % NS8, (v / NS8) & 1, p.wait_limit_ns);
+                for (int v = (uv > NS8 ? uv - NS8 : 0); v < uv; ++v)
+                    mbar_wait_drain(v8_full + v % NS8, (v / NS8) & 1, p.wait_limit_ns);
+            } else {
+                for (int v = (uk > NS ? uk - NS : 0); v < uk; ++v)
+                    mbar_wait_drain(k_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
+                for (int v = (uv > NS ? uv - NS : 0); v < uv; ++v)
+                    mbar_wait_drain(v_full + v % NS, (v / NS) & 1, p.wait_limit_ns);
+            }
             for (int v = (nq > NQ ? nq - NQ : 0); v < nq; ++v)
                 mbar_wait_drain(bar_q + v % NQ, (v / NQ) & 1, p.wait_limit_ns);
             for (int v = (n_items > kSkItemSlots ? n_items - kSkItemSlots : 0); v < n_items; ++v)
@@ -895,7 +1139,35 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
         uint32_t negrp = 0;
         bool ok = true;
         long long g;
-        while (pop_item(ok, g)) {
+        // Over an E4M3 pool these two warps are expanders 1 and 2: every wait whose end
+        // may need their share of the expansion keeps expanding meanwhile.
+        int ekx = 0, evx = 0;
+        auto epi_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            if constexpr (!kE4M3) {
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, ctl));
+            } else {
+                uint64_t t0 = global_timer_ns();
+                for (uint32_t it = 1;; ++it) {
+                    if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
+                    if (expand_step(1 + warp, ekx, evx)) {
+                        t0 = global_timer_ns();
+                        continue;
+                    }
+                    __nanosleep(p.poll_ns);
+                    if ((it & 15) == 0) {
+                        const bool aborted = *abort_flag != 0;
+                        if (__any_sync(0xffffffffu, aborted || global_timer_ns() - t0 > p.wait_limit_ns)) {
+                            if (lane == 0 && !aborted) {
+                                *abort_flag = 1;
+                                report(p.status, (int)UNIPIN_ERR_DEVICE_TIMEOUT);
+                            }
+                            return false;
+                        }
+                    }
+                }
+            }
+        };
+        while (pop_item_w(ok, g, epi_wait)) {
             const SkWork w = sk_make_work<N>(p, g);
             // Column t = (candidate t / G, query head w.h * G + t % G): its output row, its own
             // key/value row, and its own score (log2 units), taken while the item's keys stream.
@@ -905,7 +1177,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             const float ss_own = mine ? p.sl2 * sk_dot_bf16<D>(p.q + qrow * D, p.k_self + kvrow * D) : -INFINITY;
             // the item's statistics
             const int hb = nh & 1;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(h_full + hb, (nh >> 1) & 1, ctl)))) break;
+            if (!(ok = epi_wait(h_full + hb, (nh >> 1) & 1))) break;
             const float l_c = t < N ? hand_l[hb * N + t] : 0.f;
             const float m_c = t < N ? hand_m[hb * N + t] : -INFINITY;
             __syncwarp();
@@ -916,7 +1188,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N>::kCtasPerSm)
             const int ob = nb & 1;
             const bool have_o = w.nt > 0 && warp * 32 < N;
             if (w.nt > 0) {
-                if (!(ok = __all_sync(0xffffffffu, mbar_wait(o_full + ob, (nb >> 1) & 1, ctl)))) break;
+                if (!(ok = epi_wait(o_full + ob, (nb >> 1) & 1))) break;
                 tc_fence_after_sync();
             }
             // final coefficients (one split): out = (a O + b v_self) / (a l + b)

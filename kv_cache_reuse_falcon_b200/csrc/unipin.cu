@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "unipin.h"
@@ -84,25 +85,26 @@ int set_attn_attrs()
     return set_attn_attr(attn_fwd_kernel<D, true>, AttnCfg<D, true>::kSmemBytes);
 }
 
-template <int D, int N>
+template <int D, int N, bool kE4M3>
 int set_sk_attr()
 {
-    if (cudaFuncSetAttribute(decode_smallk_kernel<D, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SkCfg<D, N>::kSmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(decode_smallk_kernel<D, N, kE4M3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SkCfg<D, N, kE4M3>::kSmemBytes) != cudaSuccess)
         return UNIPIN_ERR_CUDA;
     // All of the SM's on-chip memory as shared memory, so that two blocks fit where they are meant to.
-    if (cudaFuncSetAttribute(decode_smallk_kernel<D, N>, cudaFuncAttributePreferredSharedMemoryCarveout,
+    if (cudaFuncSetAttribute(decode_smallk_kernel<D, N, kE4M3>, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
         return UNIPIN_ERR_CUDA;
     return UNIPIN_OK;
 }
 
-template <int D>
+template <int D, bool kE4M3>
 int set_sk_attrs()
 {
-    int rc = set_sk_attr<D, 16>();
-    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 32>();
-    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 64>();
+    int rc = set_sk_attr<D, 16, kE4M3>();
+    if (rc == UNIPIN_OK) rc = set_sk_attr<D, 32, kE4M3>();
+    if constexpr (!(kE4M3 && D == 64))   // that pool is decoded from a dequantized copy (sk_takes_pool)
+        if (rc == UNIPIN_OK) rc = set_sk_attr<D, 64, kE4M3>();
     return rc;
 }
 
@@ -133,8 +135,10 @@ int ensure_device()
     int rc = set_attn_attrs<32>();
     if (rc == UNIPIN_OK) rc = set_attn_attrs<64>();
     if (rc == UNIPIN_OK) rc = set_attn_attrs<128>();
-    if (rc == UNIPIN_OK) rc = set_sk_attrs<64>();
-    if (rc == UNIPIN_OK) rc = set_sk_attrs<128>();
+    if (rc == UNIPIN_OK) rc = set_sk_attrs<64, false>();
+    if (rc == UNIPIN_OK) rc = set_sk_attrs<128, false>();
+    if (rc == UNIPIN_OK) rc = set_sk_attrs<64, true>();
+    if (rc == UNIPIN_OK) rc = set_sk_attrs<128, true>();
     if (rc == UNIPIN_OK &&
         (cudaFuncSetAttribute(bwd_kv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               BwCfg<32>::kSmemBytes) != cudaSuccess ||
@@ -171,6 +175,21 @@ int make_token_map(CUtensorMap* m, const void* base, int T, int H, int D, int ro
     const uint32_t box_d = D >= 64 ? 64u : (uint32_t)D;
     return make_map(m, base, (uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)D * 2, (uint64_t)H * D * 2, box_d,
                     (uint32_t)heads, (uint32_t)rows, D);
+}
+
+// E4M3 pool [L, S, H, n_cap, D] of one-byte codes viewed as (D, n_cap, L*S*H):
+// boxes of `rows` whole rows (D bytes each) of one plane, unswizzled.
+int make_pool_map_e4m3(CUtensorMap* m, const void* base, const unipin_kvpool* pool, int rows)
+{
+    const int D = pool->D;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)pool->n_cap, (cuuint64_t)pool->L * pool->S * pool->H};
+    cuuint64_t strides[2] = {(cuuint64_t)D, (cuuint64_t)pool->n_cap * D};
+    cuuint32_t box[3] = {(cuuint32_t)D, (cuuint32_t)rows, 1};
+    cuuint32_t elem[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, elem,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 
 // Pool [L, S, H, n_cap, D] viewed as (D, n_cap, L*S*H): boxes of `rows` history rows of one plane.
@@ -308,20 +327,62 @@ bool use_small_k(int D, int max_k, int G)
     return (D == 64 || D == 128) && max_k >= 1 && (long long)max_k * G <= kSmallKMax && kSmallKMax % G == 0;
 }
 
-int sk_ctas_per_sm(int D, int N)
+// An E4M3 scale as the bfloat16x2 factors of the small-k kernel's code
+// expansion (see SkE4M3Mul); false where the scale is not a bfloat16 value in
+// [2^-117, 2^118], the range in which the expansion equals the pool's reading rule.
+bool sk_e4m3_mul(float scale, SkE4M3Mul* m)
+{
+    uint32_t bits;
+    std::memcpy(&bits, &scale, sizeof bits);
+    if ((bits & 0xFFFFu) != 0 || !(scale >= std::ldexp(1.f, -117) && scale <= std::ldexp(1.f, 118))) return false;
+    auto bf16x2 = [](float x) {
+        uint32_t b;
+        std::memcpy(&b, &x, sizeof b);
+        return (b >> 16) | (b & 0xFFFF0000u);
+    };
+    if (scale < 128.f) {   // scale * 2^120 stays below 2^127
+        m->c1 = bf16x2(std::ldexp(scale, 120));
+        m->c2 = 0;
+    } else {
+        m->c1 = bf16x2(std::ldexp(1.f, 120));
+        m->c2 = bf16x2(scale);
+    }
+    return true;
+}
+
+// Whether the small-k kernel decodes this pool in place: a bfloat16 pool, or an
+// E4M3 pool whose two scales the kernel's expansion takes, except at D = 64 with
+// 64 candidate columns, where the code staging leaves room for one block per SM
+// only and decoding a dequantized copy measured faster.
+bool sk_takes_pool(const unipin_kvpool* pool, int D, int max_k, int G)
+{
+    if (!use_small_k(D, max_k, G)) return false;
+    if (pool->dtype != UNIPIN_POOL_E4M3) return true;
+    if (D == 64 && sk_pad_n(max_k * G) == 64) return false;
+    SkE4M3Mul m;
+    return sk_e4m3_mul(pool->k_scale, &m) && sk_e4m3_mul(pool->v_scale, &m);
+}
+
+template <bool kE4M3>
+int sk_ctas_per_sm_t(int D, int N)
 {
     if (D == 64) {
         switch (N) {
-        case 16: return SkCfg<64, 16>::kCtasPerSm;
-        case 32: return SkCfg<64, 32>::kCtasPerSm;
-        default: return SkCfg<64, 64>::kCtasPerSm;
+        case 16: return SkCfg<64, 16, kE4M3>::kCtasPerSm;
+        case 32: return SkCfg<64, 32, kE4M3>::kCtasPerSm;
+        default: return SkCfg<64, 64, kE4M3>::kCtasPerSm;
         }
     }
     switch (N) {
-    case 16: return SkCfg<128, 16>::kCtasPerSm;
-    case 32: return SkCfg<128, 32>::kCtasPerSm;
-    default: return SkCfg<128, 64>::kCtasPerSm;
+    case 16: return SkCfg<128, 16, kE4M3>::kCtasPerSm;
+    case 32: return SkCfg<128, 32, kE4M3>::kCtasPerSm;
+    default: return SkCfg<128, 64, kE4M3>::kCtasPerSm;
     }
+}
+
+int sk_ctas_per_sm(int D, int N, bool e4m3)
+{
+    return e4m3 ? sk_ctas_per_sm_t<true>(D, N) : sk_ctas_per_sm_t<false>(D, N);
 }
 
 // Tile ranges (blocks) per resident block slot (1: one wave of blocks);
@@ -361,11 +422,11 @@ struct SkPlan {
 // least tpp / (kSkMaxSplit - 1) tiles).  With split = false one range per
 // pair (no partials).  The candidate columns of a pair are (candidate, query
 // head of the group): max_k * G of them.
-SkPlan sk_plan(int R, int H_kv, int G, int D, int max_k, int n_cap, int sms, bool split = true)
+SkPlan sk_plan(int R, int H_kv, int G, int D, int max_k, int n_cap, int sms, bool e4m3, bool split = true)
 {
     SkPlan pl;
     pl.N = sk_pad_n(max_k * G);
-    pl.blocks_per_sm = sk_ctas_per_sm(D, pl.N);
+    pl.blocks_per_sm = sk_ctas_per_sm(D, pl.N, e4m3);
     pl.tpp = (n_cap + kSkKeys - 1) / kSkKeys;
     const long long pairs = (long long)R * H_kv;
     pl.total_tiles = pairs * pl.tpp;
@@ -399,22 +460,26 @@ size_t sk_workspace_bytes(const SkPlan& pl, int R, int H, int D, int total_cand)
     return kSchedBytes + sk_counter_bytes(R, H) + rows * (size_t)D * sizeof(float) + rows * 2 * sizeof(float);
 }
 
-template <int D, int N>
+template <int D, int N, bool kE4M3>
 int launch_sk_kernel(unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const SkParams& p, cudaStream_t s)
 {
-    decode_smallk_kernel<D, N><<<grid, kSkThreads, SkCfg<D, N>::kSmemBytes, s>>>(tq, tk, tv, p);
+    decode_smallk_kernel<D, N, kE4M3><<<grid, kSkThreads, SkCfg<D, N, kE4M3>::kSmemBytes, s>>>(tq, tk, tv, p);
     return cudaGetLastError() == cudaSuccess ? UNIPIN_OK : UNIPIN_ERR_CUDA;
 }
 
-template <int D>
+template <int D, bool kE4M3>
 int launch_sk_d(int N, unsigned grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                 const SkParams& p, cudaStream_t s)
 {
     switch (N) {
-    case 16: return launch_sk_kernel<D, 16>(grid, tq, tk, tv, p, s);
-    case 32: return launch_sk_kernel<D, 32>(grid, tq, tk, tv, p, s);
-    default: return launch_sk_kernel<D, 64>(grid, tq, tk, tv, p, s);
+    case 16: return launch_sk_kernel<D, 16, kE4M3>(grid, tq, tk, tv, p, s);
+    case 32: return launch_sk_kernel<D, 32, kE4M3>(grid, tq, tk, tv, p, s);
+    default:
+        if constexpr (kE4M3 && D == 64)
+            return UNIPIN_ERR_UNSUPPORTED;   // not routed here (sk_takes_pool)
+        else
+            return launch_sk_kernel<D, 64, kE4M3>(grid, tq, tk, tv, p, s);
     }
 }
 
@@ -424,17 +489,23 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
                         void* workspace, size_t workspace_bytes, int* dev_status, cudaStream_t s)
 {
     const int G = H / pool->H;
-    SkPlan pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms());
+    const bool e4m3 = pool->dtype == UNIPIN_POOL_E4M3;
+    SkPlan pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms(), e4m3);
     if (pl.nsplit > 1 && (!workspace || workspace_bytes < sk_workspace_bytes(pl, R, H, D, total_cand)))
-        pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms(), false);
+        pl = sk_plan(R, pool->H, G, D, max_k, pool->n_cap, current_sms(), e4m3, false);
     if (pl.nsplit > 1 && cudaMemsetAsync(workspace, 0, kSchedBytes + sk_counter_bytes(R, H), s) != cudaSuccess)
         return UNIPIN_ERR_CUDA;
     CUtensorMap tq, tk, tv;
     int rc;
     // the N candidate columns: N / G tokens x the G query heads of one key/value head
     if ((rc = make_token_map(&tq, q_c, total_cand, H, D, pl.N / G, G)) != UNIPIN_OK) return rc;
-    if ((rc = make_pool_map(&tk, pool->k, pool, kSkKeys)) != UNIPIN_OK) return rc;
-    if ((rc = make_pool_map(&tv, pool->v, pool, kSkKeys)) != UNIPIN_OK) return rc;
+    if (e4m3) {
+        if ((rc = make_pool_map_e4m3(&tk, pool->k, pool, kSkKeys)) != UNIPIN_OK) return rc;
+        if ((rc = make_pool_map_e4m3(&tv, pool->v, pool, kSkKeys)) != UNIPIN_OK) return rc;
+    } else {
+        if ((rc = make_pool_map(&tk, pool->k, pool, kSkKeys)) != UNIPIN_OK) return rc;
+        if ((rc = make_pool_map(&tv, pool->v, pool, kSkKeys)) != UNIPIN_OK) return rc;
+    }
 
     SkParams p = {};
     p.q = static_cast<const __nv_bfloat16*>(q_c);
@@ -460,6 +531,10 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
     p.status = dev_status;
     p.wait_limit_ns = wait_limit_ns();
     p.poll_ns = sk_poll_ns();
+    p.k_scale = pool->k_scale;
+    p.v_scale = pool->v_scale;
+    if (e4m3 && (!sk_e4m3_mul(pool->k_scale, &p.k_mul) || !sk_e4m3_mul(pool->v_scale, &p.v_mul)))
+        return UNIPIN_ERR_INVALID_ARG;
     if (pl.nsplit > 1) {
         char* ws = static_cast<char*>(workspace);
         p.pair_cnt = reinterpret_cast<unsigned*>(ws + kSchedBytes);
@@ -467,7 +542,11 @@ int rank_decode_small_k(const void* q_c, const void* k_c, const void* v_c, void*
         p.part_ml = p.part_o + (size_t)pl.nsplit * total_cand * H * D;
     }
     const unsigned grid = (unsigned)pl.nranges;
-    return D == 64 ? launch_sk_d<64>(pl.N, grid, tq, tk, tv, p, s) : launch_sk_d<128>(pl.N, grid, tq, tk, tv, p, s);
+    if (e4m3)
+        return D == 64 ? launch_sk_d<64, true>(pl.N, grid, tq, tk, tv, p, s)
+                       : launch_sk_d<128, true>(pl.N, grid, tq, tk, tv, p, s);
+    return D == 64 ? launch_sk_d<64, false>(pl.N, grid, tq, tk, tv, p, s)
+                   : launch_sk_d<128, false>(pl.N, grid, tq, tk, tv, p, s);
 }
 
 __global__ void bounded_wait_selftest_kernel(int* status, unsigned long long limit_ns)
@@ -688,7 +767,7 @@ size_t unipin_rank_decode_workspace_size(int R, int H, int H_kv, int D, int max_
     const int sms = current_sms() > kNumSmsHint ? current_sms() : kNumSmsHint;
     const int G = H / H_kv;
     if (use_small_k(D, max_k, G))
-        return sk_workspace_bytes(sk_plan(R, H_kv, G, D, max_k, n_cap, sms), R, H, D, total_cand);
+        return sk_workspace_bytes(sk_plan(R, H_kv, G, D, max_k, n_cap, sms, false), R, H, D, total_cand);
     return decode_workspace_bytes(decode_nsplit(R, H, D, max_k, n_cap, sms), total_cand, H, D);
 }
 
@@ -697,6 +776,14 @@ size_t unipin_rank_decode_pool_workspace_size(const unipin_kvpool* pool, int R, 
     if (!pool || pool->H < 1 || H < 1 || H % pool->H != 0) return 0;
     const size_t base = unipin_rank_decode_workspace_size(R, H, pool->H, pool->D, max_k, total_cand, pool->n_cap);
     if (base == 0 || pool->dtype != UNIPIN_POOL_E4M3) return base;
+    const int G = H / pool->H;
+    if (sk_takes_pool(pool, pool->D, max_k, G)) {
+        // the small-k kernel reads the codes itself: only its partials
+        const int sms = current_sms() > kNumSmsHint ? current_sms() : kNumSmsHint;
+        const size_t e = sk_workspace_bytes(sk_plan(R, pool->H, G, pool->D, max_k, pool->n_cap, sms, true), R, H,
+                                            pool->D, total_cand);
+        return e > base ? e : base;
+    }
     return dequant_slab_bytes(pool, R) + base;
 }
 
@@ -717,7 +804,7 @@ int unipin_rank_decode_attn(const void* q_c, const void* k_c, const void* v_c, v
     rc = ensure_device();
     if (rc != UNIPIN_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (pool->dtype == UNIPIN_POOL_E4M3)
+    if (pool->dtype == UNIPIN_POOL_E4M3 && !sk_takes_pool(pool, D, max_k, H / pool->H))
         return rank_decode_e4m3(q_c, k_c, v_c, out, out_fp32, cu_seqlens_c, slot_ids, past_lens, R, H, D, max_k,
                                 total_cand, scale, pool, layer, workspace, workspace_bytes, dev_status, s);
     if (use_small_k(D, max_k, H / pool->H))
@@ -797,7 +884,9 @@ int unipin_rank_decode_attn_noalloc(const void* q_c, const void* k_c, const void
     if (!supported_d(D)) return UNIPIN_ERR_UNSUPPORTED;
     if (R == 0 || total_cand == 0 || max_k == 0) return UNIPIN_OK;
     if (pool->H < 1 || H % pool->H != 0) return UNIPIN_ERR_INVALID_ARG;
-    if (pool->dtype == UNIPIN_POOL_E4M3) return UNIPIN_ERR_UNSUPPORTED;
+    // an E4M3 pool needs a dequantised copy unless the small-k kernel reads its codes
+    if (pool->dtype == UNIPIN_POOL_E4M3 && !sk_takes_pool(pool, D, max_k, H / pool->H))
+        return UNIPIN_ERR_UNSUPPORTED;
     // A shape whose split-n partials would not fit the array runs unsplit (the
     // regular call's fallback for a small workspace): slower, same result.
     void* scratch = nullptr;

@@ -101,14 +101,25 @@ def test_e4m3_pool_host_rules_need_no_device(lib):
     f8 = Pool(16, 16, 1, 4, 2, 512, 64, 1, 0.5, 0.25)
     base = g(3, 4, 2, 64, 16, 48, 512)
     assert ws(ctypes.byref(bf), 3, 4, 16, 48) == base
-    # the dequantized rows: 3 requests x 2 heads x 512 rows x 64 bf16, for K and V, and the slot ids
-    assert ws(ctypes.byref(f8), 3, 4, 16, 48) >= base + 2 * 3 * 2 * 512 * 64 * 2 + 3 * 4
+    # 16 candidates x 2 query heads per kv head = 32 columns: the small-k kernel reads the codes, no copy
+    assert base <= ws(ctypes.byref(f8), 3, 4, 16, 48) < base + 2 * 3 * 2 * 512 * 64
+    # 32 candidates x 2 = 64 columns at D=64: the dequantized copy (measured faster there)
+    base32 = g(3, 4, 2, 64, 32, 96, 512)
+    assert ws(ctypes.byref(f8), 3, 4, 32, 96) >= base32 + 2 * 3 * 2 * 512 * 64 * 2 + 3 * 4
+    # ... when both scales are bfloat16 values in its range; otherwise the dequantized copy
+    for ks, vs in ((0.3, 0.25), (0.5, 2.0 ** -120), (0.5, 2.0 ** 119)):
+        odd = Pool(16, 16, 1, 4, 2, 512, 64, 1, ks, vs)
+        assert ws(ctypes.byref(odd), 3, 4, 16, 48) >= base + 2 * 3 * 2 * 512 * 64 * 2 + 3 * 4
+    # 100 candidates: the engine reads dequantized rows, 3 requests x 2 heads x 512 rows x 64 bf16 for
+    # K and V, and the slot ids
+    base100 = g(3, 4, 2, 64, 100, 300, 512)
+    assert ws(ctypes.byref(f8), 3, 4, 100, 300) >= base100 + 2 * 3 * 2 * 512 * 64 * 2 + 3 * 4
     assert ws(ctypes.byref(f8), 3, 3, 16, 48) == 0          # query heads not a multiple of the pool's
     na = lib.unipin_rank_decode_attn_noalloc
     na.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, ctypes.c_float, P, I, P, P]
     na.restype = I
-    assert na(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), 3, 4, 64, 16, 48, 0.1, ctypes.byref(f8), 0,
-              None, None) == -2                              # E4M3 pools are not taken by the no-alloc call
+    assert na(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), 3, 4, 64, 100, 300, 0.1, ctypes.byref(f8), 0,
+              None, None) == -2                              # nor by the no-alloc call beyond 64 columns
     dec = lib.unipin_rank_decode_attn
     dec.argtypes = [P, P, P, P, I, P, P, P, I, I, I, I, I, ctypes.c_float, P, I, P, SZ, P, P]
     dec.restype = I

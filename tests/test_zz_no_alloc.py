@@ -14,7 +14,7 @@ import pytest
 import torch
 
 from kv_cache_reuse_falcon_b200 import synth
-from tests.gpu_helpers import DevDecode, fill_pool_rows, nan_pool, parity
+from tests.gpu_helpers import DevDecode, fill_pool_rows, nan_pool, parity, to_dev_bf16, to_dev_i32
 
 pytestmark = pytest.mark.gpu
 
@@ -81,10 +81,42 @@ def test_noalloc_decode_runs_unsplit_beyond_its_array(ub):
     parity(out.cpu().numpy(), ref.cpu().numpy().astype(np.float64), "no-alloc decode, unsplit")
 
 
-def test_noalloc_decode_refuses_an_e4m3_pool(ub):
-    """Its dequantized rows would not fit a fixed array: UNSUPPORTED before any launch."""
+def test_noalloc_decode_refuses_an_e4m3_pool_beyond_small_k(ub):
+    """With more than 64 candidate columns the engine would need the pool's dequantized rows,
+    which do not fit a fixed array: UNSUPPORTED before any launch."""
     P = ctypes.c_void_p
     pool = ub.KVPool(16, 16, 1, 1, 4, 512, 64, ub.POOL_E4M3, 1.0, 1.0)   # never dereferenced
     rc = ub.LIB.unipin_rank_decode_attn_noalloc(P(16), P(16), P(16), P(16), 1, P(16), P(16), P(16), 3, 4, 64,
-                                                16, 48, 0.1, ctypes.byref(pool), 0, None, None)
+                                                100, 300, 0.1, ctypes.byref(pool), 0, None, None)
     assert rc == -2
+
+
+def test_noalloc_decode_over_an_e4m3_pool_with_small_k(ub):
+    """The small-candidate kernel reads E4M3 codes itself, so the no-alloc call takes such a pool;
+    checked against the oracle's decode over the dequantized rows."""
+    import oracle
+    H, Hkv, D, S, n_cap, layer = 8, 2, 64, 6, 2048, 0
+    past, cand = [2048, 517, 0, 1300], [8, 3, 5, 1]     # 8 x 4 query heads per kv head = 32 columns
+    scales = (0.046875, 0.0205078125)     # bfloat16 values: the kernel expands the codes itself
+    rng = np.random.Generator(np.random.PCG64(7200))
+    cu = synth.cu_from_lens(np.array(cand))
+    Tc = int(cu[-1])
+    qc = synth.normal_bf16(rng, (Tc, H, D))
+    kc = synth.normal_bf16(rng, (Tc, Hkv, D))
+    vc = synth.normal_bf16(rng, (Tc, Hkv, D))
+    slots = np.array([5, 0, 3, 2], np.int32)
+    hk = np.full((1, S, Hkv, n_cap, D), 0x7F, np.uint8)
+    hv = hk.copy()
+    for s_, n in zip(slots, past):
+        hk[0, s_, :, :n] = oracle.e4m3_encode((rng.normal(0, 1, (Hkv, n, D)) / scales[0]).astype(np.float32))
+        hv[0, s_, :, :n] = oracle.e4m3_encode((rng.normal(0, 1, (Hkv, n, D)) / scales[1]).astype(np.float32))
+    pl = np.array(past, np.int32)
+    out = torch.full((Tc, H, D), float("nan"), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ub.rank_decode_attn_noalloc(to_dev_bf16(qc), to_dev_bf16(kc), to_dev_bf16(vc), to_dev_i32(cu), to_dev_i32(slots),
+                                to_dev_i32(pl), torch.from_numpy(hk).cuda(), torch.from_numpy(hv).cuda(), layer,
+                                max(cand), out, out_fp32=True, dev_status=status, pool_scales=scales)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, ub.status_string(int(status.item()))
+    ref = oracle.decode_e4m3(qc, kc, vc, cu, slots, pl, hk, hv, 0, *scales)
+    parity(out.cpu().numpy(), ref, "no-alloc E4M3 decode")
