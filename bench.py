@@ -678,7 +678,18 @@ def run_decode_only(args, rank, world, device, dist):
     pl = torch.from_numpy(past).to(device)
     sl = torch.from_numpy(slots).to(device)
     out = [torch.empty((Tc, H, D), dtype=torch.bfloat16, device=device) for _ in range(L)]
-    ws_bytes = ub.rank_decode_workspace_size(w.B, H, D, kk, Tc, n_cap)
+    pool_scales = None
+    if args.pool == "e4m3":
+        # the same rows as E4M3 codes of x / 2^-6 (a bfloat16-valued scale: N(0,1) rows up to 7)
+        pool_scales = (2.0 ** -6, 2.0 ** -6)
+        k8 = torch.empty((L, S, H, n_cap, D), dtype=torch.float8_e4m3fn, device=device)
+        v8 = torch.empty_like(k8)
+        for layer in range(L):
+            k8[layer] = (pool_k[layer].float() / pool_scales[0]).to(torch.float8_e4m3fn)
+            v8[layer] = (pool_v[layer].float() / pool_scales[1]).to(torch.float8_e4m3fn)
+        pool_k, pool_v = k8, v8
+        torch.cuda.empty_cache()
+    ws_bytes = ub.rank_decode_pool_workspace_size(pool_k, pool_v, w.B, H, kk, Tc, pool_scales=pool_scales)
     ws = torch.empty(ws_bytes // 4 + 4, dtype=torch.float32, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     stream = torch.cuda.current_stream(device)
@@ -686,7 +697,8 @@ def run_decode_only(args, rank, world, device, dist):
     def layers(s):
         for layer in range(L):
             ub.rank_decode_attn(qs[layer], kc[layer], vc[layer], cu, sl, pl, pool_k, pool_v, layer, kk,
-                                out=out[layer], out_fp32=False, workspace=ws, dev_status=status, stream=s)
+                                out=out[layer], out_fp32=False, workspace=ws, dev_status=status, stream=s,
+                                pool_scales=pool_scales)
 
     graph = None
 
@@ -729,7 +741,7 @@ def run_decode_only(args, rank, world, device, dist):
     ms_step = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
     peaks = load_peaks()
     flops = decode_flops(past, cand, H, D) * L
-    nbytes = decode_bytes(past, cand, H, D, 2) * L
+    nbytes = decode_bytes(past, cand, H, D, 2, 1 if pool_scales else 2) * L
     tflops = flops / (ms_step * 1e-3) / 1e12
     gbs = nbytes / (ms_step * 1e-3) / 1e9
     t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
@@ -739,9 +751,17 @@ def run_decode_only(args, rank, world, device, dist):
              "frac": gbs / peaks["hbm_gbs"]} if bound == "hbm" else
             {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
              "frac": tflops / peaks["bf16_tflops"]})
-    # the library sends requests of at most 64 candidates (one query head per kv head) to the small-k kernel
-    kernel = ("decode_smallk_kernel<%d,%d>" % (D, 16 if kk <= 16 else 32 if kk <= 32 else 64)
-              if kk <= 64 and D in (64, 128) else "attn_fwd_kernel<%d,decode>" % D)
+    # the library sends requests of at most 64 candidates (one query head per kv head) to the small-k
+    # kernel; over an E4M3 pool it reads the codes in place up to 32 columns at D=64 (64 at D=128)
+    n_pad = 16 if kk <= 16 else 32 if kk <= 32 else 64
+    if kk <= 64 and D in (64, 128):
+        kernel = "decode_smallk_kernel<%d,%d>" % (D, n_pad)
+        if pool_scales and (n_pad <= 32 or D == 128):
+            kernel = "decode_smallk_kernel<%d,%d,e4m3>" % (D, n_pad)
+        elif pool_scales:
+            kernel = "kvpool_dequant_kernel + " + kernel
+    else:
+        kernel = ("kvpool_dequant_kernel + " if pool_scales else "") + "attn_fwd_kernel<%d,decode>" % D
     roof.update({"kernel": kernel, "traffic": None, "peak_source": "%s (burst for tensor)" % peaks["source"]})
     return {
         "metric": METRIC, "value": float(cand.sum()) * L / (ms_step * 1e-3), "unit": "candidate tokens/s",
@@ -750,12 +770,15 @@ def run_decode_only(args, rank, world, device, dist):
         "config": {"workload": w.name if args.layers <= 0 else "%s[layers=%d]" % (w.name, L),
                    "requests": w.B, "k": kk, "n": w.n, "H": H, "D": D,
                    "pool": [L, S, H, n_cap, D], "layers_per_step": L, "split_n": ws_bytes > 256,
+                   "pool_dtype": args.pool, "pool_scales": pool_scales,
                    "cuda_graph": bool(args.graph),
                    "l2": "pool slots read per step exceed L2 (no flush)"},
         "phases": {"decode_tflops": tflops, "decode_gbs": gbs, "decode_frac_hbm": gbs / peaks["hbm_gbs"],
                    "decode_frac_tensor": tflops / peaks["bf16_tflops"],
                    "roof_time_ms": 1e3 * max(t_hbm, t_tc)},
-        "roofline": roof, "gpu_launches": args.steps * L * (2 if (ws_bytes > 256 and kk > 128) else 1),
+        "roofline": roof,
+        "gpu_launches": args.steps * L * ((2 if (ws_bytes > 256 and kk > 128) else 1) +
+                                          (1 if kernel.startswith("kvpool_dequant") else 0)),
         "clocks": clk,
     }
 
@@ -886,6 +909,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--users", type=int, default=0, help="smaller case: this many users (profiling)")
     ap.add_argument("--k", type=int, default=0, help="decode workloads: candidates per request")
+    ap.add_argument("--pool", default="bf16", choices=["bf16", "e4m3"],
+                    help="decode workloads: the pool's element type (E4M3 codes with scale 2^-6)")
     ap.add_argument("--layers", type=int, default=0,
                     help="decode workloads: pool layers and layer calls per step (smaller case)")
     ap.add_argument("--no-sweep", action="store_true", help="headline workload only (no per-config sweep)")

@@ -137,6 +137,7 @@ struct SkCfg {
     static constexpr int kStagesFit = stages_for(kCtasPerSm, kPBufs, kStages8);
     static constexpr int kStages = kStagesFit > 6 ? 6 : kStagesFit;
     static_assert(kStages >= 2, "small-k decode: ring depth");
+    static_assert(kPBufs <= 2, "small-k decode: the barrier layout holds two P buffers");
     static constexpr int kOffP = 0;                                  // first: the 128-row reads overhang
     static constexpr int kOffRing = kPBufs * kPBytes;                // into the ring that follows
     static constexpr int kOffQ = kOffRing + kStages * kStageBytes;
