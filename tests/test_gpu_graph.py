@@ -113,3 +113,51 @@ def test_layered_rank_decode_replays_from_a_graph(ub, split):
         d = ds[layer]
         ref = oracle.decode(d.q, d.k, d.v, d.cu_seqlens, d.slot_ids, d.past_lens, hk, hv, 0)
         parity(outs[layer].cpu().numpy(), ref, "decode layer %d from a graph" % layer)
+
+
+@pytest.mark.parametrize("scales", [(0.03125, 0.0546875), (0.0625, 0.03)])
+def test_e4m3_rank_decode_replays_from_a_graph(ub, scales):
+    """Two layers of an E4M3 pool: with bfloat16-valued scales the small-k kernel reads the codes in
+    place; with 0.03 the call dequantizes into its workspace first (a second kernel in the graph)."""
+    R, H, D, S, L, n_cap = 4, 2, 64, 8, 2, 1024
+    past, cand = [1000, 257, 1024, 0], [16, 3, 9, 1]
+    rng = np.random.Generator(np.random.PCG64(7300))
+    d0 = synth.make_decode(7300, past, cand, H, D, n_slots=S, rng=rng)
+    hk = np.full((L, S, H, n_cap, D), 0x7F, np.uint8)
+    hv = hk.copy()
+    for layer in range(L):
+        for s_, n in zip(d0.slot_ids, past):
+            hk[layer, s_, :, :n] = oracle.e4m3_encode((rng.normal(0, 1, (H, n, D)) / scales[0]).astype(np.float32))
+            hv[layer, s_, :, :n] = oracle.e4m3_encode((rng.normal(0, 1, (H, n, D)) / scales[1]).astype(np.float32))
+    pk = torch.from_numpy(hk).cuda().view(torch.float8_e4m3fn)
+    pv = torch.from_numpy(hv).cuda().view(torch.float8_e4m3fn)
+    dd = DevDecode(d0)
+    max_k, Tc = max(cand), int(d0.cu_seqlens[-1])
+    nbytes = ub.rank_decode_pool_workspace_size(pk, pv, R, H, max_k, Tc, pool_scales=scales)
+    ws = torch.empty(nbytes // 4 + 4, dtype=torch.float32, device="cuda")
+    outs = [torch.empty(dd.q.shape, dtype=torch.float32, device="cuda") for _ in range(L)]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def step():
+        for layer in range(L):
+            ub.rank_decode_attn(dd.q, dd.k, dd.v, dd.cu, dd.slots, dd.past, pk, pv, layer, max_k, out=outs[layer],
+                                out_fp32=True, workspace=ws, dev_status=status, stream=torch.cuda.current_stream(),
+                                pool_scales=scales)
+
+    step()
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    for o in outs:
+        o.zero_()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0, ub.status_string(int(status.item()))
+    for layer in range(L):
+        assert torch.equal(outs[layer], eager[layer]), layer
+        ref = oracle.decode_e4m3(d0.q, d0.k, d0.v, d0.cu_seqlens, d0.slot_ids, d0.past_lens,
+                                 hk[layer:layer + 1], hv[layer:layer + 1], 0, *scales)
+        parity(outs[layer].cpu().numpy(), ref, "E4M3 decode layer %d from a graph" % layer)
