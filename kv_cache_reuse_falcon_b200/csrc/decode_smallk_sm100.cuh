@@ -51,6 +51,10 @@
 // to the epilogue through a two-entry buffer, so the key stream of the next
 // item runs while the epilogue of the last one waits on its stores and its
 // arrival counter: the ring does not stall at item boundaries.
+// Over an E4M3 pool (kE4M3) TMA brings each tile's codes into a staging ring
+// instead, and the producer and the two epilogue warps each expand a third of
+// every K and V tile into the ring's bfloat16 layout (see sk_expand_e4m3); the
+// epilogue warps expand while they wait.
 // Every mbarrier wait is bounded (see sm100_ptx.cuh); a block that gives up
 // reports UNIPIN_ERR_DEVICE_TIMEOUT and exits cleanly.  The softmax warps
 // leave their loop only together, on a named-barrier reduction, so none is
