@@ -9,10 +9,12 @@
 // candidates:
 //
 //   S^T = K Q^T   M = 128 keys, N = k padded to 16/32/64, K = D
-//   O  += P V     M = 128 candidate rows (rows past the padded count are
-//                 discarded), N = D, K = 128 keys; P (bf16) is staged through
-//                 shared memory in the 128-byte-swizzled K-major layout of a
-//                 query tile, V is read MN-major as the prefill reads it
+//   O  += P V     M = 64 candidate rows for N <= 32, else 128 (rows past the
+//                 padded count are discarded), N = D, K = 128 keys; P (bf16) is
+//                 staged through shared memory in the 128-byte-swizzled K-major
+//                 layout of a query tile, V is read MN-major as the prefill
+//                 reads it.  An M = 64 product reads half the P operand; its
+//                 row r sits in TMEM lane 32 (r / 16) + r % 16
 //
 // Softmax thread t owns key t of a tile (TMEM lane t): it loads that key's N
 // scores, and the per-candidate statistics are reductions over threads.  The
@@ -102,6 +104,8 @@ struct SkCfg {
     // whatever follows in shared memory and give discarded output rows.
     static constexpr int kPBox = N * 128;
     static constexpr int kPBytes = 2 * kPBox;
+    static constexpr bool kPv64 = N <= 32;                 // P.V with M = 64 (rows 0..63 of P)
+    static constexpr int kPvRows = kPv64 ? 64 : 128;
     // TMEM columns: kSBufs S^T buffers of N columns from 0 (four where they fit
     // beside two O buffers in the block's share, so that S runs well ahead of
     // the softmax), then two O buffers of D columns.
@@ -151,7 +155,7 @@ struct SkCfg {
     static constexpr int kSmemBytes = kOffBar + kBarBytes;
     static_assert(kSmemBytes <= kBudget, "small-k decode: shared memory budget");
     static_assert(kSkMaxSplit * N * 4 <= kPBytes, "merge weights fit a P buffer");
-    static_assert((kPBufs - 1) * kPBytes + kPBox + kSkKeys * 128 <= kSmemBytes, "P box reads stay in shared memory");
+    static_assert((kPBufs - 1) * kPBytes + kPBox + kPvRows * 128 <= kSmemBytes, "P box reads stay in shared memory");
 };
 
 struct SkE4M3Mul {
@@ -827,7 +831,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N, kE4M3>::kCtasPerSm)
         //                    from the epilogue).  Item j accumulates in O buffer j % 2.
         constexpr int NSB = C::kSBufs;
         constexpr uint32_t idesc_qk = idesc_bf16_f32(kSkKeys, N, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(C::kPvRows, D, true, false);
         const uint32_t ring_a = smem_u32(ring);
         // K (A of S^T): K-major, 128-byte rows, 8-row groups 1024 bytes apart.
         const uint64_t dk0 = smem_desc(ring_a + C::kTileKV, 16, 1024, kLayoutSw128);
@@ -1066,8 +1070,10 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N, kE4M3>::kCtasPerSm)
                     if (i > 0) {
                         // rescale the O rows accumulated so far (after the last P.V): row c is candidate c
                         ok_w = wait_pv(gp - 1);
-                        if (ok_w && wq * 32 < N) {
-                            const float cf = corr[t < N ? t : 0];
+                        // O row r: TMEM lane r (M = 128), or lane 32 (r / 16) + r % 16 (M = 64)
+                        if (ok_w && wq * (C::kPv64 ? 16 : 32) < N) {
+                            const int orow = C::kPv64 ? (lane < 16 ? wq * 16 + lane : 0) : t;
+                            const float cf = corr[orow < N ? orow : 0];
 #pragma unroll
                             for (int c0 = 0; c0 < D; c0 += 16) {
                                 uint32_t o[16];
@@ -1137,7 +1143,9 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N, kE4M3>::kCtasPerSm)
         }
     } else {
         // ----------------------------------------------------------- epilogue
-        const int t = threadIdx.x;                               // candidate column t; O row t = TMEM lane t
+        // candidate column t: O row t is TMEM lane t (M = 128 P.V) or lane 32 (t / 16) + t % 16
+        // (M = 64: lanes 16-31 of each warp hold no row and take no column)
+        const int t = C::kPv64 ? (lane < 16 ? warp * 16 + lane : kSkEpiWarps * 32) : (int)threadIdx.x;
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const int hkv = p.H / p.G;
         int nb = 0, nh = 0;
@@ -1191,7 +1199,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N, kE4M3>::kCtasPerSm)
             if (!w.rows_ok) continue;
             // O row t, 32 columns at a time (warp-collective loads where the warp holds candidate rows)
             const int ob = nb & 1;
-            const bool have_o = w.nt > 0 && warp * 32 < N;
+            const bool have_o = w.nt > 0 && warp * (C::kPv64 ? 16 : 32) < N;
             if (w.nt > 0) {
                 if (!(ok = epi_wait(o_full + ob, (nb >> 1) & 1))) break;
                 tc_fence_after_sync();
@@ -1305,7 +1313,7 @@ __global__ void __launch_bounds__(kSkThreads, SkCfg<D, N, kE4M3>::kCtasPerSm)
                     int cc[4];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        const int q = base + u * kEt + t;
+                        const int q = base + u * kEt + (int)threadIdx.x;
                         const bool act = q < total;
                         cc[u] = act ? q / kQ : -1;
                         const int c = act ? cc[u] : 0;
