@@ -73,7 +73,7 @@ def pool_write_bytes(past, H, D):
 _PREFILL_TRAFFIC_PER_TOKEN = {
     # kernel_source_key() of csrc/attn_sm100.cuh, H, D: bytes per token (reads + writes,
     # the writes including the fused store of the past K/V into the pool)
-    ("aa4830eb8ccb19ef", 8, 128): (432.141056e6 + 292.076544e6) / 70236,
+    ("1b9929abd9486744", 8, 128): (432.074752e6 + 292.394496e6) / 70236,
 }
 
 
