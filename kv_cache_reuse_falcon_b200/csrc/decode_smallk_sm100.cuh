@@ -22,8 +22,8 @@
 // exceed it by more than 2^8 (one vote per tile among the four softmax warps;
 // the exact column maxima are computed only then), so the common tile costs
 // N scalings, N exponentials, N two-byte stores of P and one warp
-// reduce-scatter of the column sums.  O accumulates in TMEM with lane =
-// candidate, so the epilogue thread of candidate c reads its own row.
+// reduce-scatter of the column sums.  O accumulates in TMEM with one lane per
+// candidate row, so the epilogue thread of candidate c reads its own row.
 //
 // Work: the 128-key tiles of all (request, key/value head) pairs, pair-major
 // (tpp tiles per pair, from the pool's capacity), are cut into one contiguous
@@ -39,9 +39,9 @@
 //
 // Warp roles (256 threads; two blocks per SM where shared memory and TMEM
 // allow):
-//   warps 0-1  epilogue: the own scores, the final O rows (TMEM lanes 0-63 =
-//              candidate rows), partials, arrival counter and merge
-//   warp 2     TMA producer: claims items, loads Q (N candidate rows), and
+//   warps 0-1  epilogue: the own scores, the final O rows (from the TMEM
+//              lanes of the candidate rows), partials, arrival counter and merge
+//   warp 2     TMA producer: walks the block's items, loads Q (N candidate rows), and
 //              drives two streams into the ring - K tiles (a slot refills as
 //              soon as its S MMA is done) and V tiles (once its P.V is done)
 //   warp 3     MMA issuer (one elected thread), owns TMEM: issues S^T as K
